@@ -1,0 +1,102 @@
+"""Planted-mistake check of the oracle pins (CPU only).
+
+Each case copies oracle/oracle.c into a temporary directory, plants one plausible
+mistake (a dropped term, a wrong sign, index or comparison, a transposed operand, a
+wrong order), compiles it, and runs the pin tests against the mutant.  Every mutant must
+make at least one pin fail; a mutant that passes every pin would mean the pins cannot
+tell that mistake from the definition.  Mistakes are planted only in the copy; the
+real oracle is untouched.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+TESTS = os.path.dirname(os.path.abspath(__file__))
+
+# Pin groups, run in a child process by name (a mutant may also crash the process, which
+# counts as rejected).
+FORMAT_PINS = "format"
+SELECT_PINS = "select"
+PRODUCT_PINS = "products"
+HALF_PINS = "half"
+
+CHILD = {
+    "half": "import test_oracle_half as H; H.test_all_half_patterns_match_numpy()",
+    "format": ("import test_oracle_format as F\n"
+               "for c in F.GOLDEN: F.test_golden_encode(c); F.test_golden_decode(c)\n"
+               "F.test_random_masks(257, 511, 0.5)\n"
+               "F.test_kept_signed_zero_and_specials_preserved()"),
+    "select": ("import test_oracle_select as S\n"
+               "[S.test_threshold_brute_force(s) for s in range(40)]\n"
+               "S.test_threshold_special_cases()\n"
+               "[S.test_topk_brute_force(s) for s in range(30)]\n"
+               "S.test_topk_ties_prefer_lower_index()"),
+    "products": ("import test_oracle_products as P\n"
+                 "[P.test_spmv_exact_rational(s) for s in range(25)]\n"
+                 "P.test_spmv_matches_numpy(65, 130, 3, 0.0)\n"
+                 "P.test_spmv_act_bits_restrict_columns(); P.test_identity_is_exact()\n"
+                 "P.test_diagonal_is_exact(); P.test_spmm_matches_numpy_and_rows()\n"
+                 "P.test_spmm_transposed_operand_would_fail()"),
+}
+
+MUTANTS = [
+    ("subnormal_exponent", "ldexp((double)fraction, -24)", "ldexp((double)fraction, -25)",
+     [HALF_PINS]),
+    ("normal_bias", "exponent - 25);", "exponent - 24);", [HALF_PINS]),
+    ("row_major_tile_order",
+     "for (int k = (int)kt * TCB_COLS; k < ((int)kt + 1) * TCB_COLS; k++)\n                for (int r = 0; r < TCB_ROWS; r++) {\n                    int n = (int)s * TCB_ROWS + r;\n                    if (!kept(",
+     "for (int r = 0; r < TCB_ROWS; r++)\n                for (int k = (int)kt * TCB_COLS; k < ((int)kt + 1) * TCB_COLS; k++) {\n                    int n = (int)s * TCB_ROWS + r;\n                    if (!kept(",
+     [FORMAT_PINS]),
+    ("no_tile_padding", "uint64_t tile_units = (j + 7) / 8;", "uint64_t tile_units = (j + 8) / 8;",
+     [FORMAT_PINS]),
+    ("bit_reversed", "word |= 1ull << r;", "word |= 1ull << (63 - r);", [FORMAT_PINS]),
+    ("section_not_aligned", "g.off_values = round_up(g.off_tileptr + 4 * (n_tiles + 1), 256);",
+     "g.off_values = round_up(g.off_tileptr + 4 * (n_tiles + 1), 16);", [FORMAT_PINS]),
+    ("threshold_le", "!(fabs(v) < t)", "!(fabs(v) <= t)", [SELECT_PINS, PRODUCT_PINS]),
+    ("zeros_kept", "return v != 0.0 && !(fabs(v) < t);", "return !(fabs(v) < t);", [SELECT_PINS]),
+    ("topk_ties_high_first", "return (p->index > q->index) - (p->index < q->index);",
+     "return (p->index < q->index) - (p->index > q->index);", [SELECT_PINS]),
+    ("topk_signed_score", "s += fabs(v);", "s += v;", [SELECT_PINS]),
+    ("spmv_act_ignored", "if (act_bits && !((act_bits[k / 32] >> (k % 32)) & 1)) continue;",
+     "", [PRODUCT_PINS]),
+    ("spmv_transposed_mask", "if (!mask[(size_t)n * ld_mask + k]) continue;",
+     "if (!mask[((size_t)n * ld_mask + k) % ((size_t)N * K)]) continue; if (k == 1) continue;",
+     [PRODUCT_PINS]),
+    ("spmm_transposed", "orc_half_to_double(X[(size_t)m * ldx + k]) *",
+     "orc_half_to_double(X[(size_t)m * ldx + (K - 1 - k)]) *", [PRODUCT_PINS]),
+    ("spmv_dropped_term", "acc += orc_half_to_double(W[(size_t)n * ldw + k]) * v;",
+     "if (k + 1 < K) acc += orc_half_to_double(W[(size_t)n * ldw + k]) * v;", [PRODUCT_PINS]),
+]
+
+
+def pins_pass(lib: str, group: str) -> bool:
+    root = os.path.dirname(TESTS)
+    path = os.pathsep.join([root, TESTS, os.environ.get("PYTHONPATH", "")])
+    env = dict(os.environ, ORACLE_LIB_OVERRIDE=lib, PYTHONPATH=path)
+    proc = subprocess.run([sys.executable, "-c", CHILD[group]], cwd=TESTS, env=env,
+                          capture_output=True, timeout=600)
+    return proc.returncode == 0
+
+
+@pytest.mark.parametrize("name,old,new,groups", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_reject_planted_mistake(tmp_path, name, old, new, groups):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    path = tmp_path / "oracle_mutant.c"
+    path.write_text(src.replace(old, new))
+    lib = tmp_path / "liboracle_mutant.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared",
+                    "-o", str(lib), str(path), "-lm"], check=True)
+    assert not all(pins_pass(str(lib), g) for g in groups), \
+        f"no pin rejects the planted mistake {name!r}"
+
+
+def test_unmutated_oracle_passes_the_same_pins():
+    lib = oracle.build()
+    for group in CHILD:
+        assert pins_pass(lib, group), group
