@@ -1,0 +1,193 @@
+/*
+ * spw.h -- C ABI of the sparse-weight SpMV / SpMM library for NVIDIA B200 (sm_100a).
+ *
+ * The library multiplies a pruned LLM linear-layer weight (fp16, moderate unstructured
+ * sparsity) by activations:
+ *   decode  (spMspV): y_b = W_masked . x~_b  for a batch of 1..16 activation vectors,
+ *                     skipping the K-columns whose activation is zero or below a threshold;
+ *   prefill (SpMM):   Y = X . W_masked^T     for M token rows, on tcgen05 tensor cores.
+ * The weight is stored once, offline, in the TCB v1 tiled column-bitmap format.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [SPDP] "Unified Static-Dynamic Pruning for Efficient LLM Inference", abstract: static
+ *          unstructured weight pruning unified with input-adaptive dynamic pruning, a
+ *          Tiled-Column-wise Bitmap Compressed (Tiled-CBC) format, a CUDA-core spMspV
+ *          decode kernel with activation skipping, a Tensor-Core SpMM prefill kernel.
+ *   [RMM]  "Reduced Matrix Multiplication" (hotelren.com article), §4.1 (score, select,
+ *          multiply on the subset, map back), §4.2 (Y[:, I] = X @ W[:, I]; FFN channel
+ *          selection), §5.1 (top-k by |activation|, ascending indices), §7.3 (one index
+ *          set shared across a block of tokens).
+ *   [3LF]  "Accelerating LLM GPU inference with moderately unstructured sparse weight
+ *          matrices", §1 (tensor cores take only 2:4 sparsity; the stored format must give
+ *          the exact product; bitmap decoding cost on CUDA cores), §2.1 (prefill [BL, H]
+ *          and decode [B, H] shapes; the pattern is precomputed and stored offline).
+ *
+ * Conventions for every call
+ *   - Device pointers are global-memory addresses on the current CUDA device.  The
+ *     caller allocates and owns every buffer; the library allocates nothing on the
+ *     decode / prefill path (spw_format_query allocates 16 bytes of scratch, offline).
+ *   - fp16 data is passed as uint16_t bit patterns (IEEE binary16).
+ *   - Matrices are row-major with a leading dimension ("ld") in elements between rows.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous on `stream` unless their comment says they synchronise.
+ *   - Arguments are validated on the host before any launch.  A bad argument returns a
+ *     status code and launches nothing.  No call aborts, traps or prints.
+ *   - Alignment: every device pointer must be 16-byte aligned (d_count and d_idx: 4).
+ *     Leading dimensions only need to cover a row, except where a call copies rows
+ *     with 16-byte bulk or tensor copies: spw_spmv's ldx and spw_spmm's ldx must be
+ *     multiples of 8 fp16 elements unless that operand has a single row.  Such copies
+ *     may read an activation row up to the next 16-byte boundary past its last
+ *     element (never across it, so never outside the row's allocation granule).
+ *
+ * The TCB v1 layout (this project's reading of Tiled-CBC; the page names the format but
+ * gives no layout).  All integers little-endian.  A strip is 64 consecutive weight rows,
+ * a tile is one strip times 64 consecutive columns; n_strips = ceil(N/64),
+ * n_ktiles = ceil(K/64), tile t = s * n_ktiles + kt.
+ *   [0, 256)      header: the spw_format struct below, then zero bytes.
+ *   off_bitmaps   uint64 bitmap[n_strips][n_ktiles*64]; bit r of bitmap[s][k] is set iff
+ *                 mask[64 s + r][k] != 0 (bits for rows >= N and columns >= K are 0).
+ *   off_tileptr   uint32 tileptr[n_strips*n_ktiles + 1]: start of tile t's values in
+ *                 16-byte units from off_values; the last entry is the total.
+ *   off_values    uint16 values: per tile, the kept weights column by column (ascending
+ *                 k), within a column by ascending row (the order of the set bits),
+ *                 fp16 bits unchanged; each tile padded with 0x0000 to 16 bytes.
+ *   Sections start at multiples of 256.  bytes_total = off_values + 16*tileptr[last].
+ *   Every other byte is zero, so a buffer is a pure function of (W, mask).
+ */
+#ifndef SPW_H
+#define SPW_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every call (0 = success). */
+typedef enum {
+    SPW_OK = 0,
+    SPW_ERR_INVALID_ARG = 1,      /* null pointer, bad size or leading dimension, bad t  */
+    SPW_ERR_ALIGNMENT = 2,        /* pointer or leading dimension breaks the 16-B rule   */
+    SPW_ERR_BUFFER_TOO_SMALL = 3, /* format buffer or workspace smaller than required    */
+    SPW_ERR_FORMAT = 4,           /* header magic/version/geometry does not match TCB v1 */
+    SPW_ERR_UNSUPPORTED = 5,      /* valid request this build does not handle            */
+    SPW_ERR_CUDA = 6,             /* a CUDA runtime call failed (launch, copy, device)   */
+    SPW_ERR_TIMEOUT = 7           /* a bounded device-side wait ran out (see below)      */
+} spw_status;
+
+/* Host copy of the TCB v1 header; byte-identical to the first 80 bytes of a buffer. */
+typedef struct {
+    uint32_t magic;          /* 0x31424354 ("TCB1")                                   */
+    uint32_t version;        /* 1                                                     */
+    uint32_t N, K;           /* weight rows (outputs) and columns (inputs)            */
+    uint32_t TN, TK;         /* 64, 64                                                */
+    uint32_t n_strips;       /* ceil(N / 64)                                          */
+    uint32_t n_ktiles;       /* ceil(K / 64)                                          */
+    uint64_t nnz;            /* kept weights                                          */
+    uint64_t bytes_total;    /* buffer length in bytes                                */
+    uint64_t off_bitmaps, off_tileptr, off_values; /* section offsets in bytes        */
+    uint32_t max_tile_units; /* largest tile, in 16-byte units                        */
+    uint32_t reserved;       /* 0                                                     */
+} spw_format;
+
+/* Text for a status code (static storage; never NULL). */
+const char* spw_status_string(int status);
+
+/* Library version: 100 * major + minor.  The TCB format version is separate (1). */
+int spw_version(void);
+
+/* Size of the TCB v1 buffer for an N x K mask (device uint8, row stride ld_mask bytes,
+ * nonzero = kept).  [SPDP] format; layout above.  Writes bytes_total and nnz (host
+ * pointers).  Synchronises `stream`.  Allocates 16 bytes of device scratch (offline).
+ * Errors: INVALID_ARG (null pointer, N or K < 1, ld_mask < K), ALIGNMENT, CUDA. */
+int spw_format_query(const uint8_t* d_mask, int N, int K, int ld_mask, uint64_t* bytes_total,
+                     uint64_t* nnz, void* stream);
+
+/* Compress a masked weight into a TCB v1 buffer ([SPDP] Tiled-CBC; [3LF] §2.1: done once,
+ * offline).  d_W: N x K fp16 bits, row stride ldw; d_mask: N x K uint8, row stride
+ * ld_mask.  Kept values are copied bit-exactly (a kept -0.0 stays 0x8000); masked-out
+ * values are ignored.  d_buf receives exactly bytes_total bytes (spw_format_query); the
+ * result is byte-identical to the oracle encoder.  When hdr_out is not NULL the header
+ * is copied back into it.  Synchronises `stream` (the size check needs the tile counts).
+ * Errors: INVALID_ARG, ALIGNMENT, BUFFER_TOO_SMALL (nothing past the header sections is
+ * written then), CUDA. */
+int spw_compress(const uint16_t* d_W, int ldw, const uint8_t* d_mask, int ld_mask, int N, int K,
+                 void* d_buf, uint64_t buf_bytes, spw_format* hdr_out, void* stream);
+
+/* Copy the header of a device TCB buffer into *hdr_out and check it (magic, version,
+ * geometry, section offsets, bytes_total <= buf_bytes).  Synchronises `stream`.
+ * Errors: INVALID_ARG, FORMAT, CUDA. */
+int spw_format_read(const void* d_buf, uint64_t buf_bytes, spw_format* hdr_out, void* stream);
+
+/* Decompress a TCB buffer into the dense masked weight W_masked (N x K fp16 bits, row
+ * stride ldw): kept positions get their stored bits, all others 0x0000.  The inverse of
+ * spw_compress ([3LF] §2.1: the stored pattern must reproduce the weight exactly).
+ * Asynchronous.  Errors: INVALID_ARG, ALIGNMENT, FORMAT, CUDA. */
+int spw_decompress(const spw_format* hdr, const void* d_buf, uint16_t* d_W_out, int ldw,
+                   void* stream);
+
+/* Threshold selection ([RMM] §4.1 step 2, §7.3).  For x (B x K fp16, row stride ldx) an
+ * entry v takes part iff v != 0 and not |v| < t (compared exactly in fp32); |v| == t and
+ * NaN take part.  Column k is active iff some row's entry takes part.  Writes the
+ * active-column bitmap d_act_bits[ceil(K/32)] (bit k%32 of word k/32; bits >= K are 0)
+ * and the number of active columns to d_count (one uint32).  1 <= B <= 16; t finite and
+ * >= 0.  Asynchronous.  Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+int spw_select_threshold(const uint16_t* d_x, int B, int K, int ldx, float t,
+                         uint32_t* d_act_bits, uint32_t* d_count, void* stream);
+
+/* Top-k selection ([RMM] §5.1).  Score of column k = sum over the B rows of |x_b[k]|,
+ * computed exactly (in units of 2^-24); a column holding Inf or NaN scores above every
+ * finite score.  The k highest-scoring columns are kept, ties going to the lower index.
+ * Writes the bitmap d_act_bits[ceil(K/32)] and, if d_idx is not NULL, the kept indices
+ * in ascending order to d_idx[k].  0 <= k <= K, 1 <= B <= 16, K <= 24576.
+ * Asynchronous.  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (K too large), CUDA. */
+int spw_select_topk(const uint16_t* d_x, int B, int K, int ldx, int k, uint32_t* d_act_bits,
+                    uint32_t* d_idx, void* stream);
+
+/* Workspace bytes spw_spmv needs for this format and batch on the current device. */
+uint64_t spw_spmv_workspace_bytes(const spw_format* hdr, int B);
+
+/* Decode spMspV ([SPDP] CUDA-core spMspV with activation skipping; [RMM] §4.2 reduced
+ * product over the reduction dimension):
+ *   y_b[n] = sum_k W[n,k] mask[n,k] x~_b[k],  b < B, n < N,
+ *   x~_b[k] = x_b[k] if k is in I, x_b[k] != 0 and not |x_b[k]| < threshold, else 0,
+ * with I = the columns set in d_act_bits, or every column when d_act_bits is NULL.
+ * Columns with no surviving entry in any row are skipped.  fp32 accumulation, one
+ * round-to-nearest-even to fp16 at the end.  x: B x K fp16 (row stride ldx); y: B x N
+ * fp16 (row stride ldy).  1 <= B <= 16; threshold finite and >= 0.
+ * Workspace: d_ws of at least spw_spmv_workspace_bytes(hdr, B) bytes.  Its first
+ * 4 * n_strips bytes are split-K arrival counters: they must be zero before the first
+ * call, and every call that completes with device status SPW_OK leaves them zero
+ * again; the rest is scratch for fp32 partial sums.  Concurrent calls must not share a
+ * workspace.  Results are deterministic (a fixed summation order).  Asynchronous.
+ * Errors: INVALID_ARG, ALIGNMENT, FORMAT, BUFFER_TOO_SMALL (workspace), CUDA; a device
+ * wait that runs out is reported by spw_last_device_status (SPW_ERR_TIMEOUT), after
+ * which y is undefined and the workspace counters must be zeroed again. */
+int spw_spmv(const spw_format* hdr, const void* d_buf, const uint16_t* d_x, int B, int ldx,
+             float threshold, const uint32_t* d_act_bits, uint16_t* d_y, int ldy, void* d_ws,
+             uint64_t ws_bytes, void* stream);
+
+/* Workspace bytes spw_spmm needs (0 in this version; d_ws may then be NULL). */
+uint64_t spw_spmm_workspace_bytes(const spw_format* hdr, int M);
+
+/* Prefill SpMM ([SPDP] Tensor-Core SpMM; [3LF] §1: tensor cores take only 2:4 sparsity,
+ * so unstructured tiles are decoded to dense in shared memory and fed to dense MMA):
+ *   Y[m,n] = sum_k X[m,k] W[n,k] mask[n,k],  m < M, n < N.
+ * X: M x K fp16 (row stride ldx); Y: M x N fp16 (row stride ldy).  tcgen05 MMA with
+ * fp32 accumulation in tensor memory, one round-to-nearest-even to fp16.  M >= 0
+ * (M == 0 does nothing).  Asynchronous.
+ * Errors: INVALID_ARG, ALIGNMENT, FORMAT, CUDA; device timeouts as for spw_spmv. */
+int spw_spmm(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int M, int ldx,
+             uint16_t* d_Y, int ldy, void* d_ws, uint64_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, then read and clear the library's device status word for the
+ * current device: *code = SPW_OK, or SPW_ERR_TIMEOUT if a bounded device wait ran out
+ * since the last read.  Errors: INVALID_ARG, CUDA. */
+int spw_last_device_status(void* stream, int* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPW_H */

@@ -1,0 +1,309 @@
+"""spmm_tiled_column_b200 -- Python binding of libspw.so, the sparse-weight SpMV/SpMM library.
+
+Argument marshalling only: every function below checks tensor dtypes/devices, allocates
+outputs with torch when the caller did not pass them, and calls the C function of the
+same name in libspw.so (see include/spw.h) on torch's current CUDA stream.  All compute
+runs in the library's CUDA kernels; there is no CPU path.  If libspw.so is missing or
+cannot be loaded, the first call raises.
+
+Tensors: fp16 weights / activations as torch.float16 (or int16/uint16 bit views), the
+mask as torch.uint8 (nonzero = kept), TCB buffers as torch.uint8, bitmaps as torch.int32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspw.so")
+
+SPW_OK = 0
+SPW_ERR_INVALID_ARG = 1
+SPW_ERR_ALIGNMENT = 2
+SPW_ERR_BUFFER_TOO_SMALL = 3
+SPW_ERR_FORMAT = 4
+SPW_ERR_UNSUPPORTED = 5
+SPW_ERR_CUDA = 6
+SPW_ERR_TIMEOUT = 7
+
+# C function name -> (argtypes, restype)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_U64 = ctypes.c_uint64
+_F = ctypes.c_float
+
+
+class spw_format(ctypes.Structure):
+    """Host copy of the TCB v1 header (same layout as the C struct)."""
+    _fields_ = [("magic", ctypes.c_uint32), ("version", ctypes.c_uint32),
+                ("N", ctypes.c_uint32), ("K", ctypes.c_uint32),
+                ("TN", ctypes.c_uint32), ("TK", ctypes.c_uint32),
+                ("n_strips", ctypes.c_uint32), ("n_ktiles", ctypes.c_uint32),
+                ("nnz", ctypes.c_uint64), ("bytes_total", ctypes.c_uint64),
+                ("off_bitmaps", ctypes.c_uint64), ("off_tileptr", ctypes.c_uint64),
+                ("off_values", ctypes.c_uint64), ("max_tile_units", ctypes.c_uint32),
+                ("reserved", ctypes.c_uint32)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+_FP = ctypes.POINTER(spw_format)
+SIGNATURES = {
+    "spw_status_string": ([_I], ctypes.c_char_p),
+    "spw_version": ([], _I),
+    "spw_format_query": ([_P, _I, _I, _I, _P, _P, _P], _I),
+    "spw_compress": ([_P, _I, _P, _I, _I, _I, _P, _U64, _FP, _P], _I),
+    "spw_format_read": ([_P, _U64, _FP, _P], _I),
+    "spw_decompress": ([_FP, _P, _P, _I, _P], _I),
+    "spw_select_threshold": ([_P, _I, _I, _I, _F, _P, _P, _P], _I),
+    "spw_select_topk": ([_P, _I, _I, _I, _I, _P, _P, _P], _I),
+    "spw_spmv_workspace_bytes": ([_FP, _I], _U64),
+    "spw_spmv": ([_FP, _P, _P, _I, _I, _F, _P, _P, _I, _P, _U64, _P], _I),
+    "spw_spmm_workspace_bytes": ([_FP, _I], _U64),
+    "spw_spmm": ([_FP, _P, _P, _I, _I, _P, _I, _P, _U64, _P], _I),
+    "spw_last_device_status": ([_P, _P], _I),
+}
+
+
+class SpwError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_string(status)}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libspw.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing; build it with "
+                               "`python -m spmm_tiled_column_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().spw_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != SPW_OK:
+        raise SpwError(fn, status)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _half(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype in (torch.int16, torch.uint16):
+        t = t.view(torch.float16)
+    if t.dtype != torch.float16:
+        raise TypeError(f"{name} must be float16 (or a 16-bit bit view), got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    return t
+
+
+def _rows(t: torch.Tensor, name: str) -> tuple[torch.Tensor, int]:
+    """2-D row-major view and its leading dimension (elements)."""
+    if t.dim() == 1:
+        t = t.unsqueeze(0)
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D tensor with unit column stride")
+    return t, max(t.stride(0), t.shape[1])
+
+
+def _hdr(h) -> spw_format:
+    if isinstance(h, spw_format):
+        return h
+    f = spw_format()
+    for k, v in dict(h).items():
+        setattr(f, k, int(v))
+    return f
+
+
+# ------------------------------------------------------------------ format
+
+def spw_format_query(mask: torch.Tensor, stream=None) -> tuple[int, int]:
+    """(bytes_total, nnz) of the TCB v1 buffer for an N x K uint8 mask."""
+    mask, ld = _rows(mask, "mask")
+    if mask.dtype != torch.uint8 or not mask.is_cuda:
+        raise TypeError("mask must be a CUDA uint8 tensor")
+    nbytes, nnz = ctypes.c_uint64(), ctypes.c_uint64()
+    _check("spw_format_query", lib().spw_format_query(
+        _ptr(mask), mask.shape[0], mask.shape[1], ld, ctypes.byref(nbytes), ctypes.byref(nnz),
+        _stream(stream)))
+    return nbytes.value, nnz.value
+
+
+def spw_compress(W: torch.Tensor, mask: torch.Tensor, buf: torch.Tensor | None = None,
+                 stream=None) -> tuple[torch.Tensor, spw_format]:
+    """Compress W * mask into a TCB v1 buffer; returns (uint8 device buffer, header)."""
+    W, ldw = _rows(_half(W, "W"), "W")
+    mask, ldm = _rows(mask, "mask")
+    N, K = W.shape
+    if tuple(mask.shape) != (N, K) or mask.dtype != torch.uint8:
+        raise ValueError("mask must be uint8 with W's shape")
+    if buf is None:
+        nbytes, _ = spw_format_query(mask, stream)
+        buf = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    hdr = spw_format()
+    _check("spw_compress", lib().spw_compress(
+        _ptr(W), ldw, _ptr(mask), ldm, N, K, _ptr(buf), buf.numel(), ctypes.byref(hdr),
+        _stream(stream)))
+    return buf, hdr
+
+
+def spw_format_read(buf: torch.Tensor, stream=None) -> spw_format:
+    hdr = spw_format()
+    _check("spw_format_read", lib().spw_format_read(_ptr(buf), buf.numel(), ctypes.byref(hdr),
+                                                    _stream(stream)))
+    return hdr
+
+
+def spw_decompress(hdr, buf: torch.Tensor, out: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """Dense masked weight (fp16, N x K) from a TCB v1 buffer."""
+    h = _hdr(hdr)
+    if out is None:
+        out = torch.empty((h.N, h.K), dtype=torch.float16, device=buf.device)
+    out2, ld = _rows(_half(out, "out"), "out")
+    _check("spw_decompress", lib().spw_decompress(ctypes.byref(h), _ptr(buf), _ptr(out2), ld,
+                                                  _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------ selection
+
+def _act_words(K: int) -> int:
+    return (K + 31) // 32
+
+
+def spw_select_threshold(x: torch.Tensor, t: float, act_bits: torch.Tensor | None = None,
+                         count: torch.Tensor | None = None, stream=None):
+    """(act_bits int32[ceil(K/32)], count int32[1]) for the threshold rule."""
+    x, ldx = _rows(_half(x, "x"), "x")
+    B, K = x.shape
+    if act_bits is None:
+        act_bits = torch.empty(_act_words(K) + 3, dtype=torch.int32, device=x.device)
+    if count is None:
+        count = torch.empty(1, dtype=torch.int32, device=x.device)
+    _check("spw_select_threshold", lib().spw_select_threshold(
+        _ptr(x), B, K, ldx, float(t), _ptr(act_bits), _ptr(count), _stream(stream)))
+    return act_bits, count
+
+
+def spw_select_topk(x: torch.Tensor, k: int, act_bits: torch.Tensor | None = None,
+                    idx: torch.Tensor | None = None, stream=None):
+    """(act_bits int32[ceil(K/32)], ascending idx int32[k]) of the top-k columns."""
+    x, ldx = _rows(_half(x, "x"), "x")
+    B, K = x.shape
+    if act_bits is None:
+        act_bits = torch.empty(_act_words(K) + 3, dtype=torch.int32, device=x.device)
+    if idx is None:
+        idx = torch.empty(max(int(k), 1), dtype=torch.int32, device=x.device)
+    _check("spw_select_topk", lib().spw_select_topk(
+        _ptr(x), B, K, ldx, int(k), _ptr(act_bits), _ptr(idx), _stream(stream)))
+    return act_bits, idx[:k]
+
+
+# ------------------------------------------------------------------ products
+
+def spw_spmv_workspace_bytes(hdr, B: int) -> int:
+    h = _hdr(hdr)
+    return int(lib().spw_spmv_workspace_bytes(ctypes.byref(h), int(B)))
+
+
+def spw_spmv(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.0,
+             act_bits: torch.Tensor | None = None, y: torch.Tensor | None = None,
+             ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decode y (B x N fp16) = W_masked . x~ with column skipping.
+
+    ws: a zero-initialised uint8 workspace of spw_spmv_workspace_bytes(hdr, B) bytes
+    (allocated here with torch.zeros when not given)."""
+    h = _hdr(hdr)
+    x2, ldx = _rows(_half(x, "x"), "x")
+    B = x2.shape[0]
+    if y is None:
+        y = torch.empty((B, h.N), dtype=torch.float16, device=x.device)
+    y2, ldy = _rows(_half(y, "y"), "y")
+    if ws is None:
+        ws = torch.zeros(max(spw_spmv_workspace_bytes(h, B), 16), dtype=torch.uint8,
+                         device=x.device)
+    _check("spw_spmv", lib().spw_spmv(
+        ctypes.byref(h), _ptr(buf), _ptr(x2), B, ldx, float(threshold), _ptr(act_bits),
+        _ptr(y2), ldy, _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def spw_spmm_workspace_bytes(hdr, M: int) -> int:
+    h = _hdr(hdr)
+    return int(lib().spw_spmm_workspace_bytes(ctypes.byref(h), int(M)))
+
+
+def spw_spmm(hdr, buf: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = None,
+             ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Prefill Y (M x N fp16) = X . W_masked^T on tcgen05 tensor cores."""
+    h = _hdr(hdr)
+    X2, ldx = _rows(_half(X, "X"), "X")
+    M = X2.shape[0]
+    if Y is None:
+        Y = torch.empty((M, h.N), dtype=torch.float16, device=X.device)
+    Y2, ldy = _rows(_half(Y, "Y"), "Y")
+    need = spw_spmm_workspace_bytes(h, M)
+    if ws is None and need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=X.device)
+    _check("spw_spmm", lib().spw_spmm(
+        ctypes.byref(h), _ptr(buf), _ptr(X2), M, ldx, _ptr(Y2), ldy, _ptr(ws),
+        0 if ws is None else ws.numel(), _stream(stream)))
+    return Y
+
+
+def spw_last_device_status(stream=None) -> int:
+    code = ctypes.c_int()
+    _check("spw_last_device_status", lib().spw_last_device_status(_stream(stream),
+                                                                  ctypes.byref(code)))
+    return code.value
+
+
+class SparseLinear:
+    """A compressed weight with its header and per-batch decode workspaces (a holder for
+    the calls above; it adds no arithmetic)."""
+
+    def __init__(self, W: torch.Tensor, mask: torch.Tensor, stream=None):
+        self.N, self.K = W.shape
+        self.buf, self.hdr = spw_compress(W, mask, stream=stream)
+        self._ws = {}
+
+    def workspace(self, B: int) -> torch.Tensor:
+        if B not in self._ws:
+            self._ws[B] = torch.zeros(max(spw_spmv_workspace_bytes(self.hdr, B), 16),
+                                      dtype=torch.uint8, device=self.buf.device)
+        return self._ws[B]
+
+    def spmv(self, x, threshold=0.0, act_bits=None, y=None, stream=None):
+        x2 = x if x.dim() == 2 else x.unsqueeze(0)
+        return spw_spmv(self.hdr, self.buf, x2, threshold, act_bits, y,
+                        self.workspace(x2.shape[0]), stream)
+
+    def spmm(self, X, Y=None, stream=None):
+        return spw_spmm(self.hdr, self.buf, X, Y, stream=stream)
+
+    def decompress(self, out=None, stream=None):
+        return spw_decompress(self.hdr, self.buf, out, stream)

@@ -1,0 +1,115 @@
+"""The C-ABI library loads and exports every symbol include/spw.h declares, and its
+host-side argument checks return status codes without touching a GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from spmm_tiled_column_b200 import build as spw_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "spw.h")
+
+
+@pytest.fixture(scope="module")
+def spw():
+    spw_build.build()
+    import spmm_tiled_column_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(spw_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("spw_compress", "spw_decompress", "spw_spmv", "spw_spmm",
+                     "spw_select_threshold", "spw_select_topk", "spw_format_query"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(spw):
+    lib = ctypes.CDLL(spw_build.LIB)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    # and the binding knows every one of them
+    assert set(declared_functions()) <= set(spw.SIGNATURES)
+
+
+def test_struct_layout_matches_header(spw):
+    assert ctypes.sizeof(spw.spw_format) == 80
+    assert spw.spw_format.max_tile_units.offset == 72
+
+
+def test_status_strings_and_version(spw):
+    L = spw.lib()
+    assert L.spw_version() == 100
+    for code in range(8):
+        assert L.spw_status_string(code).decode().startswith("SPW_")
+    assert L.spw_status_string(99).decode() == "unknown spw status"
+
+
+def valid_header(spw, N=128, K=128):
+    h = spw.spw_format()
+    h.magic, h.version, h.N, h.K, h.TN, h.TK = 0x31424354, 1, N, K, 64, 64
+    h.n_strips, h.n_ktiles = (N + 63) // 64, (K + 63) // 64
+    T = h.n_strips * h.n_ktiles
+    h.off_bitmaps = 256
+    h.off_tileptr = -(-(256 + 8 * 64 * T) // 256) * 256
+    h.off_values = -(-(h.off_tileptr + 4 * (T + 1)) // 256) * 256
+    h.bytes_total = h.off_values + 16 * T
+    h.nnz, h.max_tile_units = T * 8, 1
+    return h
+
+
+def test_host_validation_without_gpu(spw):
+    L = spw.lib()
+    h = valid_header(spw)
+    P = ctypes.c_void_p
+    good = P(0x10000)
+    odd = P(0x10008)
+    s = P(0)
+    ws_n = ctypes.c_uint64(1 << 20)
+    # spmv argument errors
+    assert L.spw_spmv(None, good, good, 1, 128, 0.0, None, good, 128, good, ws_n, s) == 1
+    assert L.spw_spmv(ctypes.byref(h), None, good, 1, 128, 0.0, None, good, 128, good, ws_n, s) == 1
+    for B in (0, 17):
+        assert L.spw_spmv(ctypes.byref(h), good, good, B, 128, 0.0, None, good, 128, good, ws_n, s) == 1
+    for t in (-1.0, float("nan"), float("inf")):
+        assert L.spw_spmv(ctypes.byref(h), good, good, 1, 128, t, None, good, 128, good, ws_n, s) == 1
+    assert L.spw_spmv(ctypes.byref(h), good, good, 2, 100, 0.0, None, good, 128, good, ws_n, s) == 1
+    assert L.spw_spmv(ctypes.byref(h), good, good, 2, 132, 0.0, None, good, 128, good, ws_n, s) == 1
+    assert L.spw_spmv(ctypes.byref(h), odd, good, 1, 128, 0.0, None, good, 128, good, ws_n, s) == 2
+    assert L.spw_spmv(ctypes.byref(h), good, good, 1, 128, 0.0, odd, good, 128, good, ws_n, s) == 2
+    # header errors
+    bad = valid_header(spw)
+    bad.magic = 0
+    assert L.spw_spmv(ctypes.byref(bad), good, good, 1, 128, 0.0, None, good, 128, good, ws_n, s) == 4
+    bad = valid_header(spw)
+    bad.off_values += 256
+    assert L.spw_decompress(ctypes.byref(bad), good, good, 128, s) == 4
+    bad = valid_header(spw)
+    bad.TN = 32
+    assert L.spw_spmm(ctypes.byref(bad), good, good, 4, 128, good, 128, None, 0, s) == 4
+    # selection
+    assert L.spw_select_threshold(None, 1, 128, 128, 0.0, good, good, s) == 1
+    assert L.spw_select_threshold(good, 1, 128, 128, -0.5, good, good, s) == 1
+    assert L.spw_select_threshold(odd, 1, 128, 128, 0.5, good, good, s) == 2
+    assert L.spw_select_topk(good, 1, 128, 128, 129, good, good, s) == 1
+    assert L.spw_select_topk(good, 1, 128, 128, -1, good, good, s) == 1
+    assert L.spw_select_topk(good, 1, 30000, 30000, 10, good, good, s) == 5
+    # format
+    n1, n2 = ctypes.c_uint64(), ctypes.c_uint64()
+    assert L.spw_format_query(good, 0, 128, 128, ctypes.byref(n1), ctypes.byref(n2), s) == 1
+    assert L.spw_format_query(good, 4, 128, 100, ctypes.byref(n1), ctypes.byref(n2), s) == 1
+    assert L.spw_spmm(ctypes.byref(h), good, good, 4, 132, good, 128, None, 0, s) == 1
+    assert L.spw_format_query(odd, 4, 128, 128, ctypes.byref(n1), ctypes.byref(n2), s) == 2
+    assert L.spw_compress(good, 128, good, 128, 128, 128, good, 100, None, s) == 3
+    assert L.spw_compress(good, 120, good, 128, 128, 128, good, 1 << 20, None, s) == 1
+    assert L.spw_format_read(good, 10, None, s) == 1
+    # device status
+    assert L.spw_last_device_status(s, None) == 1

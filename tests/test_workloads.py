@@ -38,3 +38,17 @@ def test_zero_smallest_counts_and_threshold():
 def test_shapes():
     assert workloads.LLAMA7B_LAYERS["down"] == (4096, 11008)
     assert workloads.LLAMA13B_SHAPES["gate_up"] == (13824, 5120)
+
+
+def test_magnitude_mask_ties_go_to_lower_index():
+    W = np.array([[1, -1, 2, 1, 0, -2]], dtype=np.float16)
+    np.testing.assert_array_equal(workloads.magnitude_mask(W, 0.5)[0], [1, 0, 1, 0, 0, 1])
+    np.testing.assert_array_equal(workloads.magnitude_mask(W, 0.0)[0], [1] * 6)
+    np.testing.assert_array_equal(workloads.magnitude_mask(W, 1.0)[0], [0] * 6)
+    # NaN-free magnitude order on fp16 bits matches the numeric order
+    W = workloads.weight(4, 300, "tie")
+    m = workloads.magnitude_mask(W, 0.3)
+    mag = np.abs(W.astype(np.float64))
+    for r in range(4):
+        order = sorted(range(300), key=lambda c: (-mag[r, c], c))[:300 - 90]
+        assert set(np.nonzero(m[r])[0]) == set(order)

@@ -46,18 +46,23 @@ def magnitude_mask(W: np.ndarray, sparsity: float) -> np.ndarray:
     """Per-row magnitude pruning mask (uint8, 1 = kept).
 
     In every row the K - floor(sparsity * K) entries of largest |w| are kept; ties go to
-    the lower column index.  |w| is compared on the fp16 values.
+    the lower column index.  |w| is compared on the fp16 values: the key of an entry is
+    its fp16 magnitude bits (monotone in |w|) followed by the reversed column index, so
+    keys are unique and the kept set is exactly {key >= the keep-th largest key}.
     """
-    W = np.asarray(W, dtype=np.float16)
+    W = np.ascontiguousarray(W, dtype=np.float16)
     N, K = W.shape
     drop = int(np.floor(sparsity * K + 1e-9))
     keep = K - drop
-    mag = np.abs(W.astype(np.float64))
-    # stable sort on -|w| keeps lower indices first among equal magnitudes
-    order = np.argsort(-mag, axis=1, kind="stable")
     mask = np.zeros((N, K), dtype=np.uint8)
-    rows = np.arange(N)[:, None]
-    mask[rows, order[:, :keep]] = 1
+    if keep == 0:
+        return mask
+    mag = (W.view(np.uint16) & np.uint16(0x7FFF)).astype(np.int64)
+    rev = (K - 1 - np.arange(K, dtype=np.int64))[None, :]
+    for r0 in range(0, N, 1024):   # row blocks bound the temporary memory
+        key = (mag[r0:r0 + 1024] << 20) | rev
+        kth = np.partition(key, K - keep, axis=1)[:, K - keep]
+        mask[r0:r0 + 1024] = key >= kth[:, None]
     return mask
 
 
