@@ -176,7 +176,7 @@ uint64_t spw_spmm_workspace_bytes(const spw_format* hdr, int M);
  *   Y[m,n] = sum_k X[m,k] W[n,k] mask[n,k],  m < M, n < N.
  * X: M x K fp16 (row stride ldx); Y: M x N fp16 (row stride ldy).  tcgen05 MMA with
  * fp32 accumulation in tensor memory, one round-to-nearest-even to fp16.  M >= 0
- * (M == 0 does nothing).  Asynchronous.
+ * (M == 0 does nothing and then X and Y may be NULL).  Asynchronous.
  * Errors: INVALID_ARG, ALIGNMENT, FORMAT, CUDA; device timeouts as for spw_spmv. */
 int spw_spmm(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int M, int ldx,
              uint16_t* d_Y, int ldy, void* d_ws, uint64_t ws_bytes, void* stream);

@@ -370,21 +370,30 @@ int env_int(const char* name, int dflt, int lo, int hi) {
 int make_plan(const spw_format* h, int B, Plan* pl) {
     const int sms = device_sm_count();
     if (sms <= 0) return SPW_ERR_CUDA;
-    pl->warps = env_int("SPW_SPMV_WARPS", kDefaultWarpsPerCta, 1, kMaxWarpsPerCta);
-    pl->ctas_per_sm = env_int("SPW_SPMV_CTAS_PER_SM", kDefaultCtasPerSm, 1, 8);
     const long long T = (long long)h->n_strips * h->n_ktiles;
-    pl->grid = sms * pl->ctas_per_sm;
-    pl->total_warps = (long long)pl->grid * pl->warps;
-    if (pl->total_warps > T) pl->total_warps = T;  // one tile or more per working warp
     // stage: bitmaps, x rows, column-set words, values, and 16 bytes of slack for the
     // branch-free loads one past a column's last value
     pl->stage_bytes =
         (uint32_t)round_up_u64(stage_vals_off(B) + 16ull * h->max_tile_units + 16, 128);
-    const long long budget = kSmemPerSm / pl->ctas_per_sm - 1024;
-    const long long per_warp = budget / pl->warps - warp_header_bytes(B);
-    int stages = (int)(per_warp / pl->stage_bytes);
-    if (stages > kMaxStages) stages = kMaxStages;
+    // Preferred launch shape first; fall back to fewer warps per SM when the stages of
+    // wide batches or dense formats do not fit two per warp.
+    const int want_warps = env_int("SPW_SPMV_WARPS", kDefaultWarpsPerCta, 1, kMaxWarpsPerCta);
+    const int want_ctas = env_int("SPW_SPMV_CTAS_PER_SM", kDefaultCtasPerSm, 1, 8);
+    const int shapes[][2] = {{want_warps, want_ctas}, {4, 2}, {4, 1}, {2, 1}, {1, 1}};
+    int stages = 0;
+    for (const auto& sh : shapes) {
+        pl->warps = sh[0];
+        pl->ctas_per_sm = sh[1];
+        const long long budget = kSmemPerSm / pl->ctas_per_sm - 1024;
+        const long long per_warp = budget / pl->warps - warp_header_bytes(B);
+        stages = per_warp > 0 ? (int)(per_warp / pl->stage_bytes) : 0;
+        if (stages >= kMinStages) break;
+    }
     if (stages < kMinStages) return SPW_ERR_UNSUPPORTED;
+    if (stages > kMaxStages) stages = kMaxStages;
+    pl->grid = sms * pl->ctas_per_sm;
+    pl->total_warps = (long long)pl->grid * pl->warps;
+    if (pl->total_warps > T) pl->total_warps = T;  // one tile or more per working warp
     pl->stages = stages;
     pl->warp_smem = warp_header_bytes(B) + (uint32_t)stages * pl->stage_bytes;
     pl->smem = (size_t)pl->warps * pl->warp_smem;

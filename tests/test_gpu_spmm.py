@@ -1,0 +1,112 @@
+"""GPU parity of the prefill SpMM (tcgen05) against the fp64 oracle.
+
+Bar: max|Y - Y_ref| / max|Y_ref| <= 5e-3 over each call's whole output (fp16 inputs, fp32
+accumulation in tensor memory, fp16 output); exact where the result is exact.  Full-size
+shapes are checked on seeded sampled rows (the oracle computes rows one by one)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from gpu_util import TOL, dev, host, needs_gpu, padded_rows
+import spmm_tiled_column_b200 as spw
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+
+def run(W, mask, X, ldx=None, ldy=None):
+    lin = spw.SparseLinear(dev(W), dev(mask))
+    M, K = X.shape
+    if ldx is None and M > 1 and K % 8:
+        ldx = -(-K // 8) * 8        # tensor copies need 16-byte row strides
+    Xd = dev(X) if ldx is None else padded_rows(X, ldx)
+    Y = None
+    if ldy is not None:
+        Y = torch.full((M, ldy), float("nan"), dtype=torch.float16, device="cuda")[:, :lin.N]
+    out = lin.spmm(Xd, Y)
+    torch.cuda.synchronize()
+    assert spw.spw_last_device_status() == spw.SPW_OK
+    return host(out).astype(np.float64), lin
+
+
+@pytest.mark.parametrize("N,K,M", [(256, 512, 16), (512, 256, 16), (256, 512, 256),
+                                   (300, 200, 37), (65, 130, 300), (1, 64, 1), (64, 1, 5),
+                                   (513, 1000, 600), (128, 4160, 64)])
+def test_parity_small(N, K, M):
+    W = workloads.weight(N, K, "gspmm")
+    mask = workloads.random_mask(N, K, 0.5, "gspmm")
+    X = workloads.normal_act(M, K, "gspmm")
+    Y, _ = run(W, mask, X)
+    assert oracle.rel_err(Y, oracle.spmm(W, mask, X)) <= TOL, (N, K, M)
+
+
+def test_tiny_config_layer():
+    layer = workloads.pruned_layer("tiny", 256, 512, 0.5, "cfg1")
+    X = workloads.normal_act(16, 512, "cfg1-prefill")
+    Y, _ = run(layer.W, layer.mask, X)
+    assert oracle.rel_err(Y, oracle.spmm(layer.W, layer.mask, X)) <= TOL
+
+
+def test_identity_exact_and_zero():
+    K = 384
+    X = workloads.normal_act(300, K, "gspmm-id")
+    Y, _ = run(np.eye(K, dtype=np.float16), np.eye(K, dtype=np.uint8), X)
+    np.testing.assert_array_equal(Y, X.astype(np.float64))
+    Y, _ = run(workloads.weight(200, K, "z"), np.zeros((200, K), np.uint8), X)
+    assert not Y.any()
+
+
+def test_dense_mask_matches_dense_product():
+    N, K, M = 256, 640, 256
+    W = workloads.weight(N, K, "gspmm-dense")
+    X = workloads.normal_act(M, K, "gspmm-dense")
+    Y, _ = run(W, np.ones((N, K), np.uint8), X)
+    ref = X.astype(np.float64) @ W.astype(np.float64).T
+    assert oracle.rel_err(Y, ref) <= TOL
+
+
+def test_dropped_weights_never_read():
+    N, K, M = 256, 512, 128
+    W = workloads.weight(N, K, "gspmm-drop")
+    mask = workloads.random_mask(N, K, 0.5, "gspmm-drop")
+    W2 = W.copy()
+    W2[mask == 0] = np.float16(np.nan)
+    X = workloads.normal_act(M, K, "gspmm-drop")
+    Y, _ = run(W2, mask, X)
+    assert np.isfinite(Y).all()
+    assert oracle.rel_err(Y, oracle.spmm(W, mask, X)) <= TOL
+
+
+def test_spmm_equals_spmv_rows():
+    N, K = 320, 1024
+    W = workloads.weight(N, K, "gspmm-v")
+    mask = workloads.random_mask(N, K, 0.5, "gspmm-v")
+    X = workloads.normal_act(16, K, "gspmm-v")
+    Y, lin = run(W, mask, X)
+    y = host(lin.spmv(dev(X))).astype(np.float64)
+    assert oracle.rel_err(Y, y) <= TOL
+
+
+def test_strided_and_m_zero():
+    N, K, M = 200, 264, 70
+    W = workloads.weight(N, K, "gspmm-s")
+    mask = workloads.random_mask(N, K, 0.5, "gspmm-s")
+    X = workloads.normal_act(M, K, "gspmm-s")
+    Y, lin = run(W, mask, X, ldx=272, ldy=208)
+    assert oracle.rel_err(Y, oracle.spmm(W, mask, X)) <= TOL
+    empty = torch.empty((0, K), dtype=torch.float16, device="cuda")
+    assert lin.spmm(empty).shape == (0, N)
+
+
+@pytest.mark.parametrize("name,s", [("q", 0.5), ("gate", 0.6), ("down", 0.7)])
+def test_llama7b_prefill_m2048_sampled(name, s):
+    N, K = workloads.LLAMA7B_LAYERS[name]
+    M = 2048
+    layer = workloads.pruned_layer(name, N, K, s, "cfg3")
+    X = workloads.normal_act(M, K, "cfg3", name)
+    Y, _ = run(layer.W, layer.mask, X)
+    rows = np.sort(workloads.rng("cfg3-rows", name).choice(M, 48, replace=False)).astype(np.int32)
+    ref = oracle.spmm(layer.W, layer.mask, X, rows)
+    assert oracle.rel_err(Y[rows], ref) <= TOL
+    assert np.isfinite(Y).all()
