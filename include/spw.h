@@ -168,6 +168,28 @@ int spw_spmv(const spw_format* hdr, const void* d_buf, const uint16_t* d_x, int 
              float threshold, const uint32_t* d_act_bits, uint16_t* d_y, int ldy, void* d_ws,
              uint64_t ws_bytes, void* stream);
 
+/* Allocation-free decode.  The pages have no counterpart to this call; it exists for
+ * callers that cannot call cudaMalloc, for example code running inside a framework that
+ * reserved all device memory up front and forbids further allocation, or a path that may
+ * not take the device-wide synchronisation an allocation can imply.  It computes exactly
+ * what spw_spmv computes (same arguments minus the workspace), using as its split-K
+ * workspace a fixed 8 MiB array inside the library's device image instead of caller
+ * memory.  It calls no cudaMalloc/cudaFree and no allocating library routine.
+ *   - Every GPU that loads the library holds the 8 MiB array until the process exits.
+ *   - Requests whose workspace (spw_spmv_workspace_bytes) exceeds
+ *     spw_spmv_noalloc_max_scratch_bytes() return SPW_ERR_UNSUPPORTED and launch nothing;
+ *     use spw_spmv with a caller workspace for those.
+ *   - The first call on a device looks up the array's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ *   - All calls share the one array and each call clears its counters first: calls whose
+ *     executions overlap on the GPU (other streams, other threads) race and give wrong
+ *     results.  Serialise them.
+ * Errors: as spw_spmv, plus UNSUPPORTED for the size limit. */
+uint64_t spw_spmv_noalloc_max_scratch_bytes(void);
+int spw_spmv_noalloc(const spw_format* hdr, const void* d_buf, const uint16_t* d_x, int B,
+                     int ldx, float threshold, const uint32_t* d_act_bits, uint16_t* d_y, int ldy,
+                     void* stream);
+
 /* Workspace bytes spw_spmm needs (0 in this version; d_ws may then be NULL). */
 uint64_t spw_spmm_workspace_bytes(const spw_format* hdr, int M);
 

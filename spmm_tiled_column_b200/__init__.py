@@ -64,6 +64,8 @@ SIGNATURES = {
     "spw_spmm_workspace_bytes": ([_FP, _I], _U64),
     "spw_spmm": ([_FP, _P, _P, _I, _I, _P, _I, _P, _U64, _P], _I),
     "spw_last_device_status": ([_P, _P], _I),
+    "spw_spmv_noalloc_max_scratch_bytes": ([], _U64),
+    "spw_spmv_noalloc": ([_FP, _P, _P, _I, _I, _F, _P, _P, _I, _P], _I),
 }
 
 
@@ -249,6 +251,25 @@ def spw_spmv(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.0,
     _check("spw_spmv", lib().spw_spmv(
         ctypes.byref(h), _ptr(buf), _ptr(x2), B, ldx, float(threshold), _ptr(act_bits),
         _ptr(y2), ldy, _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def spw_spmv_noalloc(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.0,
+                     act_bits: torch.Tensor | None = None, y: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Decode like spw_spmv, with the library's own fixed scratch instead of a workspace.
+
+    For callers that cannot allocate device memory; see include/spw.h for the size
+    limit and for why overlapping calls race."""
+    h = _hdr(hdr)
+    x2, ldx = _rows(_half(x, "x"), "x")
+    B = x2.shape[0]
+    if y is None:
+        y = torch.empty((B, h.N), dtype=torch.float16, device=x.device)
+    y2, ldy = _rows(_half(y, "y"), "y")
+    _check("spw_spmv_noalloc", lib().spw_spmv_noalloc(
+        ctypes.byref(h), _ptr(buf), _ptr(x2), B, ldx, float(threshold), _ptr(act_bits),
+        _ptr(y2), ldy, _stream(stream)))
     return y
 
 
