@@ -97,6 +97,17 @@ const char* spw_status_string(int status);
 /* Library version: 100 * major + minor.  The TCB format version is separate (1). */
 int spw_version(void);
 
+/* Launch overlap between consecutive decode calls (process-wide; off by default).
+ * When enabled, spw_spmv launches with programmatic dependent launch: its CTAs may start
+ * while the previous kernel on the stream is still finishing, and begin streaming the
+ * compressed weight (the TCB buffer) before that kernel's writes are visible.  It also
+ * lets the next kernel start early.  Activations, column sets, outputs and the
+ * workspace are only touched after the previous kernel has completed, so chaining
+ * layers stays correct; the one requirement is that the kernel immediately before
+ * spw_spmv on the stream does not write the TCB buffer being read (true for weights
+ * compressed at load time and left alone).  Returns the previous setting. */
+int spw_set_launch_overlap(int enable);
+
 /* Size of the TCB v1 buffer for an N x K mask (device uint8, row stride ld_mask bytes,
  * nonzero = kept).  [SPDP] format; layout above.  Writes bytes_total and nnz (host
  * pointers).  Synchronises `stream`.  Allocates 16 bytes of device scratch (offline).

@@ -53,6 +53,7 @@ _FP = ctypes.POINTER(spw_format)
 SIGNATURES = {
     "spw_status_string": ([_I], ctypes.c_char_p),
     "spw_version": ([], _I),
+    "spw_set_launch_overlap": ([_I], _I),
     "spw_format_query": ([_P, _I, _I, _I, _P, _P, _P], _I),
     "spw_compress": ([_P, _I, _P, _I, _I, _I, _P, _U64, _FP, _P], _I),
     "spw_format_read": ([_P, _U64, _FP, _P], _I),
@@ -138,6 +139,12 @@ def _hdr(h) -> spw_format:
     for k, v in dict(h).items():
         setattr(f, k, int(v))
     return f
+
+
+def spw_set_launch_overlap(enable: bool) -> bool:
+    """Enable/disable programmatic launch overlap of consecutive spw_spmv calls (see
+    include/spw.h for the one condition it needs); returns the previous setting."""
+    return bool(lib().spw_set_launch_overlap(1 if enable else 0))
 
 
 # ------------------------------------------------------------------ format

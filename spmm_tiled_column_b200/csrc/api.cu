@@ -1,6 +1,7 @@
 // api.cu -- status strings, version, header checks, the device status word.
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "spw_internal.cuh"
@@ -11,6 +12,7 @@ namespace {
 __device__ int g_device_status;
 
 constexpr int kMaxDevices = 64;
+std::atomic<int> g_launch_overlap{0};
 int* g_status_ptr[kMaxDevices];
 int g_sm_count[kMaxDevices];
 std::mutex g_mutex;
@@ -43,6 +45,8 @@ int device_sm_count() {
     }
     return g_sm_count[dev];
 }
+
+bool launch_overlap() { return g_launch_overlap.load(std::memory_order_relaxed) != 0; }
 
 int check_header(const spw_format* h) {
     if (!h) return SPW_ERR_INVALID_ARG;
@@ -79,6 +83,10 @@ const char* spw_status_string(int status) {
 }
 
 int spw_version(void) { return 100; }
+
+int spw_set_launch_overlap(int enable) {
+    return g_launch_overlap.exchange(enable ? 1 : 0) != 0;
+}
 
 int spw_format_read(const void* d_buf, uint64_t buf_bytes, spw_format* hdr_out, void* stream) {
     if (!d_buf || !hdr_out || buf_bytes < (uint64_t)spw::kHeaderBytes) return SPW_ERR_INVALID_ARG;

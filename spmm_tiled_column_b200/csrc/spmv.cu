@@ -171,7 +171,22 @@ spmv_kernel(const SpmvParams p) {
     // Tile coordinates of the next tile to issue, advanced incrementally.
     int issue_t = t_begin;
     int issue_kt = t_begin % nk;
-    auto issue_next = [&](int slot) {  // warp-collective; lane 0 issues the copies
+    // Copies for the next tile.  Weights (bitmaps, values) may be fetched before the
+    // previous kernel has finished; activations and column-set words only after
+    // pdl_wait(), so the prologue issues them separately (issue_x).  The stage's
+    // expected byte count always includes them, so the stage cannot complete early.
+    auto issue_x = [&](int slot, int kt_of_tile) {  // lane 0 only
+        const uint32_t bar = smem_u32(&mbar[slot]);
+        const uint32_t st = wsm_s + HDR + (uint32_t)slot * p.stage_bytes;
+        const int kcols = min(kTileCols, p.K - kt_of_tile * kTileCols);
+        const uint32_t xbytes = (uint32_t)((kcols * 2 + 15) & ~15);
+        const uint16_t* xsrc = p.x + (size_t)kt_of_tile * kTileCols;
+#pragma unroll
+        for (int b = 0; b < B; b++) bulk_g2s(st + 512u + 128u * b, xsrc + (size_t)b * p.ldx, xbytes, bar);
+        if (p.act_bits)
+            bulk_g2s(st + 512u + 128u * B, p.act_bits + ((kt_of_tile * 2) & ~3), 16u, bar);
+    };
+    auto issue_next = [&](int slot, bool with_x) {  // warp-collective; lane 0 issues
         if (issue_t + 1 - tpc_base >= kTptrCacheEntries) {  // refill the tileptr cache
             for (int j = lane; j < kTptrCacheEntries; j += 32)
                 if (issue_t + j <= T) tpc[j] = __ldg(p.tileptr + issue_t + j);
@@ -195,17 +210,20 @@ spmv_kernel(const SpmvParams p) {
             bulk_g2s_hint(st, p.bitmaps + (size_t)issue_t * kTileCols, 512u, bar, evict_first);
             if (vbytes)
                 bulk_g2s_hint(st + VOFF, p.values + (size_t)u0 * 8, vbytes, bar, evict_first);
-            const uint16_t* xsrc = p.x + (size_t)issue_kt * kTileCols;
-#pragma unroll
-            for (int b = 0; b < B; b++) bulk_g2s(st + 512u + 128u * b, xsrc + (size_t)b * p.ldx, xbytes, bar);
-            if (p.act_bits)
-                bulk_g2s(st + 512u + 128u * B, p.act_bits + ((issue_kt * 2) & ~3), 16u, bar);
+            if (with_x) issue_x(slot, issue_kt);
         }
         issue_t++;
         if (++issue_kt == nk) issue_kt = 0;
     };
 
-    for (int i = 0; i < S - 1 && i < ntiles; i++) issue_next(i);  // prologue
+    // Prologue: weights of the first S - 1 tiles, then (once the previous kernel on the
+    // stream is complete) their activations.
+    const int n_pro = min(S - 1, ntiles);
+    for (int i = 0; i < n_pro; i++) issue_next(i, false);
+    pdl_wait();
+    if (lane == 0)
+        for (int i = 0; i < n_pro; i++) issue_x(i, (t_begin + i) % nk);
+    pdl_launch_dependents();
 
     const uint32_t lanebit = 1u << lane, ltmask = lanebit - 1u;
     float acc0[B], acc1[B];
@@ -218,7 +236,7 @@ spmv_kernel(const SpmvParams p) {
 
     for (int i = 0; i < ntiles; i++) {
         const int t = t_begin + i;
-        if (i + S - 1 < ntiles) issue_next(slot == 0 ? S - 1 : slot - 1);
+        if (i + S - 1 < ntiles) issue_next(slot == 0 ? S - 1 : slot - 1, true);
         if (!mbar_wait(smem_u32(&mbar[slot]), phase)) {
             raise_status(p.status, SPW_ERR_TIMEOUT);
             for (int j = i + 1; j < ntiles && j < i + S; j++)  // drain (bounded)
@@ -317,6 +335,7 @@ spmv_kernel(const SpmvParams p) {
                 if (r1 < p.N) p.y[(size_t)b * p.ldy + r1] = __half_as_ushort(__float2half_rn(acc1[b]));
             }
         } else {
+            // Publish this piece: store the partials, then one release atomic per warp.
             const int idx = gw - g_first;
             float* mine = p.partials + ((size_t)s * p.maxc + idx) * B * 64;
 #pragma unroll
@@ -324,22 +343,36 @@ spmv_kernel(const SpmvParams p) {
                 mine[b * 64 + lane] = acc0[b];
                 mine[b * 64 + lane + 32] = acc1[b];
             }
-            __threadfence();
+            __syncwarp();
             uint32_t old = 0;
-            if (lane == 0) old = atomicAdd(&p.counters[s], 1u);
+            if (lane == 0) old = atom_add_release_gpu(&p.counters[s], 1u);
             old = __shfl_sync(0xffffffffu, old, 0);
             if ((int)old == count - 1) {
+                // Last contributor: sum every piece in contributor order (deterministic).
+                // Lane l owns rows 2l and 2l+1; eight pieces' loads are in flight at once.
                 __threadfence();
                 const float* base = p.partials + (size_t)s * p.maxc * B * 64;
-#pragma unroll
+                const int row = s * kStripRows + 2 * lane;
+#pragma unroll 1
                 for (int b = 0; b < B; b++) {
-                    float v0 = 0.0f, v1 = 0.0f;
-                    for (int j = 0; j < count; j++) {
-                        v0 += __ldcg(base + ((size_t)j * B + b) * 64 + lane);
-                        v1 += __ldcg(base + ((size_t)j * B + b) * 64 + lane + 32);
+                    float sx = 0.0f, sy = 0.0f;
+#pragma unroll 1
+                    for (int j0 = 0; j0 < count; j0 += 8) {
+                        float2 v[8];
+#pragma unroll
+                        for (int u = 0; u < 8; u++)
+                            v[u] = (j0 + u < count)
+                                       ? __ldcg((const float2*)(base + ((size_t)(j0 + u) * B + b) * 64) + lane)
+                                       : make_float2(0.0f, 0.0f);
+#pragma unroll
+                        for (int u = 0; u < 8; u++) {
+                            sx += v[u].x;
+                            sy += v[u].y;
+                        }
                     }
-                    if (r0 < p.N) p.y[(size_t)b * p.ldy + r0] = __half_as_ushort(__float2half_rn(v0));
-                    if (r1 < p.N) p.y[(size_t)b * p.ldy + r1] = __half_as_ushort(__float2half_rn(v1));
+                    if (row < p.N) p.y[(size_t)b * p.ldy + row] = __half_as_ushort(__float2half_rn(sx));
+                    if (row + 1 < p.N)
+                        p.y[(size_t)b * p.ldy + row + 1] = __half_as_ushort(__float2half_rn(sy));
                 }
                 if (lane == 0) p.counters[s] = 0u;
             }
@@ -418,9 +451,24 @@ int launch(const Plan& pl, const SpmvParams& prm, cudaStream_t s) {
     if (attr_smem[dev] < pl.smem) {
         SPW_CUDA_TRY(cudaFuncSetAttribute(spmv_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)pl.smem));
+        // The grid is sized for this many CTAs per SM; ask for the full shared-memory
+        // carveout so small per-CTA footprints do not lower the residency.
+        SPW_CUDA_TRY(cudaFuncSetAttribute(spmv_kernel<B>,
+                                          cudaFuncAttributePreferredSharedMemoryCarveout,
+                                          (int)cudaSharedmemCarveoutMaxShared));
         attr_smem[dev] = pl.smem;
     }
-    spmv_kernel<B><<<pl.grid, pl.warps * 32, pl.smem, s>>>(prm);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.grid);
+    cfg.blockDim = dim3(pl.warps * 32);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = launch_overlap() ? 1 : 0;
+    SPW_CUDA_TRY(cudaLaunchKernelEx(&cfg, spmv_kernel<B>, prm));
     SPW_LAUNCH_CHECK();
     return SPW_OK;
 }

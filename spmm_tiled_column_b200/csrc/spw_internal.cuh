@@ -10,7 +10,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/spw.h"
+#include "spw.h"
 
 namespace spw {
 
@@ -161,6 +161,23 @@ __device__ inline float fma_f16_f32(uint16_t a, uint16_t b, float c) {
     return d;
 }
 
+// Device-scope atomic add with release semantics (orders this thread's earlier writes,
+// and by cumulativity those of threads it synchronised with, before the add).
+__device__ inline uint32_t atom_add_release_gpu(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.release.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+                 : "memory");
+    return old;
+}
+
+// Programmatic dependent launch: wait until the previous kernel on the stream has
+// completed and its memory is visible / allow the next kernel to begin launching.
+// Both are no-ops for a kernel launched without the programmatic attribute.
+__device__ inline void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ inline void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ inline uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
@@ -205,6 +222,9 @@ int* device_status_ptr();
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
+
+// Process-wide switch set by spw_set_launch_overlap.
+bool launch_overlap();
 
 }  // namespace spw
 
