@@ -57,6 +57,21 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def measured_traffic():
+    """Per-launch DRAM bytes of the decode kernel from the committed ncu summary, or None
+    when the kernel source changed since those counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "spmv_decode_step_traffic.json")
+    try:
+        rec = json.load(open(path))
+        src = open(os.path.join(ROOT, rec["kernel_source"]), "rb").read()
+    except (OSError, ValueError, KeyError):
+        return None
+    if hashlib.sha256(src).hexdigest() != rec.get("kernel_source_sha256"):
+        return None
+    return int(rec["traffic_bytes_per_launch"])
+
+
 def decode_bytes(W, mask, x, t):
     """Algorithmic bytes of one decode call: values + bitmap words of the active columns,
     activations read, outputs written."""
@@ -361,7 +376,8 @@ def run_ours(args, rank, world, local_rank):
     avg_launch_us = ms * 1e3 / (args.steps * len(LAYERS))
     achieved = per_rank_gbs
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-            "frac": round(achieved / hbm_peak, 4), "traffic": None,
+            "frac": round(achieved / hbm_peak, 4), "traffic": measured_traffic(),
+            "traffic_source": "profiles/spmv_decode_step_traffic_llama7b_b1.md (ncu, per launch)",
             "kernel": "spw::spmv_kernel<1>", "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
             "avg_launch_us": round(avg_launch_us, 3),
             "per_linear": per_linear}
