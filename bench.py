@@ -5,11 +5,14 @@
 
 A step is one decode pass over the seven pruned linear layers of one Llama-7B decoder
 layer (q, k, v, o: 4096 x 4096; gate, up: 11008 x 4096; down: 4096 x 11008), fp16
-weights from N(0, 0.02) with a 50% per-row magnitude mask, batch 1.  The inputs of q..up
-are N(0, 1); the down projection's input is SiLU(g) * u with its smallest 50% of
-entries zeroed.  Each linear is one spw_spmv launch (threshold selection fused in), so a
-step is 7 launches, replayed from a CUDA graph.  Steps rotate over 4 such layers (about
-0.9 GB of compressed weights, 7x the 126 MB L2), so weight bytes come from HBM.
+weights from N(0, 0.02) with a 50% per-row magnitude mask, batch 1.  As in a decoder
+layer, q, k and v read one input (the attention input) and gate and up read one input
+(the FFN input), all N(0, 1); o reads its own N(0, 1) input; the down projection's input
+is SiLU(g) * u with its smallest 50% of entries zeroed.  The step is four decode
+launches, one per group of linears that share an input: [q, k, v], [o], [gate, up],
+[down] (spw_spmv_group; threshold selection fused in), replayed from a CUDA graph.
+Steps rotate over 4 device copies of the layer (about 0.9 GB of compressed weights, 7x
+the 126 MB L2), so weight bytes come from HBM.
 
 value = algorithmic bytes / time (GB/s): per linear, the values and bitmap words of the
 active columns plus the activations read and the outputs written.  Prefill (spw_spmm at
@@ -42,10 +45,13 @@ LAYERS = ["q", "k", "v", "o", "gate", "up", "down"]
 SPARSITY = 0.5
 DOWN_ACT_SPARSITY = 0.5
 N_ROTATE = 4
+GROUPS = [["q", "k", "v"], ["o"], ["gate", "up"], ["down"]]
 WORKLOAD = ("Llama-7B decoder-layer decode, batch 1: 7 pruned linears (q,k,v,o 4096x4096; "
             "gate,up 11008x4096; down 4096x11008), fp16 N(0,0.02) weights, 50% per-row "
-            "magnitude mask, TCB v1; q..up inputs N(0,1); down input SiLU(g)*u with the "
-            "smallest 50% zeroed; threshold selection fused into spw_spmv")
+            "magnitude mask, TCB v1; q/k/v share an N(0,1) input, gate/up share an N(0,1) "
+            "input, o has its own; down input SiLU(g)*u with the smallest 50% zeroed; one "
+            "grouped decode launch per shared input ([q,k,v],[o],[gate,up],[down]) with the "
+            "threshold selection fused in")
 
 
 def peaks():
@@ -85,29 +91,19 @@ def decode_bytes(W, mask, x, t):
 
 
 def make_layer():
-    """[(name, W, mask, x, t)] for the 7 linears of one decoder layer (seeded)."""
+    """[(name, W, mask, x, t)] for the 7 linears of one decoder layer (seeded); the
+    linears of one group share their input array."""
+    inputs = {}
     layer = []
-    for name in LAYERS:
-        N, K = workloads.LLAMA7B_LAYERS[name]
-        lin = workloads.pruned_layer(name, N, K, SPARSITY, "bench")
-        a = DOWN_ACT_SPARSITY if name == "down" else 0.0
-        x, _ = workloads.decode_act(name, 1, K, a, "bench")
-        layer.append((name, lin.W, lin.mask, x, 0.0))
+    for group in GROUPS:
+        for name in group:
+            N, K = workloads.LLAMA7B_LAYERS[name]
+            lin = workloads.pruned_layer(name, N, K, SPARSITY, "bench")
+            if group[0] not in inputs:
+                a = DOWN_ACT_SPARSITY if name == "down" else 0.0
+                inputs[group[0]], _ = workloads.decode_act(name, 1, K, a, "bench", group[0])
+            layer.append((name, lin.W, lin.mask, inputs[group[0]], 0.0))
     return layer
-
-
-class _Rotated:
-    """A device copy of a compressed weight at a different address (same header)."""
-
-    def __init__(self, base):
-        import spmm_tiled_column_b200 as spw
-        self._spw = spw
-        self.N, self.K, self.hdr = base.N, base.K, base.hdr
-        self.buf = base.buf.clone()
-        self.ws = base.workspace(1).clone()
-
-    def spmv(self, x, t, act_bits, y):
-        return self._spw.spw_spmv(self.hdr, self.buf, x, t, act_bits, y, self.ws)
 
 
 class Clocks:
@@ -209,21 +205,27 @@ def run_ours(args, rank, world, local_rank):
     spw.spw_set_launch_overlap(True)
     layer = make_layer()
     step_bytes = sum(decode_bytes(W, m, x, t) for _, W, m, x, t in layer)
-    lin = [[] for _ in range(N_ROTATE)]  # per rotation: (weight, x_dev, y_dev, t)
-    for name, W, m, x, t in layer:
-        base = spw.SparseLinear(to_dev(W), to_dev(m))
-        for r in range(N_ROTATE):
-            sl = base if r == 0 else _Rotated(base)
-            if r == 0:
-                sl.workspace(1)
-            xd = to_dev(x)
-            yd = torch.empty((1, base.N), dtype=torch.float16, device=dev)
-            lin[r].append((sl, xd, yd, t))
+    idx = {name: i for i, (name, *_rest) in enumerate(layer)}
+    base = [spw.SparseLinear(to_dev(W), to_dev(m)) for _, W, m, _, _ in layer]
+    # per rotation, per group: (names, headers, weight buffers, shared input, outputs, ws)
+    gdata = []
+    for r in range(N_ROTATE):
+        per = []
+        for group in GROUPS:
+            ls = [base[idx[n]] for n in group]
+            hdrs = [l.hdr for l in ls]
+            bufs = [l.buf if r == 0 else l.buf.clone() for l in ls]
+            xd = to_dev(layer[idx[group[0]]][3])
+            ys = [torch.empty((1, l.N), dtype=torch.float16, device=dev) for l in ls]
+            ws = torch.zeros(max(16, spw.spw_spmv_group_workspace_bytes(hdrs, 1)),
+                             dtype=torch.uint8, device=dev)
+            per.append((group, hdrs, bufs, xd, ys, ws))
+        gdata.append(per)
     torch.cuda.synchronize()
 
     def step(r):
-        for sl, xd, yd, t in lin[r]:
-            sl.spmv(xd, t, None, yd)
+        for _, hdrs, bufs, xd, ys, ws in gdata[r]:
+            spw.spw_spmv_group(hdrs, bufs, [xd] * len(bufs), 0.0, None, ys, ws)
 
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
@@ -273,16 +275,13 @@ def run_ours(args, rank, world, local_rank):
 
     # per-linear kernel timing (dominant kernel = spw_spmv) for the roofline, on the
     # launching stream, over graph replays of single linears
-    per_linear = {}
-    for j, name in enumerate(LAYERS):
+    def time_graphs(make_call, reps=50):
         gs = []
         for r in range(N_ROTATE):
             g = torch.cuda.CUDAGraph()
-            sl, xd, yd, t = lin[r][j]
             with torch.cuda.graph(g, stream=stream):
-                sl.spmv(xd, t, None, yd)
+                make_call(r)
             gs.append(g)
-        reps = 50
         with torch.cuda.stream(stream):
             for i in range(8):
                 gs[i % N_ROTATE].replay()
@@ -293,11 +292,30 @@ def run_ours(args, rank, world, local_rank):
                 gs[i % N_ROTATE].replay()
             b.record(stream)
         stream.synchronize()
-        us = a.elapsed_time(b) * 1e3 / reps
-        nb = decode_bytes(*layer[j][1:])
-        per_linear[name] = {"us": round(us, 3), "GB/s": round(nb / (us * 1e-6) / 1e9, 1),
-                            "bytes": int(nb)}
-        del gs
+        return a.elapsed_time(b) * 1e3 / reps
+
+    # each grouped launch on its own, and each linear as a single-layer launch
+    per_group = {}
+    for gi, group in enumerate(GROUPS):
+        def call(r, gi=gi):
+            _, hdrs, bufs, xd, ys, ws = gdata[r][gi]
+            spw.spw_spmv_group(hdrs, bufs, [xd] * len(bufs), 0.0, None, ys, ws)
+        us = time_graphs(call)
+        nb = sum(decode_bytes(*layer[idx[n]][1:]) for n in group)
+        per_group["+".join(group)] = {"us": round(us, 3), "GB/s": round(nb / (us * 1e-6) / 1e9, 1),
+                                      "bytes": int(nb)}
+    per_linear = {}
+    for gi, group in enumerate(GROUPS):
+        for pi, name in enumerate(group):
+            j = idx[name]
+            ws1 = base[j].workspace(1)
+            def call(r, gi=gi, pi=pi, j=j, ws1=ws1):
+                _, hdrs, bufs, xd, ys, _ws = gdata[r][gi]
+                spw.spw_spmv(hdrs[pi], bufs[pi], xd, 0.0, None, ys[pi], ws1)
+            us = time_graphs(call)
+            nb = decode_bytes(*layer[j][1:])
+            per_linear[name] = {"us": round(us, 3), "GB/s": round(nb / (us * 1e-6) / 1e9, 1),
+                                "bytes": int(nb)}
 
     # dense cuBLAS comparison at the same shapes (fp16 in, fp32 accumulate)
     dense = {}
@@ -324,21 +342,60 @@ def run_ours(args, rank, world, local_rank):
                        "speedup": round(us / per_linear[name]["us"], 3)}
         del Ws
 
+    # the same step done densely by cuBLAS, as an engine would: fused qkv and gate/up
+    # weights, four GEMVs per step, graph-replayed over two rotated copies (> L2 each)
+    dense_shapes = [(3 * 4096, 4096), (4096, 4096), (2 * 11008, 4096), (4096, 11008)]
+    dW = [[torch.randn(sh, device=dev, dtype=torch.float16) * 0.02 for sh in dense_shapes]
+          for _ in range(2)]
+    dX = [torch.randn((1, sh[1]), device=dev, dtype=torch.float16) for sh in dense_shapes]
+    dY = [torch.empty((1, sh[0]), device=dev, dtype=torch.float16) for sh in dense_shapes]
+    dgs = []
+    for r in range(2):
+        with torch.cuda.stream(stream):
+            for w, x, y in zip(dW[r], dX, dY):
+                torch.matmul(x, w.t(), out=y)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for w, x, y in zip(dW[r], dX, dY):
+                torch.matmul(x, w.t(), out=y)
+        dgs.append(g)
+    with torch.cuda.stream(stream):
+        for i in range(6):
+            dgs[i % 2].replay()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(40):
+            dgs[i % 2].replay()
+        b.record(stream)
+    stream.synchronize()
+    dense_step_us = a.elapsed_time(b) * 1e3 / 40
+    dense_bytes = sum(2 * n * k for n, k in dense_shapes)
+    dense_step = {"us": round(dense_step_us, 2),
+                  "GB/s": round(dense_bytes / (dense_step_us * 1e-6) / 1e9, 1),
+                  "sparse_step_us": round(ms * 1e3 / args.steps, 2),
+                  "speedup": round(dense_step_us / (ms * 1e3 / args.steps), 3),
+                  "how": "cuBLAS (torch.matmul) on the dense weights of the same layer: "
+                         "fused qkv 12288x4096, o, fused gate/up 22016x4096, down; batch 1"}
+    del dW, dgs
+
     # end to end through the public API with host buffers (pinned), eager calls
     e2e = None
     if not args.no_e2e:
-        hx = [[torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).pin_memory()
-               for _, _, _, x, _ in layer] for _ in range(N_ROTATE)]
-        hy = [[torch.empty((1, sl.N), dtype=torch.int16).pin_memory() for sl, _, _, _ in row]
-              for row in lin]
-        h2d = sum(2 * x.shape[1] for _, _, _, x, _ in layer)
-        d2h = sum(2 * sl.N for sl, _, _, _ in lin[0])
+        hx = [[torch.from_numpy(np.ascontiguousarray(layer[idx[g[0]]][3]).view(np.int16)).pin_memory()
+               for g, *_ in gdata[r]] for r in range(N_ROTATE)]
+        hy = [[[torch.empty((1, int(h.N)), dtype=torch.int16).pin_memory() for h in hdrs]
+               for _, hdrs, *_ in gdata[r]] for r in range(N_ROTATE)]
+        h2d = sum(2 * layer[idx[g[0]]][3].shape[1] for g in GROUPS)
+        d2h = sum(2 * l.N for l in base)
 
         def e2e_step(r):
-            for j, (sl, xd, yd, t) in enumerate(lin[r]):
-                xd.view(torch.int16).copy_(hx[r][j], non_blocking=True)
-                sl.spmv(xd, t, None, yd)
-                hy[r][j].copy_(yd.view(torch.int16), non_blocking=True)
+            for gi, (_, hdrs, bufs, xd, ys, ws) in enumerate(gdata[r]):
+                xd.view(torch.int16).copy_(hx[r][gi], non_blocking=True)
+                spw.spw_spmv_group(hdrs, bufs, [xd] * len(bufs), 0.0, None, ys, ws)
+                for y, hyy in zip(ys, hy[r][gi]):
+                    hyy.copy_(y.view(torch.int16), non_blocking=True)
 
         e2e_steps = max(10, min(args.steps, 100))
         with torch.cuda.stream(stream):
@@ -364,8 +421,9 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": round(ebytes / (ems * 1e-3) / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(ems / e2e_steps, 4),
-               "how": "per step: 7 x (pinned H2D of x, spw_spmv via the Python binding "
-                      "and C-ABI, D2H of y), eager launches on one stream"}
+               "how": "per step: for each of the 4 input groups, pinned H2D of the shared "
+                      "input, spw_spmv_group via the Python binding and C-ABI, D2H of the "
+                      "outputs; eager launches on one stream"}
 
     prefill = None
     try:
@@ -373,14 +431,15 @@ def run_ours(args, rank, world, local_rank):
     except Exception as exc:  # the prefill leg must not hide the decode number
         prefill = {"unavailable": f"{type(exc).__name__}: {exc}"[:300]}
 
-    avg_launch_us = ms * 1e3 / (args.steps * len(LAYERS))
+    avg_launch_us = ms * 1e3 / (args.steps * len(GROUPS))
     achieved = per_rank_gbs
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4), "traffic": measured_traffic(),
             "traffic_source": "profiles/spmv_decode_step_traffic_llama7b_b1.md (ncu, per launch)",
             "kernel": "spw::spmv_kernel<1>", "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
             "avg_launch_us": round(avg_launch_us, 3),
-            "per_linear": per_linear}
+            "per_group_launch": per_group,
+            "per_linear_single_launch": per_linear}
     result = {
         "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
@@ -389,12 +448,13 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": WORKLOAD, "global_batch": world, "parallelism": "replicas",
                    "launch_overlap": "programmatic dependent launch between consecutive decode kernels",
                    "l2": f"inputs larger than L2: {N_ROTATE} device copies of the layer rotated "
-                         f"({sum(s.buf.numel() for row in lin for s, _, _, _ in row) / 1e9:.2f} GB)"},
+                         f"({N_ROTATE * sum(l.buf.numel() for l in base) / 1e9:.2f} GB)"},
         "roofline": roof,
-        "gpu_launches": args.steps * len(LAYERS),
+        "gpu_launches": args.steps * len(GROUPS),
         "clocks": clk.summary(),
         "e2e": e2e,
         "dense_cublas_decode": dense,
+        "dense_cublas_step": dense_step,
         "prefill": prefill,
     }
     return result, layer

@@ -179,6 +179,24 @@ int spw_spmv(const spw_format* hdr, const void* d_buf, const uint16_t* d_x, int 
              float threshold, const uint32_t* d_act_bits, uint16_t* d_y, int ldy, void* d_ws,
              uint64_t ws_bytes, void* stream);
 
+/* Grouped decode: up to SPW_GROUP_MAX (8) independent layers in one launch, e.g. the
+ * q/k/v projections that share an input, or gate/up.  Layer l computes exactly what
+ * spw_spmv(&hdrs[l], d_bufs[l], d_xs[l], B, ldxs[l], threshold, d_act_bits[l], d_ys[l],
+ * ldys[l], ...) computes; all layers share B and the threshold.  One launch has one
+ * ramp-up and one tail instead of one per layer: the group's tiles form one
+ * concatenated work list split evenly across the persistent grid.  hdrs, d_bufs, d_xs,
+ * ldxs, d_act_bits (may itself be NULL: no column sets), d_ys and ldys are host arrays
+ * of n entries.  The workspace (spw_spmv_group_workspace_bytes) holds every layer's
+ * split-K counters and partial sums, with the counter rules of spw_spmv (all zero before
+ * the first call, left zero after each call that completes).  Asynchronous.
+ * Errors: as spw_spmv, plus INVALID_ARG for n outside 1..SPW_GROUP_MAX. */
+#define SPW_GROUP_MAX 8
+uint64_t spw_spmv_group_workspace_bytes(int n, const spw_format* hdrs, int B);
+int spw_spmv_group(int n, const spw_format* hdrs, const void* const* d_bufs,
+                   const uint16_t* const* d_xs, const int* ldxs,
+                   const uint32_t* const* d_act_bits, uint16_t* const* d_ys, const int* ldys,
+                   int B, float threshold, void* d_ws, uint64_t ws_bytes, void* stream);
+
 /* Allocation-free decode.  The pages have no counterpart to this call; it exists for
  * callers that cannot call cudaMalloc, for example code running inside a framework that
  * reserved all device memory up front and forbids further allocation, or a path that may

@@ -65,6 +65,8 @@ SIGNATURES = {
     "spw_spmm_workspace_bytes": ([_FP, _I], _U64),
     "spw_spmm": ([_FP, _P, _P, _I, _I, _P, _I, _P, _U64, _P], _I),
     "spw_last_device_status": ([_P, _P], _I),
+    "spw_spmv_group_workspace_bytes": ([_I, _FP, _I], _U64),
+    "spw_spmv_group": ([_I, _FP, _P, _P, _P, _P, _P, _P, _I, _F, _P, _U64, _P], _I),
     "spw_spmv_noalloc_max_scratch_bytes": ([], _U64),
     "spw_spmv_noalloc": ([_FP, _P, _P, _I, _I, _F, _P, _P, _I, _P], _I),
 }
@@ -259,6 +261,40 @@ def spw_spmv(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.0,
         ctypes.byref(h), _ptr(buf), _ptr(x2), B, ldx, float(threshold), _ptr(act_bits),
         _ptr(y2), ldy, _ptr(ws), ws.numel(), _stream(stream)))
     return y
+
+
+def _hdr_array(hdrs) -> ctypes.Array:
+    arr = (spw_format * len(hdrs))()
+    for i, h in enumerate(hdrs):
+        arr[i] = _hdr(h)
+    return arr
+
+
+def spw_spmv_group_workspace_bytes(hdrs, B: int) -> int:
+    return int(lib().spw_spmv_group_workspace_bytes(len(hdrs), _hdr_array(hdrs), int(B)))
+
+
+def spw_spmv_group(hdrs, bufs, xs, threshold: float = 0.0, act_bits=None, ys=None, ws=None,
+                   stream=None):
+    """Decode several layers in one launch; returns the list of outputs (B x N_l each)."""
+    n = len(hdrs)
+    harr = _hdr_array(hdrs)
+    x2 = [_rows(_half(x, "x"), "x") for x in xs]
+    B = x2[0][0].shape[0]
+    if ys is None:
+        ys = [torch.empty((B, int(h.N)), dtype=torch.float16, device=xs[0].device) for h in harr]
+    y2 = [_rows(_half(y, "y"), "y") for y in ys]
+    if ws is None:
+        ws = torch.zeros(max(spw_spmv_group_workspace_bytes(hdrs, B), 16), dtype=torch.uint8,
+                         device=xs[0].device)
+    P = ctypes.c_void_p * n
+    I = ctypes.c_int * n
+    ab = None if act_bits is None else P(*[None if a is None else a.data_ptr() for a in act_bits])
+    _check("spw_spmv_group", lib().spw_spmv_group(
+        n, harr, P(*[b.data_ptr() for b in bufs]), P(*[t.data_ptr() for t, _ in x2]),
+        I(*[ld for _, ld in x2]), ab, P(*[t.data_ptr() for t, _ in y2]), I(*[ld for _, ld in y2]),
+        B, float(threshold), _ptr(ws), ws.numel(), _stream(stream)))
+    return ys
 
 
 def spw_spmv_noalloc(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.0,
