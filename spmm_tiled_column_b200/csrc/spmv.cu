@@ -7,22 +7,24 @@
 // (§3.1: decode is bound by reading the weight).  The kernel below is this library's
 // design for B200:
 //
-//   * Work split: the tiles of the TCB buffer, in storage order (strip-major, then k),
-//     are cut into one contiguous, equal-count range per warp of a persistent grid
-//     (a multiple of the SM count).  A range covers a piece of one or two strips.
-//   * Data movement: each warp runs its own S-stage pipeline in shared memory.  One lane
-//     issues 1-D bulk copies (cp.async.bulk, no multicast) of a tile's 64 bitmap words,
-//     its packed values, the tile's 64 activations of every batch row and, if given,
-//     the caller's column-set words; a single mbarrier per stage counts the bytes.
-//   * Activation skipping: after a stage lands, the warp applies the threshold rule to
-//     its 64 x B activations, and a ballot gives the tile's active columns (some row's
-//     entry survives and the column holds a kept weight).  Inactive columns cost nothing
-//     further.
-//   * Bitmap decode: lane l owns rows l and l+32 of the strip.  For an active column
-//     with bitmap words (lo, hi) the lane's value sits at position
-//     colstart + popc(lo & lanes_below) in the column's segment (hi rows start after
-//     popc(lo) values); column starts are a warp prefix sum of popcounts.  fp16 x fp16 is
-//     fused into an fp32 accumulator (fma.rn.f32.f16).
+//   * Work split: the tiles of the TCB buffers of a group, in storage order (layer, strip,
+//     then k), are cut into one contiguous, equal-count range per consumer warp of a
+//     persistent grid (a multiple of the SM count).  A range covers a piece of one or two
+//     strips.
+//   * Data movement: each CTA has one producer warp and up to eight consumer warps.  Lane
+//     k of the producer streams consumer k's tiles -- the 64 bitmap words and the packed
+//     values, two 1-D bulk copies (cp.async.bulk, no multicast) -- into that consumer's
+//     S-stage ring, one "full" mbarrier per stage counting the bytes and one "empty"
+//     mbarrier per stage released by the consumer.  Consumers read activations (and the
+//     caller's column-set words) with plain loads, one tile ahead.
+//   * Activation skipping: the consumer applies the threshold rule to the tile's 64 x B
+//     activations; a ballot gives the active columns (some row's entry survives and the
+//     column holds a kept weight).  Inactive columns cost nothing further.
+//   * Bitmap decode: lane l owns rows 2l and 2l+1 of the strip, both in one 32-bit half of
+//     each column's bitmap word.  One popcount of the bits below row 2l gives the rank r of
+//     its first row inside the column's packed segment; the two candidate values are at
+//     r and r + 1, and row 2l+1 takes the second only when row 2l is kept.  fp16 x fp16 is
+//     fused into fp32 accumulators (fma.rn.f32.f16) under a predicate per row.
 //   * Split-K combine: a warp writes its fp32 partial for each strip piece into the
 //     workspace; the last contributor of a strip (counted with an atomic) sums all pieces
 //     in warp order -- a fixed order, so results are deterministic -- rounds to fp16 and
@@ -35,19 +37,23 @@
 namespace spw {
 namespace {
 
-constexpr int kMaxWarpsPerCta = 8;
-constexpr int kMaxGroup = 8;  // layers per grouped launch
-constexpr int kDefaultWarpsPerCta = 8;
+constexpr int kMaxConsumers = 8;  // consumer warps per CTA (plus one producer warp)
+constexpr int kMaxGroup = 8;      // layers per grouped launch
+constexpr int kDefaultConsumers = 8;
 constexpr int kDefaultCtasPerSm = 2;
 constexpr int kMaxStages = 4;
 constexpr int kMinStages = 2;
-// Per-warp header: mbarriers at 0, tileptr cache at 64, column records at 512, x~ at 1536
+constexpr int kCtaHeader = 128;  // CTA-wide words before the consumer regions
+// Per-consumer header: full mbarriers at 0, empty mbarriers at 32, column records for the
+// low 32 rows at 128 and for the high 32 rows at 640 (64 x {bits, address}), x~ at 1152
 // (64 columns x xt_stride(B) halves).
-constexpr int kTptrCacheOff = 64;
-constexpr int kTptrCacheEntries = 65;
-constexpr int kRecOff = 512;
-constexpr int kXtOff = 1536;
+constexpr int kFullOff = 0;
+constexpr int kEmptyOff = 32;
+constexpr int kRecLoOff = 128;
+constexpr int kRecHiOff = 640;
+constexpr int kXtOff = 1152;
 constexpr int kSmemPerSm = 227 * 1024;
+constexpr uint32_t kStageValsOff = 512;  // stage: 64 bitmap words, then packed values
 
 // One layer of a decode group: its TCB buffer sections, activations, outputs, workspace
 // sections, and its range in the group's concatenated tile space.
@@ -70,8 +76,8 @@ struct SpmvParams {
     SpmvLayer L[kMaxGroup];
     int n_layers;
     int* status;
-    int n_tiles;       // all layers
-    int total_warps;
+    int n_tiles;      // all layers
+    int total_warps;  // working consumer warps
     int stages;
     uint32_t stage_bytes;
     uint32_t warp_smem;
@@ -81,15 +87,18 @@ struct SpmvParams {
 __host__ __device__ constexpr int xt_stride(int B) {
     return B <= 1 ? 1 : B <= 2 ? 2 : B <= 4 ? 4 : B <= 8 ? 8 : 16;
 }
-__host__ __device__ constexpr uint32_t stage_vals_off(int B) { return 512u + 128u * B + 16u; }
+
+__host__ __device__ constexpr uint32_t warp_header_bytes(int B) {
+    return (uint32_t)((kXtOff + 64 * 2 * xt_stride(B) + 127) / 128 * 128);
+}
 
 __host__ __device__ inline long long warp_of_tile(long long t, long long total_warps,
                                                   long long n_tiles) {
     return ((t + 1) * total_warps - 1) / n_tiles;
 }
 
-// Columns decoded per group: loads for the whole group are issued before any
-// multiply-add, so a warp has 2 * kGroup independent load chains in flight.
+// Columns decoded per group: the loads of a whole group are issued before its
+// multiply-adds, so a warp has 2 * kGroup independent load chains in flight.
 constexpr int kGroup = 4;
 
 // Split a 32-bit word into its two fp16 halves (register halves, no shifts).
@@ -97,7 +106,75 @@ __device__ inline void split_halves(uint32_t w, uint16_t& lo, uint16_t& hi) {
     asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(w));
 }
 
-// Load x~ for G consecutive compacted columns (stride XS halves per column).
+// acc[b] += a * x[b] for N batch rows when flag != 0: one predicate, N predicated fused
+// multiply-adds (fp16 inputs, fp32 accumulator, one rounding).  A skipped product never
+// touches acc, so a value that belongs to another row (possibly Inf/NaN) cannot leak in.
+template <int N>
+__device__ inline void fma_rows_chunk(uint32_t flag, uint16_t a, const uint16_t* x, float* acc);
+
+template <>
+__device__ inline void fma_rows_chunk<1>(uint32_t flag, uint16_t a, const uint16_t* x, float* acc) {
+    asm("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %1, 0;\n\t"
+        "@p fma.rn.f32.f16 %0, %2, %3, %0;\n\t}"
+        : "+f"(acc[0])
+        : "r"(flag), "h"(a), "h"(x[0]));
+}
+
+template <>
+__device__ inline void fma_rows_chunk<2>(uint32_t flag, uint16_t a, const uint16_t* x, float* acc) {
+    asm("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t"
+        "@p fma.rn.f32.f16 %0, %3, %4, %0;\n\t"
+        "@p fma.rn.f32.f16 %1, %3, %5, %1;\n\t}"
+        : "+f"(acc[0]), "+f"(acc[1])
+        : "r"(flag), "h"(a), "h"(x[0]), "h"(x[1]));
+}
+
+template <>
+__device__ inline void fma_rows_chunk<4>(uint32_t flag, uint16_t a, const uint16_t* x, float* acc) {
+    asm("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "@p fma.rn.f32.f16 %0, %5, %6, %0;\n\t"
+        "@p fma.rn.f32.f16 %1, %5, %7, %1;\n\t"
+        "@p fma.rn.f32.f16 %2, %5, %8, %2;\n\t"
+        "@p fma.rn.f32.f16 %3, %5, %9, %3;\n\t}"
+        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
+        : "r"(flag), "h"(a), "h"(x[0]), "h"(x[1]), "h"(x[2]), "h"(x[3]));
+}
+
+template <>
+__device__ inline void fma_rows_chunk<8>(uint32_t flag, uint16_t a, const uint16_t* x, float* acc) {
+    asm("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %8, 0;\n\t"
+        "@p fma.rn.f32.f16 %0, %9, %10, %0;\n\t"
+        "@p fma.rn.f32.f16 %1, %9, %11, %1;\n\t"
+        "@p fma.rn.f32.f16 %2, %9, %12, %2;\n\t"
+        "@p fma.rn.f32.f16 %3, %9, %13, %3;\n\t"
+        "@p fma.rn.f32.f16 %4, %9, %14, %4;\n\t"
+        "@p fma.rn.f32.f16 %5, %9, %15, %5;\n\t"
+        "@p fma.rn.f32.f16 %6, %9, %16, %6;\n\t"
+        "@p fma.rn.f32.f16 %7, %9, %17, %7;\n\t}"
+        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3]), "+f"(acc[4]), "+f"(acc[5]),
+          "+f"(acc[6]), "+f"(acc[7])
+        : "r"(flag), "h"(a), "h"(x[0]), "h"(x[1]), "h"(x[2]), "h"(x[3]), "h"(x[4]), "h"(x[5]),
+          "h"(x[6]), "h"(x[7]));
+}
+
+// Any batch width as chunks of 8, 4, 2 and 1 rows.
+template <int B>
+__device__ inline void fma_rows(uint32_t flag, uint16_t a, const uint16_t* x, float* acc) {
+    if constexpr (B >= 8) {
+        fma_rows_chunk<8>(flag, a, x, acc);
+        if constexpr (B > 8) fma_rows<B - 8>(flag, a, x + 8, acc + 8);
+    } else if constexpr (B >= 4) {
+        fma_rows_chunk<4>(flag, a, x, acc);
+        if constexpr (B > 4) fma_rows<B - 4>(flag, a, x + 4, acc + 4);
+    } else if constexpr (B >= 2) {
+        fma_rows_chunk<2>(flag, a, x, acc);
+        if constexpr (B > 2) fma_rows<B - 2>(flag, a, x + 2, acc + 2);
+    } else {
+        fma_rows_chunk<1>(flag, a, x, acc);
+    }
+}
+
+// x~ for G consecutive compacted columns (stride XS halves per column).
 template <int B, int G>
 __device__ inline void load_xg(const uint16_t* xt, int j, uint16_t (&xv)[G][B]) {
     constexpr int XS = xt_stride(B);
@@ -130,39 +207,42 @@ __device__ inline void load_xg(const uint16_t* xt, int j, uint16_t (&xv)[G][B]) 
         for (int b = 0; b < B; b++) xv[c][b] = h[c * XS + b];
 }
 
-// G compacted active columns of one tile, branch-free: every lane loads the value at
-// its rank position for both of its rows whether or not its bit is set (the position is
-// always inside the stage), and a predicated fused multiply-add keeps the product only
-// where the bit is set, so a value of another row (possibly Inf/NaN) never leaks in.
+// G compacted active columns of one tile (G even), branch-free.  rech holds this lane's
+// half of each column record: {32 bitmap bits of the half, shared-memory address of the
+// half's first value}.  Every lane loads the two values at its rank whether or not its
+// bits are set (both addresses stay inside the stage), and the predicated multiply-adds
+// keep only the products of kept rows.
 template <int B, int G>
-__device__ inline void decode_group(const uint4* rec, const uint16_t* xt, int j, uint32_t lanebit,
-                                    uint32_t ltmask, float* acc0, float* acc1) {
-    uint4 r[G];
+__device__ inline void decode_pairs(const uint2* rech, const uint16_t* xt, int j, uint32_t below,
+                                    uint32_t bit0, uint32_t bit1, float* acc0, float* acc1) {
+    static_assert(G % 2 == 0, "records are loaded in pairs");
+    uint2 r[G];
     uint16_t xv[G][B];
 #pragma unroll
-    for (int c = 0; c < G; c++) r[c] = rec[j + c];
+    for (int c = 0; c < G; c += 2) {
+        const uint4 q = *(const uint4*)(rech + j + c);
+        r[c] = make_uint2(q.x, q.y);
+        r[c + 1] = make_uint2(q.z, q.w);
+    }
     load_xg<B, G>(xt, j, xv);
-    uint16_t w0[G], w1[G];
+    uint16_t v0[G], v1[G];
 #pragma unroll
     for (int c = 0; c < G; c++) {
-        w0[c] = lds_u16(r[c].z + 2u * __popc(r[c].x & ltmask));
-        w1[c] = lds_u16(r[c].w + 2u * __popc(r[c].y & ltmask));
+        const uint32_t a = r[c].y + 2u * __popc(r[c].x & below);
+        v0[c] = lds_u16(a);
+        v1[c] = lds_u16(a + 2u);
     }
 #pragma unroll
-    for (int c = 0; c < G; c++)
-#pragma unroll
-        for (int b = 0; b < B; b++) {
-            acc0[b] = fma_f16_f32_if(r[c].x, lanebit, w0[c], xv[c][b], acc0[b]);
-            acc1[b] = fma_f16_f32_if(r[c].y, lanebit, w1[c], xv[c][b], acc1[b]);
-        }
+    for (int c = 0; c < G; c++) {
+        const uint32_t f0 = r[c].x & bit0, f1 = r[c].x & bit1;
+        const uint16_t u1 = f0 ? v1[c] : v0[c];  // row 2l+1 follows row 2l's value if kept
+        fma_rows<B>(f0, v0[c], xv[c], acc0);
+        fma_rows<B>(f1, u1, xv[c], acc1);
+    }
 }
 
-__host__ __device__ constexpr uint32_t warp_header_bytes(int B) {
-    return (uint32_t)((kXtOff + 64 * 2 * xt_stride(B) + 127) / 128 * 128);
-}
-
-// Position of a warp's cursor in the group's tile space: layer, tile within the layer,
-// its k-tile and strip.
+// Position of a cursor in the group's tile space: layer, tile within the layer, its k-tile
+// and strip.
 struct Cursor {
     int l, t, kt, s;
 };
@@ -189,175 +269,196 @@ __device__ inline void cursor_next(const SpmvParams& p, Cursor& c) {
     }
 }
 
+// Keeps the accumulators' producing instructions (and so the shared-memory loads they
+// depend on) ahead of the stage release that follows.
 template <int B>
-__global__ void __launch_bounds__(kMaxWarpsPerCta * 32, B <= 9 ? 2 : 1)
-spmv_kernel(const __grid_constant__ SpmvParams p) {
-    extern __shared__ __align__(1024) unsigned char smem[];
-    constexpr int XS = xt_stride(B);
-    constexpr uint32_t VOFF = stage_vals_off(B);
+__device__ inline void pin_acc(float* acc0, float* acc1) {
+#pragma unroll
+    for (int b = 0; b < B; b++) asm volatile("" : "+f"(acc0[b]), "+f"(acc1[b]));
+}
+
+// Producer warp: lane k streams consumer k's tiles (bitmap words and packed values) into
+// its ring.  Weights only, so it may run before the previous kernel on the stream is
+// complete (programmatic dependent launch).  Before it exits, every copy it issued has
+// landed, so no copy can write shared memory after the CTA is gone.
+template <int B>
+__device__ void produce(const SpmvParams& p, unsigned char* regions, int W, int lane) {
     constexpr uint32_t HDR = warp_header_bytes(B);
-    const int warps_per_cta = blockDim.x >> 5;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    unsigned char* wsm = smem + (size_t)warp * p.warp_smem;
-    const int gw = blockIdx.x * warps_per_cta + warp;
-    // PW <= T (host side), so every working warp's range is nonempty and the warps
-    // touching a strip are consecutive.
-    const int T = p.n_tiles, PW = p.total_warps;
+    const int T = p.n_tiles, PW = p.total_warps, S = p.stages;
+    const int gw = blockIdx.x * W + lane;
+    const bool has = lane < W && gw < PW;
+    int n = 0;
+    Cursor c{0, 0, 0, 0};
+    if (has) {
+        const int tb = (int)((long long)gw * T / PW);
+        n = (int)((long long)(gw + 1) * T / PW) - tb;
+        c = cursor_at(p, tb);
+    }
+    const int nmax = __reduce_max_sync(0xffffffffu, n);
+    const uint32_t reg_s = smem_u32(regions + (size_t)(has ? lane : 0) * p.warp_smem);
+    const uint64_t pol = policy_evict_first();
+    uint32_t u0 = 0, u1 = 0;  // the current tile's value range, in 16-byte units
+    if (has) {
+        const uint32_t* tp = p.L[c.l].tileptr + c.t;
+        u0 = __ldg(tp);
+        u1 = __ldg(tp + 1);
+    }
+    int issued = 0;
+    bool ok = has;
+    for (int r = 0; r < nmax; r++) {
+        if (!ok || r >= n) continue;
+        Cursor nc = c;
+        cursor_next(p, nc);
+        uint32_t nu0 = 0, nu1 = 0;  // next tile's range, fetched a round ahead
+        if (r + 1 < n) {
+            const uint32_t* tp = p.L[nc.l].tileptr + nc.t;
+            nu0 = nc.l == c.l ? u1 : __ldg(tp);
+            nu1 = __ldg(tp + 1);
+        }
+        const int slot = r % S;
+        if (r >= S && !mbar_wait(reg_s + kEmptyOff + 8 * slot, (uint32_t)((r / S - 1) & 1))) {
+            raise_status(p.status, SPW_ERR_TIMEOUT);
+            ok = false;
+            continue;
+        }
+        const SpmvLayer& L = p.L[c.l];
+        uint64_t vbytes = u1 >= u0 ? 16ull * (u1 - u0) : ~0ull;
+        if (vbytes + kStageValsOff + 16u > p.stage_bytes) {  // tile larger than the header allows
+            raise_status(p.status, SPW_ERR_FORMAT);
+            vbytes = 0;
+        }
+        const uint32_t bar = reg_s + kFullOff + 8 * slot;
+        const uint32_t st = reg_s + HDR + (uint32_t)slot * p.stage_bytes;
+        mbar_arrive_expect_tx(bar, 512u + (uint32_t)vbytes);
+        bulk_g2s_hint(st, L.bitmaps + (size_t)c.t * kTileCols, 512u, bar, pol);
+        if (vbytes) bulk_g2s_hint(st + kStageValsOff, L.values + (size_t)u0 * 8, (uint32_t)vbytes, bar, pol);
+        issued = r + 1;
+        c = nc;
+        u0 = nu0;
+        u1 = nu1;
+    }
+    for (int r = issued > S ? issued - S : 0; r < issued; r++)
+        (void)mbar_wait(reg_s + kFullOff + 8 * (r % S), (uint32_t)((r / S) & 1));
+}
+
+// Activations of tile columns 2l and 2l+1 for every batch row (one 32-bit load per row
+// when both columns exist) and the caller's two column-set bits.
+template <int B>
+__device__ inline void load_act(const SpmvParams& p, const Cursor& c, int lane, uint32_t (&xw)[B],
+                                uint32_t& aw) {
+    const SpmvLayer& L = p.L[c.l];
+    const int col = c.kt * kTileCols + 2 * lane;
+    const uint16_t* xp = L.x + col;
+    if (col + 1 < L.K) {
+#pragma unroll
+        for (int b = 0; b < B; b++) xw[b] = __ldg((const unsigned int*)(xp + (size_t)b * L.ldx));
+    } else if (col < L.K) {
+#pragma unroll
+        for (int b = 0; b < B; b++) xw[b] = __ldg((const unsigned short*)(xp + (size_t)b * L.ldx));
+    } else {
+#pragma unroll
+        for (int b = 0; b < B; b++) xw[b] = 0u;
+    }
+    aw = 3u;
+    if (L.act_bits && col < L.K) aw = (__ldg(L.act_bits + (col >> 5)) >> (col & 31)) & 3u;
+}
+
+// Consumer warp gw: its tile range, decoded from its ring; partial sums flushed per strip.
+template <int B>
+__device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lane) {
+    constexpr int XS = xt_stride(B);
+    constexpr uint32_t HDR = warp_header_bytes(B);
+    const int T = p.n_tiles, PW = p.total_warps, S = p.stages;
     if (gw >= PW) return;  // warps are independent: no block-wide barrier follows
     const int t_begin = (int)((long long)gw * T / PW);
-    const int t_end = (int)((long long)(gw + 1) * T / PW);
-    const int ntiles = t_end - t_begin;
-    const int S = p.stages;
+    const int ntiles = (int)((long long)(gw + 1) * T / PW) - t_begin;
+    const uint32_t reg_s = smem_u32(reg);
+    uint2* recL = (uint2*)(reg + kRecLoOff);
+    uint2* recH = (uint2*)(reg + kRecHiOff);
+    uint16_t* xt = (uint16_t*)(reg + kXtOff);
+    const uint32_t ltmask = lanemask_lt();
+    // This lane's rows 2l and 2l+1 sit at bits q and q+1 of the low (lanes 0-15) or high
+    // (lanes 16-31) 32 bits of a column's bitmap word.
+    const int q = 2 * (lane & 15);
+    const uint32_t below = (1u << q) - 1u, bit0 = 1u << q, bit1 = 2u << q;
+    const uint2* rech = lane < 16 ? recL : recH;
 
-    uint64_t* mbar = (uint64_t*)wsm;
-    uint32_t* tpc = (uint32_t*)(wsm + kTptrCacheOff);
-    uint4* rec = (uint4*)(wsm + kRecOff);
-    uint16_t* xt = (uint16_t*)(wsm + kXtOff);
-    const uint32_t wsm_s = smem_u32(wsm);
-
-    if (lane == 0) {
-        for (int s = 0; s < S; s++) mbar_init(smem_u32(&mbar[s]), 1);
-        fence_mbar_init();
-    }
-    __syncwarp();
-
-    const uint64_t evict_first = policy_evict_first();
-    int tpc_layer = -1, tpc_base = 0;  // tileptr cache: layer and first local tile
-    Cursor ic = cursor_at(p, t_begin);  // next tile to issue
-    // Copies for one tile.  Weights (bitmaps, values) may be fetched before the previous
-    // kernel on the stream has finished; activations and column-set words only after
-    // pdl_wait(), so the prologue issues them separately (issue_x).  The stage's expected
-    // byte count always includes them, so the stage cannot complete early.
-    auto issue_x = [&](int slot, const Cursor& c) {  // lane 0 only
-        const SpmvLayer& L = p.L[c.l];
-        const uint32_t bar = smem_u32(&mbar[slot]);
-        const uint32_t st = wsm_s + HDR + (uint32_t)slot * p.stage_bytes;
-        const int kcols = min(kTileCols, L.K - c.kt * kTileCols);
-        const uint32_t xbytes = (uint32_t)((kcols * 2 + 15) & ~15);
-        const uint16_t* xsrc = L.x + (size_t)c.kt * kTileCols;
-#pragma unroll
-        for (int b = 0; b < B; b++) bulk_g2s(st + 512u + 128u * b, xsrc + (size_t)b * L.ldx, xbytes, bar);
-        if (L.act_bits) bulk_g2s(st + 512u + 128u * B, L.act_bits + ((c.kt * 2) & ~3), 16u, bar);
-    };
-    auto issue_next = [&](int slot, bool with_x) {  // warp-collective; lane 0 issues
-        const SpmvLayer& L = p.L[ic.l];
-        if (ic.l != tpc_layer || ic.t + 1 - tpc_base >= kTptrCacheEntries) {  // refill cache
-            for (int j = lane; j < kTptrCacheEntries; j += 32)
-                if (ic.t + j <= L.n_tiles) tpc[j] = __ldg(L.tileptr + ic.t + j);
-            __syncwarp();
-            tpc_layer = ic.l;
-            tpc_base = ic.t;
-        }
-        if (lane == 0) {
-            const uint32_t bar = smem_u32(&mbar[slot]);
-            const uint32_t st = wsm_s + HDR + (uint32_t)slot * p.stage_bytes;
-            const uint32_t u0 = tpc[ic.t - tpc_base], u1 = tpc[ic.t + 1 - tpc_base];
-            uint32_t vbytes = (u1 - u0) * 16u;
-            if (vbytes + VOFF + 16u > p.stage_bytes) {  // tile larger than the header allows
-                raise_status(p.status, SPW_ERR_FORMAT);
-                vbytes = 0;
-            }
-            const int kcols = min(kTileCols, L.K - ic.kt * kTileCols);
-            const uint32_t xbytes = (uint32_t)((kcols * 2 + 15) & ~15);
-            const uint32_t total = 512u + vbytes + (uint32_t)B * xbytes + (L.act_bits ? 16u : 0u);
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(bar, total);
-            bulk_g2s_hint(st, L.bitmaps + (size_t)ic.t * kTileCols, 512u, bar, evict_first);
-            if (vbytes) bulk_g2s_hint(st + VOFF, L.values + (size_t)u0 * 8, vbytes, bar, evict_first);
-            if (with_x) issue_x(slot, ic);
-        }
-        cursor_next(p, ic);
-    };
-
-    // Prologue: weights of the first S - 1 tiles, then (once the previous kernel on the
-    // stream is complete) their activations.
-    const int n_pro = min(S - 1, ntiles);
-    for (int i = 0; i < n_pro; i++) issue_next(i, false);
+    // Activations, column sets, outputs and the workspace only after the previous kernel
+    // on the stream is complete.
     pdl_wait();
-    if (lane == 0) {
-        Cursor c = cursor_at(p, t_begin);
-        for (int i = 0; i < n_pro; i++) {
-            issue_x(i, c);
-            cursor_next(p, c);
-        }
-    }
     pdl_launch_dependents();
 
-    const uint32_t lanebit = 1u << lane, ltmask = lanebit - 1u;
     float acc0[B], acc1[B];
 #pragma unroll
     for (int b = 0; b < B; b++) acc0[b] = acc1[b] = 0.0f;
-    Cursor cc = cursor_at(p, t_begin);  // tile being consumed
+    Cursor cc = cursor_at(p, t_begin);
+    uint32_t xw[B], aw;
+    load_act<B>(p, cc, lane, xw, aw);
     int slot = 0;
     uint32_t phase = 0;
 
     for (int i = 0; i < ntiles; i++) {
-        if (i + S - 1 < ntiles) issue_next(slot == 0 ? S - 1 : slot - 1, true);
-        if (!mbar_wait(smem_u32(&mbar[slot]), phase)) {
+        const Cursor cur = cc;
+        uint32_t xc[B];
+#pragma unroll
+        for (int b = 0; b < B; b++) xc[b] = xw[b];
+        const uint32_t ac = aw;
+        cursor_next(p, cc);
+        if (i + 1 < ntiles) load_act<B>(p, cc, lane, xw, aw);  // one tile ahead
+        const SpmvLayer& L = p.L[cur.l];
+        const uint32_t st_s = reg_s + HDR + (uint32_t)slot * p.stage_bytes;
+        // Warp-uniform outcome: the ballots below need every lane.
+        if (!__all_sync(0xffffffffu, mbar_wait(reg_s + kFullOff + 8 * slot, phase))) {
             raise_status(p.status, SPW_ERR_TIMEOUT);
-            for (int j = i + 1; j < ntiles && j < i + S; j++)  // drain (bounded)
-                (void)mbar_wait(smem_u32(&mbar[j % S]), (uint32_t)((j / S) & 1));
-            return;
+            return;  // the producer drains the copies still in flight
         }
-        const SpmvLayer& L = p.L[cc.l];
-        const unsigned char* st = wsm + HDR + (uint32_t)slot * p.stage_bytes;
-        const uint64_t* bm = (const uint64_t*)st;
-        const uint16_t* xr = (const uint16_t*)(st + 512);
 
-        // Activations of the lane's two columns, threshold rule, column set.
-        const int k0 = cc.kt * kTileCols + lane;
-        bool ok0 = k0 < L.K, ok1 = k0 + 32 < L.K;
-        if (L.act_bits) {
-            const uint32_t* aw = (const uint32_t*)(st + 512 + 128 * B);
-            const int w = (cc.kt * 2) & 3;
-            ok0 = ok0 && ((aw[w] >> lane) & 1u);
-            ok1 = ok1 && ((aw[w + 1] >> lane) & 1u);
-        }
+        // Threshold rule and column set for columns 2l and 2l+1.
+        const int col = cur.kt * kTileCols + 2 * lane;
+        const bool in0 = col < L.K && (ac & 1u), in1 = col + 1 < L.K && (ac & 2u);
         uint16_t xa[B], xb[B];
         bool any0 = false, any1 = false;
 #pragma unroll
         for (int b = 0; b < B; b++) {
-            const uint16_t a0 = xr[b * 64 + lane], a1 = xr[b * 64 + lane + 32];
-            const bool p0 = ok0 && passes_threshold(a0, p.t);
-            const bool p1 = ok1 && passes_threshold(a1, p.t);
-            xa[b] = p0 ? a0 : (uint16_t)0;
-            xb[b] = p1 ? a1 : (uint16_t)0;
+            uint16_t lo, hi;
+            split_halves(xc[b], lo, hi);
+            const bool p0 = in0 && passes_threshold(lo, p.t);
+            const bool p1 = in1 && passes_threshold(hi, p.t);
+            xa[b] = p0 ? lo : (uint16_t)0;
+            xb[b] = p1 ? hi : (uint16_t)0;
             any0 |= p0;
             any1 |= p1;
         }
-        const uint64_t w0 = bm[lane], w1 = bm[lane + 32];
-        any0 = any0 && w0 != 0;
-        any1 = any1 && w1 != 0;
-        const uint32_t act_lo = __ballot_sync(0xffffffffu, any0);
-        const uint32_t act_hi = __ballot_sync(0xffffffffu, any1);
-        const int n_act = __popc(act_lo) + __popc(act_hi);
+        const uint4 bw = *(const uint4*)(reg + HDR + (size_t)slot * p.stage_bytes + 16 * lane);
+        any0 = any0 && (bw.x | bw.y) != 0u;
+        any1 = any1 && (bw.z | bw.w) != 0u;
+        const uint32_t m0 = __ballot_sync(0xffffffffu, any0);
+        const uint32_t m1 = __ballot_sync(0xffffffffu, any1);
+        const int n_act = __popc(m0) + __popc(m1);
 
         if (n_act > 0) {
-            // Column starts within the tile's values (all 64 columns, in column order):
-            // one warp scan of both counts packed as 16-bit halves (sums stay <= 2048).
-            const int c0 = __popcll(w0), c1 = __popcll(w1);
-            const int sp = warp_inclusive_scan(c0 | (c1 << 16), lane);
-            const int tot0 = __shfl_sync(0xffffffffu, sp, 31) & 0xffff;
-            const int s0 = sp & 0xffff, s1 = sp >> 16;
-            const uint32_t vb = wsm_s + HDR + (uint32_t)slot * p.stage_bytes + VOFF;
-            const uint32_t a0 = vb + 2u * (uint32_t)(s0 - c0);
-            const uint32_t a1 = vb + 2u * (uint32_t)(tot0 + s1 - c1);
-            // Records {lo bits, hi bits, address of the lo rows' first value, address of
-            // the hi rows' first value}.  When every column is active they sit at their
-            // column positions and the decode is fully unrolled; otherwise the active
-            // columns are compacted and padded with empty records to a group multiple.
+            // Column starts within the tile's values (all 64 columns, in column order).
+            const int cl0 = __popc(bw.x), c0 = cl0 + __popc(bw.y);
+            const int cl1 = __popc(bw.z), c1 = cl1 + __popc(bw.w);
+            const int incl = warp_inclusive_scan(c0 + c1, lane);
+            const uint32_t vb = st_s + kStageValsOff;
+            const uint32_t a0 = vb + 2u * (uint32_t)(incl - c0 - c1);
+            const uint32_t a1 = a0 + 2u * (uint32_t)c0;
+            // Records at their column positions when every column is active (fully
+            // unrolled decode); otherwise the active columns are compacted, in column
+            // order, and padded with empty records to a group multiple.
             const bool all = B <= 4 && n_act == 64;  // wider batches keep the loop (registers)
-            const int pos0 = all ? lane : __popc(act_lo & ltmask);
-            const int pos1 = all ? lane + 32 : __popc(act_lo) + __popc(act_hi & ltmask);
+            const int pos0 = all ? 2 * lane : __popc(m0 & ltmask) + __popc(m1 & ltmask);
+            const int pos1 = pos0 + ((all || any0) ? 1 : 0);
             if (any0) {
-                rec[pos0] = make_uint4((uint32_t)w0, (uint32_t)(w0 >> 32), a0,
-                                       a0 + 2u * __popc((uint32_t)w0));
+                recL[pos0] = make_uint2(bw.x, a0);
+                recH[pos0] = make_uint2(bw.y, a0 + 2u * (uint32_t)cl0);
 #pragma unroll
                 for (int b = 0; b < B; b++) xt[pos0 * XS + b] = xa[b];
             }
             if (any1) {
-                rec[pos1] = make_uint4((uint32_t)w1, (uint32_t)(w1 >> 32), a1,
-                                       a1 + 2u * __popc((uint32_t)w1));
+                recL[pos1] = make_uint2(bw.z, a1);
+                recH[pos1] = make_uint2(bw.w, a1 + 2u * (uint32_t)cl1);
 #pragma unroll
                 for (int b = 0; b < B; b++) xt[pos1 * XS + b] = xb[b];
             }
@@ -366,63 +467,59 @@ spmv_kernel(const __grid_constant__ SpmvParams p) {
                     __syncwarp();
 #pragma unroll
                     for (int j = 0; j < 64; j += kGroup)
-                        decode_group<B, kGroup>(rec, xt, j, lanebit, ltmask, acc0, acc1);
+                        decode_pairs<B, kGroup>(rech, xt, j, below, bit0, bit1, acc0, acc1);
                 }
             }
             if (!all) {
                 const int n_pad = (n_act + kGroup - 1) & ~(kGroup - 1);
                 if (lane < n_pad - n_act) {
-                    rec[n_act + lane] = make_uint4(0u, 0u, vb, vb);
-#pragma unroll
-                    for (int b = 0; b < B; b++) xt[(n_act + lane) * XS + b] = 0;
+                    recL[n_act + lane] = make_uint2(0u, vb);
+                    recH[n_act + lane] = make_uint2(0u, vb);
                 }
                 __syncwarp();
                 for (int j = 0; j < n_pad; j += kGroup)
-                    decode_group<B, kGroup>(rec, xt, j, lanebit, ltmask, acc0, acc1);
+                    decode_pairs<B, kGroup>(rech, xt, j, below, bit0, bit1, acc0, acc1);
             }
         }
+        pin_acc<B>(acc0, acc1);
         __syncwarp();
+        if (lane == 0) mbar_arrive(reg_s + kEmptyOff + 8 * slot);  // stage back to the producer
         if (++slot == S) {
             slot = 0;
             phase ^= 1u;
         }
 
         // End of this warp's piece of strip s: write or combine the partial sums.
-        const bool strip_end = (cc.kt == L.n_ktiles - 1) || (i + 1 == ntiles);
-        const int s = cc.s;
         const int nk = L.n_ktiles;
+        if (cur.kt != nk - 1 && i + 1 != ntiles) continue;
+        const int s = cur.s;
         const int first = L.tile_begin + s * nk;
-        cursor_next(p, cc);
-        if (!strip_end) continue;
         const int g_first = (int)warp_of_tile(first, PW, T);
         const int g_last = (int)warp_of_tile((long long)first + nk - 1, PW, T);
         const int count = g_last - g_first + 1;
-        const int r0 = s * kStripRows + lane, r1 = r0 + 32;
+        const int r0 = s * kStripRows + 2 * lane;
         if (count == 1) {
 #pragma unroll
             for (int b = 0; b < B; b++) {
                 if (r0 < L.N) L.y[(size_t)b * L.ldy + r0] = __half_as_ushort(__float2half_rn(acc0[b]));
-                if (r1 < L.N) L.y[(size_t)b * L.ldy + r1] = __half_as_ushort(__float2half_rn(acc1[b]));
+                if (r0 + 1 < L.N)
+                    L.y[(size_t)b * L.ldy + r0 + 1] = __half_as_ushort(__float2half_rn(acc1[b]));
             }
         } else {
             // Publish this piece: store the partials, then one release atomic per warp.
             const int idx = gw - g_first;
-            float* mine = L.partials + ((size_t)s * L.maxc + idx) * B * 64;
+            float2* mine = (float2*)(L.partials + ((size_t)s * L.maxc + idx) * B * 64);
 #pragma unroll
-            for (int b = 0; b < B; b++) {
-                mine[b * 64 + lane] = acc0[b];
-                mine[b * 64 + lane + 32] = acc1[b];
-            }
+            for (int b = 0; b < B; b++) mine[b * 32 + lane] = make_float2(acc0[b], acc1[b]);
             __syncwarp();
             uint32_t old = 0;
             if (lane == 0) old = atom_add_release_gpu(&L.counters[s], 1u);
             old = __shfl_sync(0xffffffffu, old, 0);
             if ((int)old == count - 1) {
-                // Last contributor: sum every piece in contributor order (deterministic).
-                // Lane l owns rows 2l and 2l+1; eight pieces' loads are in flight at once.
+                // Last contributor: sum every piece in contributor order (deterministic),
+                // eight pieces' loads in flight at once.
                 __threadfence();
                 const float* base = L.partials + (size_t)s * L.maxc * B * 64;
-                const int row = s * kStripRows + 2 * lane;
 #pragma unroll 1
                 for (int b = 0; b < B; b++) {
                     float sx = 0.0f, sy = 0.0f;
@@ -440,9 +537,9 @@ spmv_kernel(const __grid_constant__ SpmvParams p) {
                             sy += v[u].y;
                         }
                     }
-                    if (row < L.N) L.y[(size_t)b * L.ldy + row] = __half_as_ushort(__float2half_rn(sx));
-                    if (row + 1 < L.N)
-                        L.y[(size_t)b * L.ldy + row + 1] = __half_as_ushort(__float2half_rn(sy));
+                    if (r0 < L.N) L.y[(size_t)b * L.ldy + r0] = __half_as_ushort(__float2half_rn(sx));
+                    if (r0 + 1 < L.N)
+                        L.y[(size_t)b * L.ldy + r0 + 1] = __half_as_ushort(__float2half_rn(sy));
                 }
                 if (lane == 0) L.counters[s] = 0u;
             }
@@ -452,8 +549,34 @@ spmv_kernel(const __grid_constant__ SpmvParams p) {
     }
 }
 
+template <int B>
+__global__ void __launch_bounds__((kMaxConsumers + 1) * 32, B <= 8 ? 2 : 1)
+spmv_kernel(const __grid_constant__ SpmvParams p) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int W = (int)(blockDim.x >> 5) - 1;  // consumer warps; the last warp produces
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char* regions = smem + kCtaHeader;
+    if (threadIdx.x == 0) {
+        for (int k = 0; k < W; k++) {
+            const uint32_t r = smem_u32(regions + (size_t)k * p.warp_smem);
+            for (int s = 0; s < p.stages; s++) {
+                mbar_init(r + kFullOff + 8 * s, 1);
+                mbar_init(r + kEmptyOff + 8 * s, 1);
+            }
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (warp == W) {
+        produce<B>(p, regions, W, lane);
+        pdl_launch_dependents();
+        return;
+    }
+    consume<B>(p, regions + (size_t)warp * p.warp_smem, blockIdx.x * W + warp, lane);
+}
+
 struct Plan {
-    int grid, warps, ctas_per_sm, stages;
+    int grid, warps, ctas_per_sm, stages;  // warps = consumer warps per CTA
     uint32_t stage_bytes, warp_smem;
     size_t smem;
     long long n_tiles, total_warps;
@@ -463,7 +586,7 @@ struct Plan {
     uint64_t ws_bytes;
 };
 
-// Occupancy knobs: warps per CTA and CTAs per SM.  SPW_SPMV_WARPS and
+// Occupancy knobs: consumer warps per CTA and CTAs per SM.  SPW_SPMV_WARPS and
 // SPW_SPMV_CTAS_PER_SM override the defaults (a tuning aid; both change only the launch
 // shape, never the work done).
 int env_int(const char* name, int dflt, int lo, int hi) {
@@ -485,19 +608,19 @@ int make_plan(int n, const spw_format* h, int B, Plan* pl) {
     }
     if (T > 0x7fffffffll) return SPW_ERR_UNSUPPORTED;
     pl->n_tiles = T;
-    // stage: bitmaps, x rows, column-set words, values, and 16 bytes of slack for the
-    // branch-free loads one past a column's last value
-    pl->stage_bytes = (uint32_t)round_up_u64(stage_vals_off(B) + 16ull * max_units + 16, 128);
+    // stage: bitmap words, values, and 16 bytes of slack for the branch-free loads one
+    // past a column's last value
+    pl->stage_bytes = (uint32_t)round_up_u64(kStageValsOff + 16ull * max_units + 16, 128);
     // Preferred launch shape first; fall back to fewer warps per SM when the stages of
     // wide batches or dense formats do not fit two per warp.
-    const int want_warps = env_int("SPW_SPMV_WARPS", kDefaultWarpsPerCta, 1, kMaxWarpsPerCta);
+    const int want_warps = env_int("SPW_SPMV_WARPS", kDefaultConsumers, 1, kMaxConsumers);
     const int want_ctas = env_int("SPW_SPMV_CTAS_PER_SM", kDefaultCtasPerSm, 1, 32);
     const int shapes[][2] = {{want_warps, want_ctas}, {4, 2}, {4, 1}, {2, 1}, {1, 1}};
     int stages = 0;
     for (const auto& sh : shapes) {
         pl->warps = sh[0];
-        pl->ctas_per_sm = sh[1];
-        const long long budget = kSmemPerSm / pl->ctas_per_sm - 1024;
+        pl->ctas_per_sm = B > 8 && sh[1] > 1 ? 1 : sh[1];  // wide batches: one CTA per SM
+        const long long budget = kSmemPerSm / pl->ctas_per_sm - 1024 - kCtaHeader;
         const long long per_warp = budget / pl->warps - warp_header_bytes(B);
         stages = per_warp > 0 ? (int)(per_warp / pl->stage_bytes) : 0;
         if (stages >= kMinStages) break;
@@ -509,7 +632,7 @@ int make_plan(int n, const spw_format* h, int B, Plan* pl) {
     if (pl->total_warps > T) pl->total_warps = T;  // one tile or more per working warp
     pl->stages = stages;
     pl->warp_smem = warp_header_bytes(B) + (uint32_t)stages * pl->stage_bytes;
-    pl->smem = (size_t)pl->warps * pl->warp_smem;
+    pl->smem = kCtaHeader + (size_t)pl->warps * pl->warp_smem;
     // Per layer: the most warps that share one strip under this partition, and the
     // layer's workspace section (arrival counters, then fp32 partial sums).
     uint64_t off = 0;
@@ -551,7 +674,7 @@ int launch(const Plan& pl, const SpmvParams& prm, cudaStream_t s) {
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.grid);
-    cfg.blockDim = dim3(pl.warps * 32);
+    cfg.blockDim = dim3((pl.warps + 1) * 32);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
