@@ -21,10 +21,14 @@
 //     activations; a ballot gives the active columns (some row's entry survives and the
 //     column holds a kept weight).  Inactive columns cost nothing further.
 //   * Bitmap decode: lane l owns rows 2l and 2l+1 of the strip, both in one 32-bit half of
-//     each column's bitmap word.  One popcount of the bits below row 2l gives the rank r of
-//     its first row inside the column's packed segment; the two candidate values are at
-//     r and r + 1, and row 2l+1 takes the second only when row 2l is kept.  fp16 x fp16 is
-//     fused into fp32 accumulators (fma.rn.f32.f16) under a predicate per row.
+//     each column's bitmap word, at bits q and q+1 (q = 2l mod 32).  The kept rows from
+//     2l+1 upward hold the last c values of that half's packed segment, c = popc(bits >>
+//     (q+1)); row 2l+1's value, if kept, is the first of them and row 2l's, if kept, the one
+//     just before.  One popcount, one multiply-add for the
+//     address and two 16-bit loads per column; fp16 x fp16 is fused into fp32 accumulators
+//     (fma.rn.f32.f16) under a predicate per row.  A column's record {low bits, end of the
+//     low half, high bits, end of the high half} is read with one 64-bit load per lane
+//     (each half-warp reads its own 8 bytes of the same 16).
 //   * Split-K combine: a warp writes its fp32 partial for each strip piece into the
 //     workspace; the last contributor of a strip (counted with an atomic) sums all pieces
 //     in warp order -- a fixed order, so results are deterministic -- rounds to fp16 and
@@ -44,13 +48,11 @@ constexpr int kDefaultCtasPerSm = 2;
 constexpr int kMaxStages = 4;
 constexpr int kMinStages = 2;
 constexpr int kCtaHeader = 128;  // CTA-wide words before the consumer regions
-// Per-consumer header: full mbarriers at 0, empty mbarriers at 32, column records for the
-// low 32 rows at 128 and for the high 32 rows at 640 (64 x {bits, address}), x~ at 1152
-// (64 columns x xt_stride(B) halves).
+// Per-consumer header: full mbarriers at 0, empty mbarriers at 32, column records at 128
+// (64 x 16 bytes), x~ at 1152 (64 columns x xt_stride(B) halves).
 constexpr int kFullOff = 0;
 constexpr int kEmptyOff = 32;
-constexpr int kRecLoOff = 128;
-constexpr int kRecHiOff = 640;
+constexpr int kRecOff = 128;
 constexpr int kXtOff = 1152;
 constexpr int kSmemPerSm = 227 * 1024;
 constexpr uint32_t kStageValsOff = 512;  // stage: 64 bitmap words, then packed values
@@ -82,6 +84,7 @@ struct SpmvParams {
     uint32_t stage_bytes;
     uint32_t warp_smem;
     float t;
+    int neg2;  // -2, passed at run time so the address step stays a multiply-add
 };
 
 __host__ __device__ constexpr int xt_stride(int B) {
@@ -207,37 +210,32 @@ __device__ inline void load_xg(const uint16_t* xt, int j, uint16_t (&xv)[G][B]) 
         for (int b = 0; b < B; b++) xv[c][b] = h[c * XS + b];
 }
 
-// G compacted active columns of one tile (G even), branch-free.  rech holds this lane's
-// half of each column record: {32 bitmap bits of the half, shared-memory address of the
-// half's first value}.  Every lane loads the two values at its rank whether or not its
-// bits are set (both addresses stay inside the stage), and the predicated multiply-adds
-// keep only the products of kept rows.
+// G compacted active columns of one tile, branch-free.  rec2 points at this lane's 8 bytes
+// of each 16-byte column record: {32 bitmap bits of the lane's half, shared-memory address
+// just past that half's packed values}.  Every lane loads its two candidate values whether
+// or not its bits are set (both addresses stay inside the stage), and the predicated
+// multiply-adds keep only the products of kept rows.
 template <int B, int G>
-__device__ inline void decode_pairs(const uint2* rech, const uint16_t* xt, int j, uint32_t below,
-                                    uint32_t bit0, uint32_t bit1, float* acc0, float* acc1) {
-    static_assert(G % 2 == 0, "records are loaded in pairs");
+__device__ inline void decode_cols(const uint2* rec2, const uint16_t* xt, int j, int sh, int neg2,
+                                   uint32_t bit0, uint32_t bit1, float* acc0, float* acc1) {
     uint2 r[G];
     uint16_t xv[G][B];
 #pragma unroll
-    for (int c = 0; c < G; c += 2) {
-        const uint4 q = *(const uint4*)(rech + j + c);
-        r[c] = make_uint2(q.x, q.y);
-        r[c + 1] = make_uint2(q.z, q.w);
-    }
+    for (int c = 0; c < G; c++) r[c] = rec2[2 * (j + c)];
     load_xg<B, G>(xt, j, xv);
     uint16_t v0[G], v1[G];
 #pragma unroll
     for (int c = 0; c < G; c++) {
-        const uint32_t a = r[c].y + 2u * __popc(r[c].x & below);
-        v0[c] = lds_u16(a);
-        v1[c] = lds_u16(a + 2u);
+        const int above = __popc(r[c].x >> sh);  // kept rows from 2l+1 up in this half
+        uint32_t a;                             // row 2l+1's value: end - 2 * above
+        asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(a) : "r"(above), "r"(neg2), "r"(r[c].y));
+        v1[c] = lds_u16(a);
+        v0[c] = lds_u16(a - 2u);
     }
 #pragma unroll
     for (int c = 0; c < G; c++) {
-        const uint32_t f0 = r[c].x & bit0, f1 = r[c].x & bit1;
-        const uint16_t u1 = f0 ? v1[c] : v0[c];  // row 2l+1 follows row 2l's value if kept
-        fma_rows<B>(f0, v0[c], xv[c], acc0);
-        fma_rows<B>(f1, u1, xv[c], acc1);
+        fma_rows<B>(r[c].x & bit0, v0[c], xv[c], acc0);
+        fma_rows<B>(r[c].x & bit1, v1[c], xv[c], acc1);
     }
 }
 
@@ -373,15 +371,16 @@ __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lan
     const int t_begin = (int)((long long)gw * T / PW);
     const int ntiles = (int)((long long)(gw + 1) * T / PW) - t_begin;
     const uint32_t reg_s = smem_u32(reg);
-    uint2* recL = (uint2*)(reg + kRecLoOff);
-    uint2* recH = (uint2*)(reg + kRecHiOff);
+    uint4* rec = (uint4*)(reg + kRecOff);
     uint16_t* xt = (uint16_t*)(reg + kXtOff);
     const uint32_t ltmask = lanemask_lt();
     // This lane's rows 2l and 2l+1 sit at bits q and q+1 of the low (lanes 0-15) or high
     // (lanes 16-31) 32 bits of a column's bitmap word.
     const int q = 2 * (lane & 15);
-    const uint32_t below = (1u << q) - 1u, bit0 = 1u << q, bit1 = 2u << q;
-    const uint2* rech = lane < 16 ? recL : recH;
+    const int sh = q + 1;
+    const uint32_t bit0 = 1u << q, bit1 = 2u << q;
+    const uint2* rec2 = (const uint2*)rec + (lane < 16 ? 0 : 1);  // this half's 8 bytes
+    const int neg2 = p.neg2;
 
     // Activations, column sets, outputs and the workspace only after the previous kernel
     // on the stream is complete.
@@ -451,14 +450,12 @@ __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lan
             const int pos0 = all ? 2 * lane : __popc(m0 & ltmask) + __popc(m1 & ltmask);
             const int pos1 = pos0 + ((all || any0) ? 1 : 0);
             if (any0) {
-                recL[pos0] = make_uint2(bw.x, a0);
-                recH[pos0] = make_uint2(bw.y, a0 + 2u * (uint32_t)cl0);
+                rec[pos0] = make_uint4(bw.x, a0 + 2u * (uint32_t)cl0, bw.y, a0 + 2u * (uint32_t)c0);
 #pragma unroll
                 for (int b = 0; b < B; b++) xt[pos0 * XS + b] = xa[b];
             }
             if (any1) {
-                recL[pos1] = make_uint2(bw.z, a1);
-                recH[pos1] = make_uint2(bw.w, a1 + 2u * (uint32_t)cl1);
+                rec[pos1] = make_uint4(bw.z, a1 + 2u * (uint32_t)cl1, bw.w, a1 + 2u * (uint32_t)c1);
 #pragma unroll
                 for (int b = 0; b < B; b++) xt[pos1 * XS + b] = xb[b];
             }
@@ -467,18 +464,17 @@ __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lan
                     __syncwarp();
 #pragma unroll
                     for (int j = 0; j < 64; j += kGroup)
-                        decode_pairs<B, kGroup>(rech, xt, j, below, bit0, bit1, acc0, acc1);
+                        decode_cols<B, kGroup>(rec2, xt, j, sh, neg2, bit0, bit1, acc0, acc1);
                 }
             }
             if (!all) {
                 const int n_pad = (n_act + kGroup - 1) & ~(kGroup - 1);
                 if (lane < n_pad - n_act) {
-                    recL[n_act + lane] = make_uint2(0u, vb);
-                    recH[n_act + lane] = make_uint2(0u, vb);
+                    rec[n_act + lane] = make_uint4(0u, vb, 0u, vb);
                 }
                 __syncwarp();
                 for (int j = 0; j < n_pad; j += kGroup)
-                    decode_pairs<B, kGroup>(rech, xt, j, below, bit0, bit1, acc0, acc1);
+                    decode_cols<B, kGroup>(rec2, xt, j, sh, neg2, bit0, bit1, acc0, acc1);
             }
         }
         pin_acc<B>(acc0, acc1);
@@ -745,6 +741,7 @@ int decode_group_launch(int n, const spw_format* hdrs, const void* const* bufs,
     prm.stage_bytes = pl.stage_bytes;
     prm.warp_smem = pl.warp_smem;
     prm.t = threshold;
+    prm.neg2 = -2;
     switch (B) {
 #define SPW_CASE(b) \
     case b: return launch<b>(pl, prm, s);
