@@ -219,7 +219,11 @@ int spw_spmv_noalloc(const spw_format* hdr, const void* d_buf, const uint16_t* d
                      int ldx, float threshold, const uint32_t* d_act_bits, uint16_t* d_y, int ldy,
                      void* stream);
 
-/* Workspace bytes spw_spmm needs (0 in this version; d_ws may then be NULL). */
+/* Workspace bytes spw_spmm needs for M rows of X on the current device: 0 when the output
+ * tiles fill the GPU (d_ws may then be NULL); otherwise K is split across CTAs and the
+ * workspace holds per-tile arrival counters (its first bytes: zero before the first call,
+ * left zero by every call that completes) and fp32 partial tiles.  0 for an invalid
+ * header or M < 1. */
 uint64_t spw_spmm_workspace_bytes(const spw_format* hdr, int M);
 
 /* Prefill SpMM ([SPDP] Tensor-Core SpMM; [3LF] §1: tensor cores take only 2:4 sparsity,
@@ -227,10 +231,31 @@ uint64_t spw_spmm_workspace_bytes(const spw_format* hdr, int M);
  *   Y[m,n] = sum_k X[m,k] W[n,k] mask[n,k],  m < M, n < N.
  * X: M x K fp16 (row stride ldx); Y: M x N fp16 (row stride ldy).  tcgen05 MMA with
  * fp32 accumulation in tensor memory, one round-to-nearest-even to fp16.  M >= 0
- * (M == 0 does nothing and then X and Y may be NULL).  Asynchronous.
- * Errors: INVALID_ARG, ALIGNMENT, FORMAT, CUDA; device timeouts as for spw_spmv. */
+ * (M == 0 does nothing and then X and Y may be NULL).  The decoded weight tile is the MMA's
+ * A operand (128 rows), X its B operand (up to 512 tokens per tile).  A dropped weight is
+ * an explicit zero in the product, so a non-finite X entry reaches every output row
+ * (0 * Inf = NaN, as in a dense product).  Deterministic.  Asynchronous.
+ * Errors: INVALID_ARG, ALIGNMENT, FORMAT, BUFFER_TOO_SMALL (workspace), CUDA; device
+ * timeouts as for spw_spmv. */
 int spw_spmm(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int M, int ldx,
              uint16_t* d_Y, int ldy, void* d_ws, uint64_t ws_bytes, void* stream);
+
+/* Workspace bytes spw_spmv_tc needs (the rules of spw_spmm_workspace_bytes with M = B);
+ * 0 for B outside 1..16. */
+uint64_t spw_spmv_tc_workspace_bytes(const spw_format* hdr, int B);
+
+/* Decode on tensor cores ([SPDP] reads "hybrid" as a runtime choice of decode path;
+ * [RMM] §4.2 reduced product): computes what spw_spmv computes -- same arguments, the
+ * threshold rule and column set applied to x in shared memory -- with the decoded weight
+ * tiles as the A operand of tcgen05 MMA (M = 128 weight rows, N = B rounded up to 16).
+ * Worth it for wide batches (B >= 8), where spw_spmv's per-row multiply-adds grow with
+ * B.  As in spw_spmm, a non-finite x~ entry reaches every row, including rows whose weight
+ * in that column is dropped.  Workspace: spw_spmv_tc_workspace_bytes (zero-initialised
+ * counters, left zero).  Inactive columns are decoded but contribute zeros.  Deterministic.
+ * Asynchronous.  Errors: as spw_spmv. */
+int spw_spmv_tc(const spw_format* hdr, const void* d_buf, const uint16_t* d_x, int B, int ldx,
+                float threshold, const uint32_t* d_act_bits, uint16_t* d_y, int ldy, void* d_ws,
+                uint64_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, then read and clear the library's device status word for the
  * current device: *code = SPW_OK, or SPW_ERR_TIMEOUT if a bounded device wait ran out

@@ -64,6 +64,8 @@ SIGNATURES = {
     "spw_spmv": ([_FP, _P, _P, _I, _I, _F, _P, _P, _I, _P, _U64, _P], _I),
     "spw_spmm_workspace_bytes": ([_FP, _I], _U64),
     "spw_spmm": ([_FP, _P, _P, _I, _I, _P, _I, _P, _U64, _P], _I),
+    "spw_spmv_tc_workspace_bytes": ([_FP, _I], _U64),
+    "spw_spmv_tc": ([_FP, _P, _P, _I, _I, _F, _P, _P, _I, _P, _U64, _P], _I),
     "spw_last_device_status": ([_P, _P], _I),
     "spw_spmv_group_workspace_bytes": ([_I, _FP, _I], _U64),
     "spw_spmv_group": ([_I, _FP, _P, _P, _P, _P, _P, _P, _I, _F, _P, _U64, _P], _I),
@@ -337,6 +339,32 @@ def spw_spmm(hdr, buf: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = N
         ctypes.byref(h), _ptr(buf), _ptr(X2), M, ldx, _ptr(Y2), ldy, _ptr(ws),
         0 if ws is None else ws.numel(), _stream(stream)))
     return Y
+
+
+def spw_spmv_tc_workspace_bytes(hdr, B: int) -> int:
+    h = _hdr(hdr)
+    return int(lib().spw_spmv_tc_workspace_bytes(ctypes.byref(h), int(B)))
+
+
+def spw_spmv_tc(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.0,
+                act_bits: torch.Tensor | None = None, y: torch.Tensor | None = None,
+                ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decode y (B x N fp16) on tensor cores; arguments as spw_spmv.  ws: a zero-initialised
+    uint8 workspace of spw_spmv_tc_workspace_bytes(hdr, B) bytes (allocated here when
+    needed and not given)."""
+    h = _hdr(hdr)
+    x2, ldx = _rows(_half(x, "x"), "x")
+    B = x2.shape[0]
+    if y is None:
+        y = torch.empty((B, h.N), dtype=torch.float16, device=x.device)
+    y2, ldy = _rows(_half(y, "y"), "y")
+    need = spw_spmv_tc_workspace_bytes(h, B)
+    if ws is None and need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=x.device)
+    _check("spw_spmv_tc", lib().spw_spmv_tc(
+        ctypes.byref(h), _ptr(buf), _ptr(x2), B, ldx, float(threshold), _ptr(act_bits),
+        _ptr(y2), ldy, _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return y
 
 
 def spw_last_device_status(stream=None) -> int:

@@ -1,4 +1,6 @@
-// spmm.cu -- prefill SpMM on tcgen05 tensor cores: Y = X . W_masked^T.
+// spmm.cu -- products on tcgen05 tensor cores with the compressed weight as the A operand:
+//   prefill  Y = X . W_masked^T            (spw_spmm, M tokens)
+//   decode   y_b = W_masked . x~_b         (spw_spmv_tc, B <= 16 rows, threshold rule)
 //
 // Method: "Unified Static-Dynamic Pruning for Efficient LLM Inference" (abstract) pairs
 // its bitmap format with a Tensor-Core SpMM for prefill.  Dense tensor cores take only
@@ -6,23 +8,36 @@
 // sparse weight matrices", §1, challenge 1), so unstructured tiles are decoded to dense
 // in shared memory and fed to dense MMA; the weight crosses HBM compressed.
 //
-// This library's design for B200 (one CTA per SM, one 256 x 256 output tile per CTA):
-//   * Y tile = 256 tokens (two M = 128 accumulators, 2 x 256 fp32 TMEM columns = all 512)
-//     by 256 weight rows (four 64-row TCB strips), K stepped by 64 (one TCB k-tile).
-//   * warp 0 (producer): TMA loads the X tile (256 x 64 fp16, 128-byte swizzle, no
-//     multicast) and 1-D bulk copies the four TCB tiles (bitmaps + packed values).
-//   * warp 1 (MMA): allocates TMEM; one thread issues tcgen05.mma.kind::f16 (A = X,
-//     B = decoded W, both K-major 128B-swizzled shared memory) and commits stage releases.
-//   * warps 2..9 (decoders, then epilogue): each owns one strip and 32 of its 64 columns;
-//     lane l produces rows l and l+32: the value of a kept weight sits at
-//     colstart + popc(bitmap & lanes_below); dense rows are written as 16-byte chunks in
-//     the swizzled layout the MMA reads.  After the K loop the same warps read the fp32
-//     accumulators (tcgen05.ld), round to fp16 and store Y.
+// This library's design for B200 (one output tile per CTA):
+//   * Output tile = 128 weight rows (two 64-row TCB strips; the MMA's M) by MT tokens or
+//     batch rows (the MMA's N: MT <= 256 in one MMA, 512 as two), K stepped by 64 (one
+//     TCB k-tile).  The fp32 accumulator, 128 lanes x MT columns, lives in TMEM.  Each
+//     decoded 64-column weight tile feeds up to 512 tokens.
+//   * When output tiles are fewer than the SMs can hold, K is split across CTAs: each
+//     stores its fp32 partial tile; the last CTA of a tile (counted with an atomic) sums
+//     the partials in K order -- deterministic -- and writes fp16.
+//   * warp 0 (producer): TMA loads the X tile (MT rows x 64, fp16, 128-byte swizzle, no
+//     multicast) and 1-D bulk-copies the two TCB tiles (bitmaps + packed values).
+//   * warp 1 (MMA): allocates TMEM; for decode all its lanes first apply the threshold
+//     rule (and the caller's column set) to the X tile in place; one thread issues
+//     tcgen05.mma.kind::f16 (A = decoded W, B = X, both K-major 128B-swizzled shared
+//     memory) and commits stage releases.
+//   * warps 2..9 (decoders, then epilogue): warp d decodes strip d/4, columns
+//     16 (d%4) .. 16 (d%4) + 15.  Lane l owns rows 2l and 2l+1 at bits q, q+1 (q = 2l mod
+//     32) of one half of each column's bitmap word; the kept rows from 2l+1 upward are the
+//     last c = popc(bits >> (q+1)) values of that half, so row 2l+1's value is at end - 2c
+//     and row 2l's just before it.  Dense rows are written as 16-byte chunks in the
+//     swizzled layout the MMA reads.  After the K loop the same warps read the fp32
+//     accumulators (tcgen05.ld) and write Y (or the split-K partials).
 //   * Every mbarrier wait is bounded and also polls a CTA-wide abort flag; on a timeout
 //     the kernel raises SPW_ERR_TIMEOUT, drains outstanding copies and MMAs (bounded),
 //     frees TMEM and returns.
+// A decoded tile holds explicit zeros where the mask drops a weight, so a non-finite
+// activation reaches every row through the MMA (0 * Inf = NaN, as in a dense product);
+// the CUDA-core decode (spmv.cu) skips dropped weights instead.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <string.h>
 
 #include <mutex>
 
@@ -31,29 +46,36 @@
 namespace spw {
 namespace {
 
-constexpr int kBM = 256;                // tokens per CTA tile (two M = 128 MMAs)
-constexpr int kBN = 256;                // weight rows per CTA tile (four strips)
+constexpr int kTileRows = 128;          // weight rows per CTA tile (the MMA's M)
+constexpr int kTileStrips = kTileRows / kStripRows;
 constexpr int kBK = 64;                 // one TCB k-tile
-constexpr int kStrips = kBN / kStripRows;
+constexpr int kMaxTokens = 512;         // tokens per CTA tile (TMEM columns)
 constexpr int kThreads = 320;           // 10 warps
 constexpr int kDecoderWarps = 8;
-constexpr uint32_t kXStageBytes = kBM * kBK * 2;  // 32 KB
-constexpr uint32_t kWStageBytes = kBN * kBK * 2;  // 32 KB
+constexpr uint32_t kWStageBytes = kTileRows * kBK * 2;  // 16 KB
 constexpr int kWStages = 2;
 constexpr int kSmemLimit = 227 * 1024;
-constexpr uint32_t kTmemCols = 512;
 
 struct SpmmParams {
     const uint64_t* bitmaps;
     const uint32_t* tileptr;
     const uint16_t* values;
     uint16_t* Y;
+    uint32_t* counters;         // split-K arrivals per output tile (ksplit > 1)
+    float* partials;            // split-K fp32 partial tiles
+    const uint32_t* act_bits;   // decode: caller's column set, or NULL
     int* status;
     int M, N, K, ldy;
     int n_strips, n_ktiles;
+    int MT, nh;                 // tokens per tile; MMAs per k-slice (MT / nh each)
+    int ksplit;
     int sx, sr;                 // X and raw-tile stage counts
-    uint32_t raw_stage_bytes;   // 2048 + 4 * val_slot
+    int rule;                   // decode: apply the threshold rule to X in shared memory
+    float t;
+    uint32_t x_stage_bytes;     // MT * 128
+    uint32_t raw_stage_bytes;   // 1024 + 2 * val_slot
     uint32_t val_slot;          // bytes per strip's values slot (incl. 16 bytes of slack)
+    uint32_t tmem_cols;
     uint32_t off_w, off_raw, off_rec, off_tptr, off_bar;  // dynamic smem offsets
 };
 
@@ -139,21 +161,44 @@ __device__ inline void flag_abort(volatile int* abort_flag, int* status) {
     raise_status(status, SPW_ERR_TIMEOUT);
 }
 
-__device__ inline uint32_t pack2(uint16_t lo, uint16_t hi) {
-    return (uint32_t)lo | ((uint32_t)hi << 16);
+
+
+// Threshold rule and column set applied in place to one X stage (decode): every lane
+// takes 16-byte chunks of the swizzled tile, rows b < MT, logical columns kt*64 + k.
+__device__ inline void apply_rule_to_x(const SpmmParams& p, unsigned char* xs, int kt, int lane) {
+    const int chunks = p.MT * 8;
+    for (int i = lane; i < chunks; i += 32) {
+        const int b = i >> 3, phys = i & 7;
+        const int k0 = kt * kBK + 8 * (phys ^ (b & 7));  // swizzle: chunk c sits at c ^ (b & 7)
+        uint4* ptr = (uint4*)(xs + (size_t)b * 128 + 16 * phys);
+        uint4 v = *ptr;
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 8; e++) {
+            const int k = k0 + e;
+            const uint16_t h = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
+            bool keep = k < p.K && passes_threshold(h, p.t);
+            if (p.act_bits && keep) keep = (__ldg(p.act_bits + (k >> 5)) >> (k & 31)) & 1u;
+            if (!keep) w[e >> 1] &= (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+        }
+        *ptr = make_uint4(w[0], w[1], w[2], w[3]);
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const SpmmParams p) {
+spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ SpmmParams p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the swizzled operand tiles
     unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * kBM;
-    const int n0 = blockIdx.y * kBN;
+    const int m0 = blockIdx.x * p.MT;
+    const int n0 = blockIdx.y * kTileRows;
     const int s0 = n0 / kStripRows;
     const int nk = p.n_ktiles;
+    const int kz = blockIdx.z;
+    const int k_begin = (int)((long long)kz * nk / p.ksplit);
+    const int k_end = (int)((long long)(kz + 1) * nk / p.ksplit);
     const int SX = p.sx, SR = p.sr;
 
     uint64_t* bars = (uint64_t*)(smem + p.off_bar);
@@ -167,6 +212,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const SpmmParams p) {
     uint64_t* drain = acc_full + 1;
     uint32_t* tmem_slot = (uint32_t*)(drain + 1);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+    volatile uint32_t* last_flag = (volatile uint32_t*)(tmem_slot + 2);
     uint32_t* tptr = (uint32_t*)(smem + p.off_tptr);
 
     if (threadIdx.x == 0) {
@@ -185,10 +231,11 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const SpmmParams p) {
         mbar_init(smem_u32(acc_full), 1);
         mbar_init(smem_u32(drain), 1);
         *abort_flag = 0;
+        *last_flag = 0;
         fence_mbar_init();
     }
     // tile pointers of the CTA's strips, for every k-tile (row j = strip s0 + j)
-    for (int i = threadIdx.x; i < kStrips * (nk + 1); i += kThreads) {
+    for (int i = threadIdx.x; i < kTileStrips * (nk + 1); i += kThreads) {
         const int j = i / (nk + 1), kt = i % (nk + 1);
         const int s = s0 + j;
         tptr[i] = (s < p.n_strips) ? __ldg(p.tileptr + (size_t)s * nk + kt) : 0u;
@@ -196,7 +243,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const SpmmParams p) {
     if (warp == 1) {  // TMEM allocation (whole warp)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
-                     "r"(kTmemCols)
+                     "r"(p.tmem_cols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -210,47 +257,51 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const SpmmParams p) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap_x) : "memory");
+            const int rows = p.MT / p.nh;  // TMA box height
             int xs = 0, rs = 0;
             uint32_t xph = 0, rph = 0;
-            for (int kt = 0; kt < nk; kt++) {
-                // X tile: rows m0..m0+255, columns 64 kt.. (zero fill outside X)
-                if (kt >= SX && !wait_or_abort(smem_u32(&x_empty[xs]), xph ^ 1u, abort_flag)) {
+            for (int kt = k_begin; kt < k_end; kt++) {
+                const int i = kt - k_begin;
+                // X tile: rows m0..m0+MT-1, columns 64 kt.. (zero fill outside X)
+                if (i >= SX && !wait_or_abort(smem_u32(&x_empty[xs]), xph ^ 1u, abort_flag)) {
                     flag_abort(abort_flag, p.status);
                     break;
                 }
                 const uint32_t xbar = smem_u32(&x_full[xs]);
-                mbar_arrive_expect_tx(xbar, kXStageBytes);
-                tma_load_2d(sbase + (uint32_t)xs * kXStageBytes, &tmap_x, kt * kBK, m0, xbar);
+                mbar_arrive_expect_tx(xbar, p.x_stage_bytes);
+                for (int h = 0; h < p.nh; h++)
+                    tma_load_2d(sbase + (uint32_t)xs * p.x_stage_bytes + (uint32_t)(h * rows * 128),
+                                &tmap_x, kt * kBK, m0 + h * rows, xbar);
                 x_issued++;
                 if (++xs == SX) { xs = 0; xph ^= 1u; }
-                // the four TCB tiles of this k-step
-                if (kt >= SR && !wait_or_abort(smem_u32(&r_empty[rs]), rph ^ 1u, abort_flag)) {
+                // the two TCB tiles of this k-step
+                if (i >= SR && !wait_or_abort(smem_u32(&r_empty[rs]), rph ^ 1u, abort_flag)) {
                     flag_abort(abort_flag, p.status);
                     break;
                 }
                 const uint32_t rbar = smem_u32(&r_full[rs]);
                 const uint32_t rst = sbase + p.off_raw + (uint32_t)rs * p.raw_stage_bytes;
-                uint32_t total = 0, vb[kStrips], u0[kStrips];
-                for (int j = 0; j < kStrips; j++) {
+                uint32_t total = 0, vb[kTileStrips], u0[kTileStrips];
+                for (int j = 0; j < kTileStrips; j++) {
                     vb[j] = 0;
                     u0[j] = 0;
                     if (s0 + j >= p.n_strips) continue;
                     u0[j] = tptr[j * (nk + 1) + kt];
-                    vb[j] = (tptr[j * (nk + 1) + kt + 1] - u0[j]) * 16u;
-                    if (vb[j] + 16u > p.val_slot) {  // larger than the header allows
+                    const uint32_t u1 = tptr[j * (nk + 1) + kt + 1];
+                    vb[j] = u1 >= u0[j] ? (u1 - u0[j]) * 16u : 0xFFFFFFFFu;
+                    if (vb[j] > p.val_slot - 16u) {  // larger than the header allows
                         raise_status(p.status, SPW_ERR_FORMAT);
                         vb[j] = 0;
                     }
                     total += 512u + vb[j];
                 }
-                fence_proxy_async_smem();
                 mbar_arrive_expect_tx(rbar, total);
-                for (int j = 0; j < kStrips; j++) {
+                for (int j = 0; j < kTileStrips; j++) {
                     if (s0 + j >= p.n_strips) continue;
                     const size_t t = (size_t)(s0 + j) * nk + kt;
                     bulk_g2s(rst + 512u * j, p.bitmaps + t * kTileCols, 512u, rbar);
                     if (vb[j])
-                        bulk_g2s(rst + 2048u + (uint32_t)j * p.val_slot, p.values + (size_t)u0[j] * 8,
+                        bulk_g2s(rst + 1024u + (uint32_t)j * p.val_slot, p.values + (size_t)u0[j] * 8,
                                  vb[j], rbar);
                 }
                 r_issued++;
@@ -259,104 +310,113 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const SpmmParams p) {
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = idesc_f16(128, kBN);
-            int xs = 0, ws = 0;
-            uint32_t xph = 0, wph = 0;
-            for (int kt = 0; kt < nk; kt++) {
-                if (!wait_or_abort(smem_u32(&x_full[xs]), xph, abort_flag) ||
-                    !wait_or_abort(smem_u32(&w_full[ws]), wph, abort_flag)) {
-                    flag_abort(abort_flag, p.status);
-                    break;
-                }
+        const uint32_t idesc = idesc_f16(kTileRows, p.MT / p.nh);
+        const uint32_t half_cols = (uint32_t)(p.MT / p.nh);
+        int xs = 0, ws = 0;
+        uint32_t xph = 0, wph = 0;
+        bool ok = true;
+        for (int kt = k_begin; kt < k_end && ok; kt++) {
+            ok = __all_sync(0xffffffffu, wait_or_abort(smem_u32(&x_full[xs]), xph, abort_flag));
+            if (ok && p.rule) {  // decode: x~ in place, before the tensor core reads it
+                apply_rule_to_x(p, smem + (size_t)xs * p.x_stage_bytes, kt, lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            ok = ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_full[ws]), wph, abort_flag));
+            if (!ok) {
+                if (lane == 0) flag_abort(abort_flag, p.status);
+                break;
+            }
+            if (lane == 0) {
                 tc_fence_after();
-                const uint32_t xa = sbase + (uint32_t)xs * kXStageBytes;
+                const uint32_t xa = sbase + (uint32_t)xs * p.x_stage_bytes;
                 const uint32_t wa = sbase + p.off_w + (uint32_t)ws * kWStageBytes;
 #pragma unroll
                 for (int j = 0; j < kBK / 16; j++) {
-                    const uint64_t bdesc = umma_desc_sw128(wa + 32u * j);
-#pragma unroll
-                    for (int h = 0; h < 2; h++) {
-                        const uint64_t adesc = umma_desc_sw128(xa + 16384u * h + 32u * j);
-                        umma_f16(tmem + 256u * h, adesc, bdesc, idesc, (kt > 0 || j > 0) ? 1u : 0u);
+                    const uint64_t adesc = umma_desc_sw128(wa + 32u * j);
+                    for (int h = 0; h < p.nh; h++) {
+                        const uint64_t bdesc = umma_desc_sw128(xa + half_cols * 128u * h + 32u * j);
+                        umma_f16(tmem + half_cols * h, adesc, bdesc, idesc,
+                                 (kt > k_begin || j > 0) ? 1u : 0u);
                     }
                 }
                 umma_commit(smem_u32(&x_empty[xs]));
                 umma_commit(smem_u32(&w_empty[ws]));
-                if (++xs == SX) { xs = 0; xph ^= 1u; }
-                if (++ws == kWStages) { ws = 0; wph ^= 1u; }
             }
+            __syncwarp();
+            if (++xs == SX) { xs = 0; xph ^= 1u; }
+            if (++ws == kWStages) { ws = 0; wph ^= 1u; }
+        }
+        if (lane == 0) {
             umma_commit(smem_u32(acc_full));
             umma_commit(smem_u32(drain));
             (void)mbar_wait(smem_u32(drain), 0);  // every issued MMA has completed
         }
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ decoders
         const int d = warp - 2;          // 0..7
-        const int q = d & 3;             // strip within the tile
-        const int h = d >> 2;            // column half
+        const int q = d >> 2;            // strip within the tile
+        const int g = d & 3;             // 16-column group
         const bool strip_ok = s0 + q < p.n_strips;
-        uint4* rec = (uint4*)(smem + p.off_rec + 512u * d);
-        const uint32_t lanebit = 1u << lane, ltmask = lanebit - 1u;
-        const uint32_t nl0 = 64u * q + lane, nl1 = nl0 + 32u;  // local W rows
+        uint4* rec = (uint4*)(smem + p.off_rec + 256u * d);  // 16 columns x 16 bytes
+        const int qb = 2 * (lane & 15);  // this lane's rows sit at bits qb, qb+1 of one half
+        const int sh = qb + 1;
+        const uint32_t bit0 = 1u << qb, bit1 = 2u << qb;
+        const uint2* rec2 = (const uint2*)rec + (lane < 16 ? 0 : 1);
+        const uint32_t nl0 = 64u * q + 2u * lane, nl1 = nl0 + 1u;  // local W rows
         int rs = 0, ws = 0;
         uint32_t rph = 0, wph = 0;
-        bool ok = true;
-        for (int kt = 0; kt < nk && ok; kt++) {
+        for (int kt = k_begin; kt < k_end; kt++) {
+            const int i = kt - k_begin;
             // every lane waits; __all_sync keeps the outcome warp-uniform
             if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&r_full[rs]), rph, abort_flag))) {
                 flag_abort(abort_flag, p.status);
                 break;
             }
-            const unsigned char* rst = smem + p.off_raw + (uint32_t)rs * p.raw_stage_bytes;
+            const uint32_t rst_s = sbase + p.off_raw + (uint32_t)rs * p.raw_stage_bytes;
             if (strip_ok) {
-                const uint64_t* bm = (const uint64_t*)(rst + 512u * q);
-                const uint64_t wa = bm[lane], wb = bm[lane + 32];
-                const int ca = __popcll(wa), cb = __popcll(wb);
-                const int sa = warp_inclusive_scan(ca, lane);
-                const int tot = __shfl_sync(0xffffffffu, sa, 31);
-                const int sb = warp_inclusive_scan(cb, lane);
-                const uint64_t w = h ? wb : wa;
-                const uint32_t start = (uint32_t)(h ? tot + sb - cb : sa - ca);
-                const uint32_t va = sbase + p.off_raw + (uint32_t)rs * p.raw_stage_bytes + 2048u +
-                                    (uint32_t)q * p.val_slot + 2u * start;
-                rec[lane] = make_uint4((uint32_t)w, (uint32_t)(w >> 32), va,
-                                       va + 2u * __popc((uint32_t)w));
+                // columns 2l and 2l+1 of the strip: counts, starts, and the records of the
+                // warp's 16 columns (lanes 8g .. 8g+7 hold them)
+                const uint4 bw = *(const uint4*)(smem + p.off_raw + (size_t)rs * p.raw_stage_bytes +
+                                                 512u * q + 16u * lane);
+                const int cl0 = __popc(bw.x), c0 = cl0 + __popc(bw.y);
+                const int cl1 = __popc(bw.z), c1 = cl1 + __popc(bw.w);
+                const int incl = warp_inclusive_scan(c0 + c1, lane);
+                const uint32_t vb = rst_s + 1024u + (uint32_t)q * p.val_slot;
+                const uint32_t a0 = vb + 2u * (uint32_t)(incl - c0 - c1);
+                const uint32_t a1 = a0 + 2u * (uint32_t)c0;
+                if ((lane >> 3) == g) {
+                    const int j = 2 * (lane & 7);
+                    rec[j] = make_uint4(bw.x, a0 + 2u * (uint32_t)cl0, bw.y, a1);
+                    rec[j + 1] = make_uint4(bw.z, a1 + 2u * (uint32_t)cl1, bw.w, a1 + 2u * (uint32_t)c1);
+                }
             }
             __syncwarp();
-            if (kt >= kWStages &&
+            if (i >= kWStages &&
                 !__all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_empty[ws]), wph ^ 1u, abort_flag))) {
                 flag_abort(abort_flag, p.status);
                 break;
             }
             unsigned char* wst = smem + p.off_w + (uint32_t)ws * kWStageBytes;
 #pragma unroll
-            for (int g = 0; g < 4; g++) {  // 8 columns -> one 16-byte chunk per row
-                uint32_t o0[4], o1[4];
+            for (int cc = 0; cc < 2; cc++) {  // 8 columns -> one 16-byte chunk per row
+                uint32_t o0[4] = {0u, 0u, 0u, 0u}, o1[4] = {0u, 0u, 0u, 0u};
                 if (strip_ok) {
-                    uint16_t v0[8], v1[8];
 #pragma unroll
                     for (int c = 0; c < 8; c++) {
-                        const uint4 r = rec[8 * g + c];
-                        const uint16_t a = lds_u16(r.z + 2u * __popc(r.x & ltmask));
-                        const uint16_t b = lds_u16(r.w + 2u * __popc(r.y & ltmask));
-                        v0[c] = (r.x & lanebit) ? a : (uint16_t)0;
-                        v1[c] = (r.y & lanebit) ? b : (uint16_t)0;
+                        const uint2 r = rec2[2 * (8 * cc + c)];
+                        uint32_t a;
+                        asm("mad.lo.s32 %0, %1, -2, %2;" : "=r"(a) : "r"(__popc(r.x >> sh)), "r"(r.y));
+                        const uint32_t v1 = lds_u16(a), v0 = lds_u16(a - 2u);
+                        const uint32_t sft = 16u * (uint32_t)(c & 1);
+                        o0[c >> 1] |= ((r.x & bit0) ? v0 : 0u) << sft;
+                        o1[c >> 1] |= ((r.x & bit1) ? v1 : 0u) << sft;
                     }
-#pragma unroll
-                    for (int c = 0; c < 4; c++) {
-                        o0[c] = pack2(v0[2 * c], v0[2 * c + 1]);
-                        o1[c] = pack2(v1[2 * c], v1[2 * c + 1]);
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 4; c++) o0[c] = o1[c] = 0u;
                 }
-                const uint32_t chunk = 4u * h + g;
-                *(uint4*)(wst + nl0 * 128u + ((chunk ^ (nl0 & 7u)) << 4)) =
-                    make_uint4(o0[0], o0[1], o0[2], o0[3]);
-                *(uint4*)(wst + nl1 * 128u + ((chunk ^ (nl1 & 7u)) << 4)) =
-                    make_uint4(o1[0], o1[1], o1[2], o1[3]);
+                const uint32_t chunk = 2u * g + cc;
+                *(uint4*)(wst + nl0 * 128u + ((chunk ^ (nl0 & 7u)) << 4)) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+                *(uint4*)(wst + nl1 * 128u + ((chunk ^ (nl1 & 7u)) << 4)) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
             }
             fence_proxy_async_smem();  // generic-proxy stores -> tensor-core reads
             __syncwarp();
@@ -373,31 +433,32 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const SpmmParams p) {
             __all_sync(0xffffffffu, !*abort_flag && wait_or_abort(smem_u32(acc_full), 0, abort_flag));
         if (acc_ready) {
             tc_fence_after();
-            const int quarter = warp & 3;           // TMEM lanes this warp may access
-            const int acc = (warp - 2) >> 2;        // accumulator 0 (warps 2-5) or 1 (6-9)
-            const int m = m0 + 128 * acc + 32 * quarter + lane;
-            const bool vec = (p.ldy % 8) == 0;
-            for (int j = 0; j < kBN / 32; j++) {
+            const int quarter = warp & 3;       // TMEM lanes this warp may access
+            const int half = (warp - 2) >> 2;   // which 32-column chunks: j % 2 == half
+            const int row = 32 * quarter + lane;
+            const int n = n0 + row;
+            const size_t tile = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+            float* part = p.partials + (tile * p.ksplit + kz) * (size_t)p.MT * kTileRows;
+            // 32 accumulator columns per load; the allocation is a power of two >= 32, so a
+            // tile of 16 tokens reads 16 valid columns and 16 unused ones.
+            for (int j = half; j < (p.MT + 31) / 32; j += 2) {
                 uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + 256u * acc + 32u * j, r);
-                const int n = n0 + 32 * j;
-                if (m >= p.M || n >= p.N) continue;
-                uint16_t* yrow = p.Y + (size_t)m * p.ldy + n;
-                uint32_t packed[16];
+                tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + 32u * j, r);
+                const int lim = min(32, p.MT - 32 * j);
+                if (p.ksplit > 1) {
 #pragma unroll
-                for (int c = 0; c < 16; c++)
-                    packed[c] = pack2(__half_as_ushort(__float2half_rn(__uint_as_float(r[2 * c]))),
-                                      __half_as_ushort(__float2half_rn(__uint_as_float(r[2 * c + 1]))));
-                if (vec && n + 32 <= p.N) {
+                    for (int c = 0; c < 32; c++)
+                        if (c < lim) part[(size_t)(32 * j + c) * kTileRows + row] = __uint_as_float(r[c]);
+                } else if (n < p.N) {
 #pragma unroll
-                    for (int c = 0; c < 4; c++)
-                        *(uint4*)(yrow + 8 * c) = make_uint4(packed[4 * c], packed[4 * c + 1],
-                                                             packed[4 * c + 2], packed[4 * c + 3]);
-                } else {
-                    const int lim = min(32, p.N - n);
-                    for (int c = 0; c < lim; c++) yrow[c] = (uint16_t)(packed[c >> 1] >> (16 * (c & 1)));
+                    for (int c = 0; c < 32; c++) {
+                        const int m = m0 + 32 * j + c;
+                        if (c < lim && m < p.M)
+                            p.Y[(size_t)m * p.ldy + n] = __half_as_ushort(__float2half_rn(__uint_as_float(r[c])));
+                    }
                 }
             }
+            if (p.ksplit > 1) __threadfence();  // partials before the arrival below
         } else {
             flag_abort(abort_flag, p.status);
         }
@@ -405,6 +466,27 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const SpmmParams p) {
 
     tc_fence_before();
     __syncthreads();
+    if (p.ksplit > 1 && !*abort_flag) {
+        // Split-K: the last CTA of this output tile sums every partial in K order.
+        const size_t tile = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+        if (threadIdx.x == 0) {
+            const uint32_t old = atom_add_release_gpu(&p.counters[tile], 1u);
+            *last_flag = old == (uint32_t)(p.ksplit - 1) ? 1u : 0u;
+            if (*last_flag) p.counters[tile] = 0u;
+        }
+        __syncthreads();
+        if (*last_flag) {
+            __threadfence();
+            const float* base = p.partials + tile * p.ksplit * (size_t)p.MT * kTileRows;
+            for (int idx = threadIdx.x; idx < p.MT * kTileRows; idx += kThreads) {
+                const int tok = idx / kTileRows, row = idx % kTileRows;
+                const int m = m0 + tok, n = n0 + row;
+                float s = 0.0f;
+                for (int z = 0; z < p.ksplit; z++) s += __ldcg(base + (size_t)z * p.MT * kTileRows + idx);
+                if (m < p.M && n < p.N) p.Y[(size_t)m * p.ldy + n] = __half_as_ushort(__float2half_rn(s));
+            }
+        }
+    }
     if (warp == 0 && lane == 0 && *abort_flag) {
         // Drain the copies this CTA armed (bounded): for each slot, the phase of its
         // last issue.  Phases a consumer already waited for return at once.
@@ -421,12 +503,16 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const SpmmParams p) {
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                     "r"(kTmemCols)
+                     "r"(p.tmem_cols)
                      : "memory");
     }
 }
 
+}  // namespace
+
 // ------------------------------------------------------------------ host side
+namespace {
+
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::mutex g_encode_mutex;
 
@@ -444,22 +530,37 @@ int get_encoder() {
 }
 
 struct SpmmPlan {
-    int sx, sr;
-    uint32_t val_slot, raw_stage_bytes, off_w, off_raw, off_rec, off_tptr, off_bar;
+    int MT, nh, m_tiles, n_tiles, ksplit, sx, sr, ctas_per_sm;
+    uint32_t x_stage_bytes, val_slot, raw_stage_bytes, tmem_cols;
+    uint32_t off_w, off_raw, off_rec, off_tptr, off_bar;
     size_t smem;
+    uint64_t ws_counters, ws_bytes;
 };
 
-int make_spmm_plan(const spw_format* h, SpmmPlan* pl) {
+// Token tile, split-K factor, stage counts and shared-memory layout for M rows of X.
+int make_spmm_plan(const spw_format* h, int M, SpmmPlan* pl) {
+    const int sms = device_sm_count();
+    if (sms <= 0) return SPW_ERR_CUDA;
+    pl->m_tiles = (M + kMaxTokens - 1) / kMaxTokens;
+    const int per = (M + pl->m_tiles - 1) / pl->m_tiles;
+    pl->nh = per > 256 ? 2 : 1;
+    pl->MT = (int)round_up_u64((uint64_t)per, 16u * pl->nh);  // each MMA's N a multiple of 16
+    pl->n_tiles = (int)((h->N + kTileRows - 1) / kTileRows);
+    pl->x_stage_bytes = (uint32_t)pl->MT * 128u;
+    uint32_t cols = 32;
+    while (cols < (uint32_t)pl->MT) cols <<= 1;
+    pl->tmem_cols = cols;
     pl->val_slot = (uint32_t)round_up_u64(16ull * h->max_tile_units + 16, 16);
-    pl->raw_stage_bytes = 2048u + (uint32_t)kStrips * pl->val_slot;
-    const uint32_t tptr_bytes = (uint32_t)round_up_u64(4ull * kStrips * (h->n_ktiles + 1), 16);
+    pl->raw_stage_bytes = 1024u + (uint32_t)kTileStrips * pl->val_slot;
+    const uint32_t tptr_bytes = (uint32_t)round_up_u64(4ull * kTileStrips * (h->n_ktiles + 1), 16);
     const int options[][2] = {{4, 4}, {4, 3}, {3, 3}, {3, 2}, {2, 3}, {2, 2}};
+    bool found = false;
     for (const auto& o : options) {
         const int sx = o[0], sr = o[1];
-        const uint32_t off_w = (uint32_t)sx * kXStageBytes;
+        const uint32_t off_w = (uint32_t)sx * pl->x_stage_bytes;
         const uint32_t off_raw = off_w + (uint32_t)kWStages * kWStageBytes;
         const uint32_t off_rec = off_raw + (uint32_t)sr * pl->raw_stage_bytes;
-        const uint32_t off_tptr = off_rec + 512u * kDecoderWarps;
+        const uint32_t off_tptr = off_rec + 256u * kDecoderWarps;
         const uint32_t off_bar = (uint32_t)round_up_u64(off_tptr + tptr_bytes, 8);
         const uint32_t bar_bytes = 8u * (2 * sx + 2 * sr + 2 * kWStages + 2) + 16u;
         const size_t total = (size_t)off_bar + bar_bytes + 1024;  // + base alignment slack
@@ -472,39 +573,38 @@ int make_spmm_plan(const spw_format* h, SpmmPlan* pl) {
             pl->off_tptr = off_tptr;
             pl->off_bar = off_bar;
             pl->smem = total;
-            return SPW_OK;
+            found = true;
+            break;
         }
     }
-    return SPW_ERR_UNSUPPORTED;
+    if (!found) return SPW_ERR_UNSUPPORTED;
+    // Split K when the output tiles cannot fill the SMs (two k-tiles per split at least).
+    pl->ctas_per_sm = 1;  // 320 threads at ~120 registers: one CTA per SM
+    const long long tiles = (long long)pl->m_tiles * pl->n_tiles;
+    const long long slots = (long long)sms * pl->ctas_per_sm;
+    long long ks = tiles >= slots ? 1 : slots / tiles;
+    const long long kmax = h->n_ktiles / 2 > 0 ? h->n_ktiles / 2 : 1;
+    if (ks > kmax) ks = kmax;
+    pl->ksplit = (int)ks;
+    pl->ws_counters = pl->ksplit > 1 ? round_up_u64(4ull * (uint64_t)tiles, 256) : 0;
+    pl->ws_bytes = pl->ksplit > 1
+                       ? pl->ws_counters + 4ull * (uint64_t)tiles * pl->ksplit * pl->MT * kTileRows
+                       : 0;
+    return SPW_OK;
 }
 
-}  // namespace
-}  // namespace spw
-
-using namespace spw;
-
-extern "C" {
-
-uint64_t spw_spmm_workspace_bytes(const spw_format* hdr, int M) {
-    (void)hdr;
-    (void)M;
-    return 0;
-}
-
-int spw_spmm(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int M, int ldx,
-             uint16_t* d_Y, int ldy, void* d_ws, uint64_t ws_bytes, void* stream) {
-    int rc = check_header(hdr);
-    if (rc != SPW_OK) return rc;
-    if (M < 0) return SPW_ERR_INVALID_ARG;
-    if (M == 0) return SPW_OK;  // nothing to compute; X and Y may be NULL
-    if (!d_buf || !d_X || !d_Y) return SPW_ERR_INVALID_ARG;
-    if (!ld_ok(ldx, (int)hdr->K, M) || ldy < (int)hdr->N) return SPW_ERR_INVALID_ARG;
-    if (!aligned16(d_buf) || !aligned16(d_X) || !aligned16(d_Y)) return SPW_ERR_ALIGNMENT;
-    (void)d_ws;
-    (void)ws_bytes;
+// Shared by spw_spmm and spw_spmv_tc: checks, tensor map, launch.
+int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int M, int ldx,
+               uint16_t* d_Y, int ldy, int rule, float t, const uint32_t* act_bits, void* d_ws,
+               uint64_t ws_bytes, cudaStream_t stream) {
     SpmmPlan pl;
-    rc = make_spmm_plan(hdr, &pl);
+    int rc = make_spmm_plan(hdr, M, &pl);
     if (rc != SPW_OK) return rc;
+    if (pl.ws_bytes) {
+        if (!d_ws) return SPW_ERR_INVALID_ARG;
+        if (ws_bytes < pl.ws_bytes) return SPW_ERR_BUFFER_TOO_SMALL;
+        if (!aligned16(d_ws)) return SPW_ERR_ALIGNMENT;
+    }
     rc = get_encoder();
     if (rc != SPW_OK) return rc;
     int* status = device_status_ptr();
@@ -515,7 +615,7 @@ int spw_spmm(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int 
     const cuuint64_t dims[2] = {(cuuint64_t)hdr->K, (cuuint64_t)M};
     const cuuint64_t ld_bytes = (cuuint64_t)((M > 1 ? ldx : ((ldx + 7) / 8 * 8)) * 2);
     const cuuint64_t strides[1] = {ld_bytes};
-    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBM};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)(pl.MT / pl.nh)};
     const cuuint32_t estr[2] = {1, 1};
     CUresult cr = g_encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)d_X, dims, strides, box,
                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -524,10 +624,14 @@ int spw_spmm(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int 
 
     const uint8_t* buf = (const uint8_t*)d_buf;
     SpmmParams prm;
+    memset(&prm, 0, sizeof(prm));
     prm.bitmaps = (const uint64_t*)(buf + hdr->off_bitmaps);
     prm.tileptr = (const uint32_t*)(buf + hdr->off_tileptr);
     prm.values = (const uint16_t*)(buf + hdr->off_values);
     prm.Y = d_Y;
+    prm.counters = pl.ws_bytes ? (uint32_t*)d_ws : nullptr;
+    prm.partials = pl.ws_bytes ? (float*)((uint8_t*)d_ws + pl.ws_counters) : nullptr;
+    prm.act_bits = act_bits;
     prm.status = status;
     prm.M = M;
     prm.N = (int)hdr->N;
@@ -535,10 +639,17 @@ int spw_spmm(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int 
     prm.ldy = ldy;
     prm.n_strips = (int)hdr->n_strips;
     prm.n_ktiles = (int)hdr->n_ktiles;
+    prm.MT = pl.MT;
+    prm.nh = pl.nh;
+    prm.ksplit = pl.ksplit;
     prm.sx = pl.sx;
     prm.sr = pl.sr;
+    prm.rule = rule;
+    prm.t = t;
+    prm.x_stage_bytes = pl.x_stage_bytes;
     prm.raw_stage_bytes = pl.raw_stage_bytes;
     prm.val_slot = pl.val_slot;
+    prm.tmem_cols = pl.tmem_cols;
     prm.off_w = pl.off_w;
     prm.off_raw = pl.off_raw;
     prm.off_rec = pl.off_rec;
@@ -554,11 +665,57 @@ int spw_spmm(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int 
                                           (int)pl.smem));
         attr_smem[dev] = pl.smem;
     }
-    const dim3 grid((M + kBM - 1) / kBM, (hdr->N + kBN - 1) / kBN);
-    if (grid.y > 65535u) return SPW_ERR_UNSUPPORTED;
-    spmm_kernel<<<grid, kThreads, pl.smem, (cudaStream_t)stream>>>(tmap, prm);
+    if (pl.n_tiles > 65535 || pl.ksplit > 65535) return SPW_ERR_UNSUPPORTED;
+    const dim3 grid(pl.m_tiles, pl.n_tiles, pl.ksplit);
+    spmm_kernel<<<grid, kThreads, pl.smem, stream>>>(tmap, prm);
     SPW_LAUNCH_CHECK();
     return SPW_OK;
+}
+
+}  // namespace
+}  // namespace spw
+
+using namespace spw;
+
+extern "C" {
+
+uint64_t spw_spmm_workspace_bytes(const spw_format* hdr, int M) {
+    if (check_header(hdr) != SPW_OK || M < 1) return 0;
+    SpmmPlan pl;
+    if (make_spmm_plan(hdr, M, &pl) != SPW_OK) return 0;
+    return pl.ws_bytes;
+}
+
+int spw_spmm(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int M, int ldx,
+             uint16_t* d_Y, int ldy, void* d_ws, uint64_t ws_bytes, void* stream) {
+    int rc = check_header(hdr);
+    if (rc != SPW_OK) return rc;
+    if (M < 0) return SPW_ERR_INVALID_ARG;
+    if (M == 0) return SPW_OK;  // nothing to compute; X and Y may be NULL
+    if (!d_buf || !d_X || !d_Y) return SPW_ERR_INVALID_ARG;
+    if (!ld_ok(ldx, (int)hdr->K, M) || ldy < (int)hdr->N) return SPW_ERR_INVALID_ARG;
+    if (!aligned16(d_buf) || !aligned16(d_X) || !aligned16(d_Y)) return SPW_ERR_ALIGNMENT;
+    return tc_product(hdr, d_buf, d_X, M, ldx, d_Y, ldy, 0, 0.0f, nullptr, d_ws, ws_bytes,
+                      (cudaStream_t)stream);
+}
+
+uint64_t spw_spmv_tc_workspace_bytes(const spw_format* hdr, int B) {
+    if (B < 1 || B > 16) return 0;
+    return spw_spmm_workspace_bytes(hdr, B);
+}
+
+int spw_spmv_tc(const spw_format* hdr, const void* d_buf, const uint16_t* d_x, int B, int ldx,
+                float threshold, const uint32_t* d_act_bits, uint16_t* d_y, int ldy, void* d_ws,
+                uint64_t ws_bytes, void* stream) {
+    int rc = check_header(hdr);
+    if (rc != SPW_OK) return rc;
+    if (B < 1 || B > 16 || !d_buf || !d_x || !d_y) return SPW_ERR_INVALID_ARG;
+    if (!(threshold >= 0.0f) || isinf(threshold)) return SPW_ERR_INVALID_ARG;
+    if (!ld_ok(ldx, (int)hdr->K, B) || ldy < (int)hdr->N) return SPW_ERR_INVALID_ARG;
+    if (!aligned16(d_buf) || !aligned16(d_x) || !aligned16(d_y) || !aligned16(d_act_bits))
+        return SPW_ERR_ALIGNMENT;
+    return tc_product(hdr, d_buf, d_x, B, ldx, d_y, ldy, 1, threshold, d_act_bits, d_ws, ws_bytes,
+                      (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -36,7 +36,8 @@ import sys
 import numpy as np
 import torch
 
-from . import SparseLinear, spw_last_device_status, spw_select_topk, spw_spmm, spw_spmv
+from . import (SparseLinear, spw_last_device_status, spw_select_topk, spw_spmm, spw_spmv,
+               spw_spmv_tc, spw_spmv_tc_workspace_bytes)
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
@@ -133,6 +134,13 @@ def _decode_point(layer: _Layer, x: np.ndarray, t: float, act_bits=None) -> dict
     us = _time_rotating(calls)
     assert spw_last_device_status() == 0
     out = {"sparse_us": round(us, 3)}
+    if B >= 4:  # the tensor-core decode path as well
+        need = spw_spmv_tc_workspace_bytes(layer.lin.hdr, B)
+        tws = [torch.zeros(max(16, need), dtype=torch.uint8, device="cuda") for _ in layer.bufs]
+        tcalls = [(lambda r=r: spw_spmv_tc(layer.lin.hdr, layer.bufs[r], xd, t, act_bits, ys[r],
+                                           tws[r])) for r in range(len(layer.bufs))]
+        out["tc_us"] = round(_time_rotating(tcalls), 3)
+        assert spw_last_device_status() == 0
     if layer.dense is not None:
         yd = [torch.empty((B, layer.N), dtype=torch.float16, device="cuda") for _ in layer.dense]
         dcalls = [(lambda r=r: torch.matmul(xd, layer.dense[r].t(), out=yd[r]))
