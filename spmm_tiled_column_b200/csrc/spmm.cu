@@ -12,18 +12,23 @@
 //   * Output tile = 128 weight rows (two 64-row TCB strips; the MMA's M) by MT tokens or
 //     batch rows (the MMA's N: MT <= 256 in one MMA, 512 as two), K stepped by 64 (one
 //     TCB k-tile).  The fp32 accumulator, 128 lanes x MT columns, lives in TMEM.  Each
-//     decoded 64-column weight tile feeds up to 512 tokens.
+//     decoded 64-column weight tile feeds up to 512 tokens.  For narrow tiles (decode
+//     batches, MT <= 32) the 16-wide k-slices rotate over 4 accumulators, so the MMAs
+//     form 4 independent chains instead of one; the epilogue adds them.
 //   * When output tiles are fewer than the SMs can hold, K is split across CTAs: each
 //     stores its fp32 partial tile; the last CTA of a tile (counted with an atomic) sums
 //     the partials in K order -- deterministic -- and writes fp16.
-//   * warp 0 (producer): TMA loads the X tile (MT rows x 64, fp16, 128-byte swizzle, no
-//     multicast) and 1-D bulk-copies the two TCB tiles (bitmaps + packed values).
-//   * warp 1 (MMA): allocates TMEM; for decode all its lanes first apply the threshold
-//     rule (and the caller's column set) to the X tile in place; one thread issues
-//     tcgen05.mma.kind::f16 (A = decoded W, B = X, both K-major 128B-swizzled shared
-//     memory) and commits stage releases.
-//   * warps 2..9 (decoders, then epilogue): warp d decodes strip d/4, columns
-//     16 (d%4) .. 16 (d%4) + 15.  Lane l owns rows 2l and 2l+1 at bits q, q+1 (q = 2l mod
+//   * warp 0 (producer): lane 0 TMA-loads the X tiles (MT rows x 64, fp16, 128-byte
+//     swizzle, no multicast); lane 1, independently, 1-D bulk-copies the two TCB tiles
+//     (bitmaps + packed values) of each k-step.
+//   * warp 1 (MMA): allocates TMEM; one thread issues tcgen05.mma.kind::f16 (A = decoded
+//     W, B = X, both K-major 128B-swizzled shared memory) and commits stage releases.
+//   * Decode (spw_spmv_tc) with a threshold above zero or a column set first writes x~ to
+//     the workspace with a small kernel (rule_kernel); with threshold 0 and no column set
+//     x~ differs from x only in dropping exact zeros, which contribute nothing, and X is
+//     read as given.
+//   * warps 2..17 (decoders, then epilogue): warp d decodes strip d/8, columns
+//     8 (d%8) .. 8 (d%8) + 7, one 16-byte chunk of each of its rows.  Lane l owns rows 2l and 2l+1 at bits q, q+1 (q = 2l mod
 //     32) of one half of each column's bitmap word; the kept rows from 2l+1 upward are the
 //     last c = popc(bits >> (q+1)) values of that half, so row 2l+1's value is at end - 2c
 //     and row 2l's just before it.  Dense rows are written as 16-byte chunks in the
@@ -50,10 +55,9 @@ constexpr int kTileRows = 128;          // weight rows per CTA tile (the MMA's M
 constexpr int kTileStrips = kTileRows / kStripRows;
 constexpr int kBK = 64;                 // one TCB k-tile
 constexpr int kMaxTokens = 512;         // tokens per CTA tile (TMEM columns)
-constexpr int kThreads = 320;           // 10 warps
-constexpr int kDecoderWarps = 8;
+constexpr int kDecoderWarps = 16;
+constexpr int kThreads = 32 * (2 + kDecoderWarps);      // producer, MMA, decoders
 constexpr uint32_t kWStageBytes = kTileRows * kBK * 2;  // 16 KB
-constexpr int kWStages = 2;
 constexpr int kSmemLimit = 227 * 1024;
 
 struct SpmmParams {
@@ -63,15 +67,13 @@ struct SpmmParams {
     uint16_t* Y;
     uint32_t* counters;         // split-K arrivals per output tile (ksplit > 1)
     float* partials;            // split-K fp32 partial tiles
-    const uint32_t* act_bits;   // decode: caller's column set, or NULL
     int* status;
     int M, N, K, ldy;
     int n_strips, n_ktiles;
     int MT, nh;                 // tokens per tile; MMAs per k-slice (MT / nh each)
+    int n_acc;                  // independent accumulators (32 columns apart) for MT <= 32
     int ksplit;
-    int sx, sr;                 // X and raw-tile stage counts
-    int rule;                   // decode: apply the threshold rule to X in shared memory
-    float t;
+    int sx, sr, sw;             // X, raw-tile and decoded-weight stage counts
     uint32_t x_stage_bytes;     // MT * 128
     uint32_t raw_stage_bytes;   // 1024 + 2 * val_slot
     uint32_t val_slot;          // bytes per strip's values slot (incl. 16 bytes of slack)
@@ -163,26 +165,34 @@ __device__ inline void flag_abort(volatile int* abort_flag, int* status) {
 
 
 
-// Threshold rule and column set applied in place to one X stage (decode): every lane
-// takes 16-byte chunks of the swizzled tile, rows b < MT, logical columns kt*64 + k.
-__device__ inline void apply_rule_to_x(const SpmmParams& p, unsigned char* xs, int kt, int lane) {
-    const int chunks = p.MT * 8;
-    for (int i = lane; i < chunks; i += 32) {
-        const int b = i >> 3, phys = i & 7;
-        const int k0 = kt * kBK + 8 * (phys ^ (b & 7));  // swizzle: chunk c sits at c ^ (b & 7)
-        uint4* ptr = (uint4*)(xs + (size_t)b * 128 + 16 * phys);
-        uint4 v = *ptr;
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// Decode's x~ for the tensor-core path: the threshold rule and the caller's column set
+// applied once per call, into the workspace (B rows of ld halves), 8 halves per thread.
+__global__ void __launch_bounds__(256) rule_kernel(const uint16_t* __restrict__ x, int ldx, int B, int K,
+                                                   float t, const uint32_t* __restrict__ act_bits,
+                                                   uint16_t* __restrict__ xt, int ld) {
+    const int per_row = (K + 7) / 8;
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= B * per_row) return;
+    const int b = i / per_row, k0 = 8 * (i % per_row);
+    uint16_t out[8];
 #pragma unroll
-        for (int e = 0; e < 8; e++) {
-            const int k = k0 + e;
-            const uint16_t h = (uint16_t)(w[e >> 1] >> (16 * (e & 1)));
-            bool keep = k < p.K && passes_threshold(h, p.t);
-            if (p.act_bits && keep) keep = (__ldg(p.act_bits + (k >> 5)) >> (k & 31)) & 1u;
-            if (!keep) w[e >> 1] &= (e & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+    for (int e = 0; e < 8; e++) {
+        const int k = k0 + e;
+        uint16_t v = 0;
+        if (k < K) {
+            v = x[(size_t)b * ldx + k];
+            bool keep = passes_threshold(v, t);
+            if (act_bits && keep) keep = (act_bits[k >> 5] >> (k & 31)) & 1u;
+            if (!keep) v = 0;
         }
-        *ptr = make_uint4(w[0], w[1], w[2], w[3]);
+        out[e] = v;
     }
+    uint4 w;
+    w.x = (uint32_t)out[0] | ((uint32_t)out[1] << 16);
+    w.y = (uint32_t)out[2] | ((uint32_t)out[3] << 16);
+    w.z = (uint32_t)out[4] | ((uint32_t)out[5] << 16);
+    w.w = (uint32_t)out[6] | ((uint32_t)out[7] << 16);
+    *(uint4*)(xt + (size_t)b * ld + k0) = w;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -206,9 +216,10 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     uint64_t* x_empty = x_full + SX;
     uint64_t* r_full = x_empty + SX;
     uint64_t* r_empty = r_full + SR;
+    const int SW = p.sw;
     uint64_t* w_full = r_empty + SR;
-    uint64_t* w_empty = w_full + kWStages;
-    uint64_t* acc_full = w_empty + kWStages;
+    uint64_t* w_empty = w_full + SW;
+    uint64_t* acc_full = w_empty + SW;
     uint64_t* drain = acc_full + 1;
     uint32_t* tmem_slot = (uint32_t*)(drain + 1);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
@@ -224,7 +235,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             mbar_init(smem_u32(&r_full[i]), 1);
             mbar_init(smem_u32(&r_empty[i]), kDecoderWarps);
         }
-        for (int i = 0; i < kWStages; i++) {
+        for (int i = 0; i < SW; i++) {
             mbar_init(smem_u32(&w_full[i]), kDecoderWarps);
             mbar_init(smem_u32(&w_empty[i]), 1);
         }
@@ -252,18 +263,17 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    int x_issued = 0, r_issued = 0;  // producer lane 0: stages armed on each ring
+    int x_issued = 0, r_issued = 0;  // producer lanes 0 (X) and 1 (TCB): stages armed
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
+        if (lane == 0) {  // X ring
             asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap_x) : "memory");
             const int rows = p.MT / p.nh;  // TMA box height
-            int xs = 0, rs = 0;
-            uint32_t xph = 0, rph = 0;
+            int xs = 0;
+            uint32_t xph = 0;
             for (int kt = k_begin; kt < k_end; kt++) {
-                const int i = kt - k_begin;
                 // X tile: rows m0..m0+MT-1, columns 64 kt.. (zero fill outside X)
-                if (i >= SX && !wait_or_abort(smem_u32(&x_empty[xs]), xph ^ 1u, abort_flag)) {
+                if (kt - k_begin >= SX && !wait_or_abort(smem_u32(&x_empty[xs]), xph ^ 1u, abort_flag)) {
                     flag_abort(abort_flag, p.status);
                     break;
                 }
@@ -274,8 +284,12 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                                 &tmap_x, kt * kBK, m0 + h * rows, xbar);
                 x_issued++;
                 if (++xs == SX) { xs = 0; xph ^= 1u; }
-                // the two TCB tiles of this k-step
-                if (i >= SR && !wait_or_abort(smem_u32(&r_empty[rs]), rph ^ 1u, abort_flag)) {
+            }
+        } else if (lane == 1) {  // TCB ring: the two tiles of each k-step
+            int rs = 0;
+            uint32_t rph = 0;
+            for (int kt = k_begin; kt < k_end; kt++) {
+                if (kt - k_begin >= SR && !wait_or_abort(smem_u32(&r_empty[rs]), rph ^ 1u, abort_flag)) {
                     flag_abort(abort_flag, p.status);
                     break;
                 }
@@ -317,11 +331,6 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         bool ok = true;
         for (int kt = k_begin; kt < k_end && ok; kt++) {
             ok = __all_sync(0xffffffffu, wait_or_abort(smem_u32(&x_full[xs]), xph, abort_flag));
-            if (ok && p.rule) {  // decode: x~ in place, before the tensor core reads it
-                apply_rule_to_x(p, smem + (size_t)xs * p.x_stage_bytes, kt, lane);
-                fence_proxy_async_smem();
-                __syncwarp();
-            }
             ok = ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_full[ws]), wph, abort_flag));
             if (!ok) {
                 if (lane == 0) flag_abort(abort_flag, p.status);
@@ -334,10 +343,12 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 #pragma unroll
                 for (int j = 0; j < kBK / 16; j++) {
                     const uint64_t adesc = umma_desc_sw128(wa + 32u * j);
+                    const int slice = (kt - k_begin) * (kBK / 16) + j;
+                    const uint32_t acc = p.n_acc > 1 ? 32u * (uint32_t)(slice % p.n_acc) : 0u;
+                    const uint32_t first = p.n_acc > 1 ? (uint32_t)(slice < p.n_acc) : (uint32_t)(slice == 0);
                     for (int h = 0; h < p.nh; h++) {
                         const uint64_t bdesc = umma_desc_sw128(xa + half_cols * 128u * h + 32u * j);
-                        umma_f16(tmem + half_cols * h, adesc, bdesc, idesc,
-                                 (kt > k_begin || j > 0) ? 1u : 0u);
+                        umma_f16(tmem + acc + half_cols * h, adesc, bdesc, idesc, first ? 0u : 1u);
                     }
                 }
                 umma_commit(smem_u32(&x_empty[xs]));
@@ -345,7 +356,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             }
             __syncwarp();
             if (++xs == SX) { xs = 0; xph ^= 1u; }
-            if (++ws == kWStages) { ws = 0; wph ^= 1u; }
+            if (++ws == SW) { ws = 0; wph ^= 1u; }
         }
         if (lane == 0) {
             umma_commit(smem_u32(acc_full));
@@ -355,11 +366,11 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         __syncwarp();
     } else {
         // ------------------------------------------------------------ decoders
-        const int d = warp - 2;          // 0..7
-        const int q = d >> 2;            // strip within the tile
-        const int g = d & 3;             // 16-column group
+        const int d = warp - 2;          // 0..15
+        const int q = d >> 3;            // strip within the tile
+        const int g = d & 7;             // 8-column group: one 16-byte chunk per row
         const bool strip_ok = s0 + q < p.n_strips;
-        uint4* rec = (uint4*)(smem + p.off_rec + 256u * d);  // 16 columns x 16 bytes
+        uint4* rec = (uint4*)(smem + p.off_rec + 128u * d);  // 8 columns x 16 bytes
         const int qb = 2 * (lane & 15);  // this lane's rows sit at bits qb, qb+1 of one half
         const int sh = qb + 1;
         const uint32_t bit0 = 1u << qb, bit1 = 2u << qb;
@@ -377,7 +388,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             const uint32_t rst_s = sbase + p.off_raw + (uint32_t)rs * p.raw_stage_bytes;
             if (strip_ok) {
                 // columns 2l and 2l+1 of the strip: counts, starts, and the records of the
-                // warp's 16 columns (lanes 8g .. 8g+7 hold them)
+                // warp's 8 columns (lanes 4g .. 4g+3 hold them)
                 const uint4 bw = *(const uint4*)(smem + p.off_raw + (size_t)rs * p.raw_stage_bytes +
                                                  512u * q + 16u * lane);
                 const int cl0 = __popc(bw.x), c0 = cl0 + __popc(bw.y);
@@ -386,26 +397,25 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 const uint32_t vb = rst_s + 1024u + (uint32_t)q * p.val_slot;
                 const uint32_t a0 = vb + 2u * (uint32_t)(incl - c0 - c1);
                 const uint32_t a1 = a0 + 2u * (uint32_t)c0;
-                if ((lane >> 3) == g) {
-                    const int j = 2 * (lane & 7);
+                if ((lane >> 2) == g) {
+                    const int j = 2 * (lane & 3);
                     rec[j] = make_uint4(bw.x, a0 + 2u * (uint32_t)cl0, bw.y, a1);
                     rec[j + 1] = make_uint4(bw.z, a1 + 2u * (uint32_t)cl1, bw.w, a1 + 2u * (uint32_t)c1);
                 }
             }
             __syncwarp();
-            if (i >= kWStages &&
+            if (i >= SW &&
                 !__all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_empty[ws]), wph ^ 1u, abort_flag))) {
                 flag_abort(abort_flag, p.status);
                 break;
             }
             unsigned char* wst = smem + p.off_w + (uint32_t)ws * kWStageBytes;
-#pragma unroll
-            for (int cc = 0; cc < 2; cc++) {  // 8 columns -> one 16-byte chunk per row
+            {  // 8 columns -> one 16-byte chunk per row
                 uint32_t o0[4] = {0u, 0u, 0u, 0u}, o1[4] = {0u, 0u, 0u, 0u};
                 if (strip_ok) {
 #pragma unroll
                     for (int c = 0; c < 8; c++) {
-                        const uint2 r = rec2[2 * (8 * cc + c)];
+                        const uint2 r = rec2[2 * c];
                         uint32_t a;
                         asm("mad.lo.s32 %0, %1, -2, %2;" : "=r"(a) : "r"(__popc(r.x >> sh)), "r"(r.y));
                         const uint32_t v1 = lds_u16(a), v0 = lds_u16(a - 2u);
@@ -414,7 +424,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                         o1[c >> 1] |= ((r.x & bit1) ? v1 : 0u) << sft;
                     }
                 }
-                const uint32_t chunk = 2u * g + cc;
+                const uint32_t chunk = (uint32_t)g;
                 *(uint4*)(wst + nl0 * 128u + ((chunk ^ (nl0 & 7u)) << 4)) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
                 *(uint4*)(wst + nl1 * 128u + ((chunk ^ (nl1 & 7u)) << 4)) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
             }
@@ -425,7 +435,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 mbar_arrive(smem_u32(&r_empty[rs]));
             }
             if (++rs == SR) { rs = 0; rph ^= 1u; }
-            if (++ws == kWStages) { ws = 0; wph ^= 1u; }
+            if (++ws == SW) { ws = 0; wph ^= 1u; }
         }
 
         // ------------------------------------------------------------ epilogue
@@ -434,16 +444,24 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         if (acc_ready) {
             tc_fence_after();
             const int quarter = warp & 3;       // TMEM lanes this warp may access
-            const int half = (warp - 2) >> 2;   // which 32-column chunks: j % 2 == half
+            const int part_of = (warp - 2) >> 2;  // which 32-column chunks: j % 4 == part_of
             const int row = 32 * quarter + lane;
             const int n = n0 + row;
             const size_t tile = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
             float* part = p.partials + (tile * p.ksplit + kz) * (size_t)p.MT * kTileRows;
             // 32 accumulator columns per load; the allocation is a power of two >= 32, so a
             // tile of 16 tokens reads 16 valid columns and 16 unused ones.
-            for (int j = half; j < (p.MT + 31) / 32; j += 2) {
+            // accumulators written by this CTA's k-slices (each k-slice writes one of them)
+            const int n_used = min(p.n_acc, (k_end - k_begin) * (kBK / 16));
+            for (int j = part_of; j < (p.MT + 31) / 32; j += 4) {
                 uint32_t r[32];
                 tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + 32u * j, r);
+                for (int a = 1; a < n_used; a++) {  // narrow tiles: add the other chains
+                    uint32_t r2[32];
+                    tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + 32u * (uint32_t)a, r2);
+#pragma unroll
+                    for (int c = 0; c < 32; c++) r[c] = __float_as_uint(__uint_as_float(r[c]) + __uint_as_float(r2[c]));
+                }
                 const int lim = min(32, p.MT - 32 * j);
                 if (p.ksplit > 1) {
 #pragma unroll
@@ -487,14 +505,15 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             }
         }
     }
-    if (warp == 0 && lane == 0 && *abort_flag) {
-        // Drain the copies this CTA armed (bounded): for each slot, the phase of its
-        // last issue.  Phases a consumer already waited for return at once.
-        for (int i = 0; i < SX && i < x_issued; i++) {
+    if (warp == 0 && *abort_flag) {
+        // Drain the copies this CTA armed (bounded), each producer lane its own ring: for
+        // each slot, the phase of its last issue.  Phases a consumer already waited for
+        // return at once.
+        for (int i = 0; lane == 0 && i < SX && i < x_issued; i++) {
             const int last = i + ((x_issued - 1 - i) / SX) * SX;
             (void)mbar_wait(smem_u32(&x_full[i]), (uint32_t)((last / SX) & 1));
         }
-        for (int i = 0; i < SR && i < r_issued; i++) {
+        for (int i = 0; lane == 1 && i < SR && i < r_issued; i++) {
             const int last = i + ((r_issued - 1 - i) / SR) * SR;
             (void)mbar_wait(smem_u32(&r_full[i]), (uint32_t)((last / SR) & 1));
         }
@@ -530,15 +549,16 @@ int get_encoder() {
 }
 
 struct SpmmPlan {
-    int MT, nh, m_tiles, n_tiles, ksplit, sx, sr, ctas_per_sm;
+    int MT, nh, n_acc, m_tiles, n_tiles, ksplit, sx, sr, sw, ctas_per_sm;
     uint32_t x_stage_bytes, val_slot, raw_stage_bytes, tmem_cols;
     uint32_t off_w, off_raw, off_rec, off_tptr, off_bar;
     size_t smem;
     uint64_t ws_counters, ws_bytes;
+    uint64_t ws_xt;  // decode with a rule: offset of x~ (B rows of K rounded up to 8)
 };
 
 // Token tile, split-K factor, stage counts and shared-memory layout for M rows of X.
-int make_spmm_plan(const spw_format* h, int M, SpmmPlan* pl) {
+int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl) {
     const int sms = device_sm_count();
     if (sms <= 0) return SPW_ERR_CUDA;
     pl->m_tiles = (M + kMaxTokens - 1) / kMaxTokens;
@@ -547,26 +567,30 @@ int make_spmm_plan(const spw_format* h, int M, SpmmPlan* pl) {
     pl->MT = (int)round_up_u64((uint64_t)per, 16u * pl->nh);  // each MMA's N a multiple of 16
     pl->n_tiles = (int)((h->N + kTileRows - 1) / kTileRows);
     pl->x_stage_bytes = (uint32_t)pl->MT * 128u;
+    pl->n_acc = pl->MT <= 32 ? 4 : 1;
     uint32_t cols = 32;
-    while (cols < (uint32_t)pl->MT) cols <<= 1;
+    while (cols < (uint32_t)(pl->n_acc > 1 ? 32 * pl->n_acc : pl->MT)) cols <<= 1;
     pl->tmem_cols = cols;
     pl->val_slot = (uint32_t)round_up_u64(16ull * h->max_tile_units + 16, 16);
     pl->raw_stage_bytes = 1024u + (uint32_t)kTileStrips * pl->val_slot;
     const uint32_t tptr_bytes = (uint32_t)round_up_u64(4ull * kTileStrips * (h->n_ktiles + 1), 16);
-    const int options[][2] = {{4, 4}, {4, 3}, {3, 3}, {3, 2}, {2, 3}, {2, 2}};
+    // {X, TCB, decoded-weight} stages, deepest first
+    const int options[][3] = {{4, 4, 4}, {3, 4, 4}, {2, 4, 4}, {2, 4, 3}, {2, 3, 3},
+                              {2, 3, 2}, {2, 2, 2}};
     bool found = false;
     for (const auto& o : options) {
-        const int sx = o[0], sr = o[1];
+        const int sx = o[0], sr = o[1], sw = o[2];
         const uint32_t off_w = (uint32_t)sx * pl->x_stage_bytes;
-        const uint32_t off_raw = off_w + (uint32_t)kWStages * kWStageBytes;
+        const uint32_t off_raw = off_w + (uint32_t)sw * kWStageBytes;
         const uint32_t off_rec = off_raw + (uint32_t)sr * pl->raw_stage_bytes;
-        const uint32_t off_tptr = off_rec + 256u * kDecoderWarps;
+        const uint32_t off_tptr = off_rec + 128u * kDecoderWarps;
         const uint32_t off_bar = (uint32_t)round_up_u64(off_tptr + tptr_bytes, 8);
-        const uint32_t bar_bytes = 8u * (2 * sx + 2 * sr + 2 * kWStages + 2) + 16u;
+        const uint32_t bar_bytes = 8u * (2 * sx + 2 * sr + 2 * sw + 2) + 16u;
         const size_t total = (size_t)off_bar + bar_bytes + 1024;  // + base alignment slack
         if (total <= (size_t)kSmemLimit) {
             pl->sx = sx;
             pl->sr = sr;
+            pl->sw = sw;
             pl->off_w = off_w;
             pl->off_raw = off_raw;
             pl->off_rec = off_rec;
@@ -579,17 +603,30 @@ int make_spmm_plan(const spw_format* h, int M, SpmmPlan* pl) {
     }
     if (!found) return SPW_ERR_UNSUPPORTED;
     // Split K when the output tiles cannot fill the SMs (two k-tiles per split at least).
-    pl->ctas_per_sm = 1;  // 320 threads at ~120 registers: one CTA per SM
+    pl->ctas_per_sm = 1;  // 576 threads: one CTA per SM
     const long long tiles = (long long)pl->m_tiles * pl->n_tiles;
     const long long slots = (long long)sms * pl->ctas_per_sm;
-    long long ks = tiles >= slots ? 1 : slots / tiles;
-    const long long kmax = h->n_ktiles / 2 > 0 ? h->n_ktiles / 2 : 1;
-    if (ks > kmax) ks = kmax;
+    // Only grids smaller than one wave are split: the split with the fewest waves per unit
+    // of work, lightly penalised per extra split (partial tiles cost traffic).
+    long long kmax = h->n_ktiles / 2 > 0 ? (h->n_ktiles / 2 < 16 ? h->n_ktiles / 2 : 16) : 1;
+    if (tiles >= slots) kmax = 1;
+    long long ks = 1;
+    double best = 1e30;
+    for (long long k = 1; k <= kmax; k++) {
+        const double waves = (double)((tiles * k + slots - 1) / slots);
+        const double cost = waves / (double)k + 0.02 * (double)(k - 1);
+        if (cost < best - 1e-9) {
+            best = cost;
+            ks = k;
+        }
+    }
     pl->ksplit = (int)ks;
     pl->ws_counters = pl->ksplit > 1 ? round_up_u64(4ull * (uint64_t)tiles, 256) : 0;
     pl->ws_bytes = pl->ksplit > 1
                        ? pl->ws_counters + 4ull * (uint64_t)tiles * pl->ksplit * pl->MT * kTileRows
                        : 0;
+    pl->ws_xt = round_up_u64(pl->ws_bytes, 256);
+    if (rule) pl->ws_bytes = pl->ws_xt + 2ull * (uint64_t)M * round_up_u64(h->K, 8);
     return SPW_OK;
 }
 
@@ -597,8 +634,9 @@ int make_spmm_plan(const spw_format* h, int M, SpmmPlan* pl) {
 int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int M, int ldx,
                uint16_t* d_Y, int ldy, int rule, float t, const uint32_t* act_bits, void* d_ws,
                uint64_t ws_bytes, cudaStream_t stream) {
+    const bool needs_rule = rule && (t > 0.0f || act_bits);
     SpmmPlan pl;
-    int rc = make_spmm_plan(hdr, M, &pl);
+    int rc = make_spmm_plan(hdr, M, needs_rule, &pl);
     if (rc != SPW_OK) return rc;
     if (pl.ws_bytes) {
         if (!d_ws) return SPW_ERR_INVALID_ARG;
@@ -610,6 +648,15 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
     int* status = device_status_ptr();
     if (!status) return SPW_ERR_CUDA;
 
+    if (needs_rule) {  // x~ into the workspace; the product reads it instead of X
+        const int ld = (int)round_up_u64(hdr->K, 8);
+        uint16_t* xt = (uint16_t*)((uint8_t*)d_ws + pl.ws_xt);
+        const int n = M * ((int)(hdr->K + 7) / 8);
+        rule_kernel<<<(n + 255) / 256, 256, 0, stream>>>(d_X, ldx, M, (int)hdr->K, t, act_bits, xt, ld);
+        SPW_LAUNCH_CHECK();
+        d_X = xt;
+        ldx = ld;
+    }
     // X as a 2-D tensor map: dim 0 = K (contiguous), dim 1 = M rows at ldx elements.
     CUtensorMap tmap;
     const cuuint64_t dims[2] = {(cuuint64_t)hdr->K, (cuuint64_t)M};
@@ -631,7 +678,6 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
     prm.Y = d_Y;
     prm.counters = pl.ws_bytes ? (uint32_t*)d_ws : nullptr;
     prm.partials = pl.ws_bytes ? (float*)((uint8_t*)d_ws + pl.ws_counters) : nullptr;
-    prm.act_bits = act_bits;
     prm.status = status;
     prm.M = M;
     prm.N = (int)hdr->N;
@@ -641,11 +687,11 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
     prm.n_ktiles = (int)hdr->n_ktiles;
     prm.MT = pl.MT;
     prm.nh = pl.nh;
+    prm.n_acc = pl.n_acc;
     prm.ksplit = pl.ksplit;
     prm.sx = pl.sx;
     prm.sr = pl.sr;
-    prm.rule = rule;
-    prm.t = t;
+    prm.sw = pl.sw;
     prm.x_stage_bytes = pl.x_stage_bytes;
     prm.raw_stage_bytes = pl.raw_stage_bytes;
     prm.val_slot = pl.val_slot;
@@ -682,7 +728,7 @@ extern "C" {
 uint64_t spw_spmm_workspace_bytes(const spw_format* hdr, int M) {
     if (check_header(hdr) != SPW_OK || M < 1) return 0;
     SpmmPlan pl;
-    if (make_spmm_plan(hdr, M, &pl) != SPW_OK) return 0;
+    if (make_spmm_plan(hdr, M, false, &pl) != SPW_OK) return 0;
     return pl.ws_bytes;
 }
 
@@ -700,8 +746,10 @@ int spw_spmm(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int 
 }
 
 uint64_t spw_spmv_tc_workspace_bytes(const spw_format* hdr, int B) {
-    if (B < 1 || B > 16) return 0;
-    return spw_spmm_workspace_bytes(hdr, B);
+    if (B < 1 || B > 16 || check_header(hdr) != SPW_OK) return 0;
+    SpmmPlan pl;
+    if (make_spmm_plan(hdr, B, true, &pl) != SPW_OK) return 0;
+    return pl.ws_bytes;  // room for x~ whatever the threshold and column set
 }
 
 int spw_spmv_tc(const spw_format* hdr, const void* d_buf, const uint16_t* d_x, int B, int ldx,
