@@ -495,13 +495,40 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         __syncthreads();
         if (*last_flag) {
             __threadfence();
-            const float* base = p.partials + tile * p.ksplit * (size_t)p.MT * kTileRows;
-            for (int idx = threadIdx.x; idx < p.MT * kTileRows; idx += kThreads) {
-                const int tok = idx / kTileRows, row = idx % kTileRows;
-                const int m = m0 + tok, n = n0 + row;
-                float s = 0.0f;
-                for (int z = 0; z < p.ksplit; z++) s += __ldcg(base + (size_t)z * p.MT * kTileRows + idx);
-                if (m < p.M && n < p.N) p.Y[(size_t)m * p.ldy + n] = __half_as_ushort(__float2half_rn(s));
+            // Four consecutive rows of one token per thread (16-byte loads), four such
+            // groups in flight; the partials are summed in split order (deterministic).
+            const float4* base = (const float4*)(p.partials + tile * p.ksplit * (size_t)p.MT * kTileRows);
+            const int n4 = p.MT * kTileRows / 4, stride4 = p.MT * kTileRows / 4;
+            for (int i0 = threadIdx.x; i0 < n4; i0 += 4 * kThreads) {
+                float4 acc[4];
+#pragma unroll
+                for (int u = 0; u < 4; u++) acc[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                for (int z = 0; z < p.ksplit; z++) {
+#pragma unroll
+                    for (int u = 0; u < 4; u++) {
+                        const int i = i0 + u * kThreads;
+                        if (i < n4) {
+                            const float4 v = __ldcg(base + (size_t)z * stride4 + i);
+                            acc[u].x += v.x;
+                            acc[u].y += v.y;
+                            acc[u].z += v.z;
+                            acc[u].w += v.w;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    const int i = i0 + u * kThreads;
+                    if (i >= n4) continue;
+                    const int tok = (4 * i) / kTileRows, row = (4 * i) % kTileRows;
+                    const int m = m0 + tok;
+                    if (m >= p.M) continue;
+                    const float v[4] = {acc[u].x, acc[u].y, acc[u].z, acc[u].w};
+#pragma unroll
+                    for (int e = 0; e < 4; e++)
+                        if (n0 + row + e < p.N)
+                            p.Y[(size_t)m * p.ldy + n0 + row + e] = __half_as_ushort(__float2half_rn(v[e]));
+                }
             }
         }
     }
@@ -561,11 +588,39 @@ struct SpmmPlan {
 int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl) {
     const int sms = device_sm_count();
     if (sms <= 0) return SPW_ERR_CUDA;
-    pl->m_tiles = (M + kMaxTokens - 1) / kMaxTokens;
+    // Token tile (512, 256 or 128 tokens, or all M when smaller) and split-K factor from a
+    // small cost model in microseconds, per CTA wave: k-steps x max(decode ~0.7, MMA
+    // ~0.76 x MT / 512) plus, when K is split, the fp32 partial tile written and summed
+    // (~0.1 GB/ms per CTA).  One CTA per SM.
+    pl->n_tiles = (int)((h->N + kTileRows - 1) / kTileRows);
+    const long long slots = sms;
+    const long long nk_all = h->n_ktiles;
+    const long long kcap = nk_all / 2 > 0 ? (nk_all / 2 < 16 ? nk_all / 2 : 16) : 1;
+    double best = 1e300;
+    int best_mt_max = kMaxTokens, best_ks = 1;
+    for (int tok_max = kMaxTokens; tok_max >= 128; tok_max /= 2) {
+        const int mt = (M + tok_max - 1) / tok_max;
+        const int per_t = (M + mt - 1) / mt;
+        const int nh_t = per_t > 256 ? 2 : 1;
+        const double MTd = (double)round_up_u64((uint64_t)per_t, 16u * nh_t);
+        const long long tiles_t = (long long)mt * pl->n_tiles;
+        for (long long k = 1; k <= kcap; k++) {
+            const double waves = (double)((tiles_t * k + slots - 1) / slots);
+            const double step = MTd * 0.76 / 512.0 > 0.7 ? MTd * 0.76 / 512.0 : 0.7;
+            const double split = k > 1 ? MTd * 512.0 * (double)(k + 1) / 1e5 : 0.0;
+            const double cost = waves * ((double)nk_all / (double)k * step + split);
+            if (cost < best * 0.98) {
+                best = cost;
+                best_mt_max = tok_max;
+                best_ks = (int)k;
+            }
+        }
+        if (M <= tok_max / 2) continue;  // smaller token caps change nothing more for small M
+    }
+    pl->m_tiles = (M + best_mt_max - 1) / best_mt_max;
     const int per = (M + pl->m_tiles - 1) / pl->m_tiles;
     pl->nh = per > 256 ? 2 : 1;
     pl->MT = (int)round_up_u64((uint64_t)per, 16u * pl->nh);  // each MMA's N a multiple of 16
-    pl->n_tiles = (int)((h->N + kTileRows - 1) / kTileRows);
     pl->x_stage_bytes = (uint32_t)pl->MT * 128u;
     pl->n_acc = pl->MT <= 32 ? 4 : 1;
     uint32_t cols = 32;
@@ -602,25 +657,9 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl) {
         }
     }
     if (!found) return SPW_ERR_UNSUPPORTED;
-    // Split K when the output tiles cannot fill the SMs (two k-tiles per split at least).
     pl->ctas_per_sm = 1;  // 576 threads: one CTA per SM
     const long long tiles = (long long)pl->m_tiles * pl->n_tiles;
-    const long long slots = (long long)sms * pl->ctas_per_sm;
-    // Only grids smaller than one wave are split: the split with the fewest waves per unit
-    // of work, lightly penalised per extra split (partial tiles cost traffic).
-    long long kmax = h->n_ktiles / 2 > 0 ? (h->n_ktiles / 2 < 16 ? h->n_ktiles / 2 : 16) : 1;
-    if (tiles >= slots) kmax = 1;
-    long long ks = 1;
-    double best = 1e30;
-    for (long long k = 1; k <= kmax; k++) {
-        const double waves = (double)((tiles * k + slots - 1) / slots);
-        const double cost = waves / (double)k + 0.02 * (double)(k - 1);
-        if (cost < best - 1e-9) {
-            best = cost;
-            ks = k;
-        }
-    }
-    pl->ksplit = (int)ks;
+    pl->ksplit = best_ks;
     pl->ws_counters = pl->ksplit > 1 ? round_up_u64(4ull * (uint64_t)tiles, 256) : 0;
     pl->ws_bytes = pl->ksplit > 1
                        ? pl->ws_counters + 4ull * (uint64_t)tiles * pl->ksplit * pl->MT * kTileRows
