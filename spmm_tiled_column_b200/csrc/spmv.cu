@@ -31,8 +31,8 @@
 //     (each half-warp reads its own 8 bytes of the same 16).
 //   * Split-K combine: a warp writes its fp32 partial for each strip piece into the
 //     workspace; the last contributor of a strip (counted with an atomic) sums all pieces
-//     in warp order -- a fixed order, so results are deterministic -- rounds to fp16 and
-//     resets the counter.  A strip with a single contributor is written directly.
+//     in a fixed order (even pieces, odd pieces, then the two sums), so results are
+//     deterministic, rounds to fp16 and resets the counter.  A strip with a single contributor is written directly.
 #include <stdlib.h>
 #include <string.h>
 
@@ -512,30 +512,44 @@ __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lan
             if (lane == 0) old = atom_add_release_gpu(&L.counters[s], 1u);
             old = __shfl_sync(0xffffffffu, old, 0);
             if ((int)old == count - 1) {
-                // Last contributor: sum every piece in contributor order (deterministic),
-                // eight pieces' loads in flight at once.
+                // Last contributor: sum every piece in a fixed order (deterministic).  Lanes
+                // l and l+16 read rows 4(l mod 16)..+3 of the even and odd pieces with 16-byte
+                // loads, 32 pieces in flight per round; the two halves then add up.
                 __threadfence();
                 const float* base = L.partials + (size_t)s * L.maxc * B * 64;
+                const int half = lane >> 4, r4 = 4 * (lane & 15);
 #pragma unroll 1
                 for (int b = 0; b < B; b++) {
-                    float sx = 0.0f, sy = 0.0f;
+                    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll 1
-                    for (int j0 = 0; j0 < count; j0 += 8) {
-                        float2 v[8];
+                    for (int j0 = half; j0 < count; j0 += 32) {
+                        float4 v[16];
 #pragma unroll
-                        for (int u = 0; u < 8; u++)
-                            v[u] = (j0 + u < count)
-                                       ? __ldcg((const float2*)(base + ((size_t)(j0 + u) * B + b) * 64) + lane)
-                                       : make_float2(0.0f, 0.0f);
+                        for (int u = 0; u < 16; u++) {
+                            const int j = j0 + 2 * u;
+                            v[u] = j < count ? __ldcg((const float4*)(base + ((size_t)j * B + b) * 64 + r4))
+                                             : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        }
 #pragma unroll
-                        for (int u = 0; u < 8; u++) {
-                            sx += v[u].x;
-                            sy += v[u].y;
+                        for (int u = 0; u < 16; u++) {
+                            acc.x += v[u].x;
+                            acc.y += v[u].y;
+                            acc.z += v[u].z;
+                            acc.w += v[u].w;
                         }
                     }
-                    if (r0 < L.N) L.y[(size_t)b * L.ldy + r0] = __half_as_ushort(__float2half_rn(sx));
-                    if (r0 + 1 < L.N)
-                        L.y[(size_t)b * L.ldy + r0 + 1] = __half_as_ushort(__float2half_rn(sy));
+                    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
+                    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 16);
+                    acc.z += __shfl_xor_sync(0xffffffffu, acc.z, 16);
+                    acc.w += __shfl_xor_sync(0xffffffffu, acc.w, 16);
+                    const int r = s * kStripRows + r4;
+                    uint16_t* yb = L.y + (size_t)b * L.ldy;
+                    if (half == 0) {
+                        if (r < L.N) yb[r] = __half_as_ushort(__float2half_rn(acc.x));
+                        if (r + 1 < L.N) yb[r + 1] = __half_as_ushort(__float2half_rn(acc.y));
+                        if (r + 2 < L.N) yb[r + 2] = __half_as_ushort(__float2half_rn(acc.z));
+                        if (r + 3 < L.N) yb[r + 3] = __half_as_ushort(__float2half_rn(acc.w));
+                    }
                 }
                 if (lane == 0) L.counters[s] = 0u;
             }
