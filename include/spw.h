@@ -38,6 +38,13 @@
  *     multiples of 8 fp16 elements unless that operand has a single row.  Such copies
  *     may read an activation row up to the next 16-byte boundary past its last
  *     element (never across it, so never outside the row's allocation granule).
+ *   - Buffer contents: the header is checked on the host.  The product kernels check each
+ *     tile they read against it -- its tile pointers inside the values section and at
+ *     most max_tile_units apart, its bitmaps' kept count within what max_tile_units
+ *     allows -- and decode a tile that fails as empty, reporting SPW_ERR_FORMAT through
+ *     spw_last_device_status.  Other disagreements between a buffer's sections give
+ *     undefined numbers but no access outside the buffer.  spw_compress writes
+ *     consistent buffers.
  *
  * The TCB v1 layout (this project's reading of Tiled-CBC; the page names the format but
  * gives no layout).  All integers little-endian.  A strip is 64 consecutive weight rows,
@@ -258,8 +265,9 @@ int spw_spmv_tc(const spw_format* hdr, const void* d_buf, const uint16_t* d_x, i
                 uint64_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, then read and clear the library's device status word for the
- * current device: *code = SPW_OK, or SPW_ERR_TIMEOUT if a bounded device wait ran out
- * since the last read.  Errors: INVALID_ARG, CUDA. */
+ * current device: *code = SPW_OK, SPW_ERR_TIMEOUT if a bounded device wait ran out, or
+ * SPW_ERR_FORMAT if a product kernel met a tile that disagrees with its header (see
+ * "Buffer contents"), since the last read.  Errors: INVALID_ARG, CUDA. */
 int spw_last_device_status(void* stream, int* code);
 
 #ifdef __cplusplus

@@ -64,6 +64,7 @@ struct SpmmParams {
     const uint64_t* bitmaps;
     const uint32_t* tileptr;
     const uint16_t* values;
+    uint64_t values_units;      // the values section, in 16-byte units
     uint16_t* Y;
     uint32_t* counters;         // split-K arrivals per output tile (ksplit > 1)
     float* partials;            // split-K fp32 partial tiles
@@ -302,8 +303,8 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     if (s0 + j >= p.n_strips) continue;
                     u0[j] = tptr[j * (nk + 1) + kt];
                     const uint32_t u1 = tptr[j * (nk + 1) + kt + 1];
-                    vb[j] = u1 >= u0[j] ? (u1 - u0[j]) * 16u : 0xFFFFFFFFu;
-                    if (vb[j] > p.val_slot - 16u) {  // larger than the header allows
+                    vb[j] = u1 >= u0[j] && u1 <= p.values_units ? (u1 - u0[j]) * 16u : 0xFFFFFFFFu;
+                    if (vb[j] > p.val_slot - 16u) {  // outside the section or larger than the header allows
                         raise_status(p.status, SPW_ERR_FORMAT);
                         vb[j] = 0;
                     }
@@ -386,6 +387,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 break;
             }
             const uint32_t rst_s = sbase + p.off_raw + (uint32_t)rs * p.raw_stage_bytes;
+            bool dec = strip_ok;  // warp-uniform
             if (strip_ok) {
                 // columns 2l and 2l+1 of the strip: counts, starts, and the records of the
                 // warp's 8 columns (lanes 4g .. 4g+3 hold them)
@@ -397,7 +399,12 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 const uint32_t vb = rst_s + 1024u + (uint32_t)q * p.val_slot;
                 const uint32_t a0 = vb + 2u * (uint32_t)(incl - c0 - c1);
                 const uint32_t a1 = a0 + 2u * (uint32_t)c0;
-                if ((lane >> 2) == g) {
+                // More values than the slot holds means the bitmaps and the tile pointers
+                // disagree: report it and decode the tile as empty rather than read past it.
+                if (2u * (uint32_t)__shfl_sync(0xffffffffu, incl, 31) > p.val_slot - 16u) {
+                    if (lane == 0) raise_status(p.status, SPW_ERR_FORMAT);
+                    dec = false;
+                } else if ((lane >> 2) == g) {
                     const int j = 2 * (lane & 3);
                     rec[j] = make_uint4(bw.x, a0 + 2u * (uint32_t)cl0, bw.y, a1);
                     rec[j + 1] = make_uint4(bw.z, a1 + 2u * (uint32_t)cl1, bw.w, a1 + 2u * (uint32_t)c1);
@@ -412,7 +419,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             unsigned char* wst = smem + p.off_w + (uint32_t)ws * kWStageBytes;
             {  // 8 columns -> one 16-byte chunk per row
                 uint32_t o0[4] = {0u, 0u, 0u, 0u}, o1[4] = {0u, 0u, 0u, 0u};
-                if (strip_ok) {
+                if (dec) {
 #pragma unroll
                     for (int c = 0; c < 8; c++) {
                         const uint2 r = rec2[2 * c];
@@ -714,6 +721,7 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
     prm.bitmaps = (const uint64_t*)(buf + hdr->off_bitmaps);
     prm.tileptr = (const uint32_t*)(buf + hdr->off_tileptr);
     prm.values = (const uint16_t*)(buf + hdr->off_values);
+    prm.values_units = (hdr->bytes_total - hdr->off_values) / 16;
     prm.Y = d_Y;
     prm.counters = pl.ws_bytes ? (uint32_t*)d_ws : nullptr;
     prm.partials = pl.ws_bytes ? (float*)((uint8_t*)d_ws + pl.ws_counters) : nullptr;

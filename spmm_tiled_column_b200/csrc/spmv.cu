@@ -72,6 +72,7 @@ struct SpmvLayer {
     int n_ktiles;
     int maxc;
     int tile_begin, n_tiles;
+    uint64_t values_units;  // the values section, in 16-byte units
 };
 
 struct SpmvParams {
@@ -320,8 +321,8 @@ __device__ void produce(const SpmvParams& p, unsigned char* regions, int W, int 
             continue;
         }
         const SpmvLayer& L = p.L[c.l];
-        uint64_t vbytes = u1 >= u0 ? 16ull * (u1 - u0) : ~0ull;
-        if (vbytes + kStageValsOff + 16u > p.stage_bytes) {  // tile larger than the header allows
+        uint64_t vbytes = u1 >= u0 && u1 <= L.values_units ? 16ull * (u1 - u0) : ~0ull;
+        if (vbytes > p.stage_bytes - kStageValsOff - 16u) {  // outside the section or larger than the header allows
             raise_status(p.status, SPW_ERR_FORMAT);
             vbytes = 0;
         }
@@ -381,6 +382,8 @@ __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lan
     const uint32_t bit0 = 1u << q, bit1 = 2u << q;
     const uint2* rec2 = (const uint2*)rec + (lane < 16 ? 0 : 1);  // this half's 8 bytes
     const int neg2 = p.neg2;
+    // Largest value count a stage holds (the slack after it serves the branch-free loads).
+    const int cap = (int)((p.stage_bytes - kStageValsOff - 16u) / 2u);
 
     // Activations, column sets, outputs and the workspace only after the previous kernel
     // on the stream is complete.
@@ -429,17 +432,22 @@ __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lan
             any1 |= p1;
         }
         const uint4 bw = *(const uint4*)(reg + HDR + (size_t)slot * p.stage_bytes + 16 * lane);
-        any0 = any0 && (bw.x | bw.y) != 0u;
-        any1 = any1 && (bw.z | bw.w) != 0u;
+        // Column starts within the tile's values (all 64 columns, in column order).
+        const int cl0 = __popc(bw.x), c0 = cl0 + __popc(bw.y);
+        const int cl1 = __popc(bw.z), c1 = cl1 + __popc(bw.w);
+        const int incl = warp_inclusive_scan(c0 + c1, lane);
+        // A lane's columns index values below incl.  More than a stage holds means the
+        // bitmaps and the tile pointers disagree: report it and skip those columns rather
+        // than read beyond the stage.
+        const bool fits = incl <= cap;
+        if (!fits) raise_status(p.status, SPW_ERR_FORMAT);
+        any0 = fits && any0 && (bw.x | bw.y) != 0u;
+        any1 = fits && any1 && (bw.z | bw.w) != 0u;
         const uint32_t m0 = __ballot_sync(0xffffffffu, any0);
         const uint32_t m1 = __ballot_sync(0xffffffffu, any1);
         const int n_act = __popc(m0) + __popc(m1);
 
         if (n_act > 0) {
-            // Column starts within the tile's values (all 64 columns, in column order).
-            const int cl0 = __popc(bw.x), c0 = cl0 + __popc(bw.y);
-            const int cl1 = __popc(bw.z), c1 = cl1 + __popc(bw.w);
-            const int incl = warp_inclusive_scan(c0 + c1, lane);
             const uint32_t vb = st_s + kStageValsOff;
             const uint32_t a0 = vb + 2u * (uint32_t)(incl - c0 - c1);
             const uint32_t a1 = a0 + 2u * (uint32_t)c0;
@@ -745,6 +753,7 @@ int decode_group_launch(int n, const spw_format* hdrs, const void* const* bufs,
         L.maxc = pl.maxc[l];
         L.tile_begin = (int)begin;
         L.n_tiles = (int)((long long)h.n_strips * h.n_ktiles);
+        L.values_units = (h.bytes_total - h.off_values) / 16;
         begin += L.n_tiles;
     }
     prm.n_layers = n;
