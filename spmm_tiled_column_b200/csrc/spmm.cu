@@ -210,6 +210,12 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     const int kz = blockIdx.z;
     const int k_begin = (int)((long long)kz * nk / p.ksplit);
     const int k_end = (int)((long long)(kz + 1) * nk / p.ksplit);
+    // Every role walks the CTA's k-steps from a start rotated by the weight-row tile: the
+    // CTAs that share an X tile then read different k-columns of it at any moment instead
+    // of all hitting the same L2 lines together.
+    const int n_kc = k_end - k_begin;
+    const int k_rot = n_kc > 0 ? (int)(blockIdx.y % (unsigned)n_kc) : 0;
+    auto kstep = [&](int i) { return k_begin + (i + k_rot < n_kc ? i + k_rot : i + k_rot - n_kc); };
     const int SX = p.sx, SR = p.sr;
 
     uint64_t* bars = (uint64_t*)(smem + p.off_bar);
@@ -272,9 +278,10 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             const int rows = p.MT / p.nh;  // TMA box height
             int xs = 0;
             uint32_t xph = 0;
-            for (int kt = k_begin; kt < k_end; kt++) {
+            for (int i = 0; i < n_kc; i++) {
+                const int kt = kstep(i);
                 // X tile: rows m0..m0+MT-1, columns 64 kt.. (zero fill outside X)
-                if (kt - k_begin >= SX && !wait_or_abort(smem_u32(&x_empty[xs]), xph ^ 1u, abort_flag)) {
+                if (i >= SX && !wait_or_abort(smem_u32(&x_empty[xs]), xph ^ 1u, abort_flag)) {
                     flag_abort(abort_flag, p.status);
                     break;
                 }
@@ -289,8 +296,9 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         } else if (lane == 1) {  // TCB ring: the two tiles of each k-step
             int rs = 0;
             uint32_t rph = 0;
-            for (int kt = k_begin; kt < k_end; kt++) {
-                if (kt - k_begin >= SR && !wait_or_abort(smem_u32(&r_empty[rs]), rph ^ 1u, abort_flag)) {
+            for (int i = 0; i < n_kc; i++) {
+                const int kt = kstep(i);
+                if (i >= SR && !wait_or_abort(smem_u32(&r_empty[rs]), rph ^ 1u, abort_flag)) {
                     flag_abort(abort_flag, p.status);
                     break;
                 }
@@ -330,7 +338,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         int xs = 0, ws = 0;
         uint32_t xph = 0, wph = 0;
         bool ok = true;
-        for (int kt = k_begin; kt < k_end && ok; kt++) {
+        for (int i = 0; i < n_kc && ok; i++) {
             ok = __all_sync(0xffffffffu, wait_or_abort(smem_u32(&x_full[xs]), xph, abort_flag));
             ok = ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_full[ws]), wph, abort_flag));
             if (!ok) {
@@ -344,7 +352,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 #pragma unroll
                 for (int j = 0; j < kBK / 16; j++) {
                     const uint64_t adesc = umma_desc_sw128(wa + 32u * j);
-                    const int slice = (kt - k_begin) * (kBK / 16) + j;
+                    const int slice = i * (kBK / 16) + j;
                     const uint32_t acc = p.n_acc > 1 ? 32u * (uint32_t)(slice % p.n_acc) : 0u;
                     const uint32_t first = p.n_acc > 1 ? (uint32_t)(slice < p.n_acc) : (uint32_t)(slice == 0);
                     for (int h = 0; h < p.nh; h++) {
@@ -379,8 +387,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         const uint32_t nl0 = 64u * q + 2u * lane, nl1 = nl0 + 1u;  // local W rows
         int rs = 0, ws = 0;
         uint32_t rph = 0, wph = 0;
-        for (int kt = k_begin; kt < k_end; kt++) {
-            const int i = kt - k_begin;
+        for (int i = 0; i < n_kc; i++) {
             // every lane waits; __all_sync keeps the outcome warp-uniform
             if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&r_full[rs]), rph, abort_flag))) {
                 flag_abort(abort_flag, p.status);
@@ -390,18 +397,27 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             bool dec = strip_ok;  // warp-uniform
             if (strip_ok) {
                 // columns 2l and 2l+1 of the strip: counts, starts, and the records of the
-                // warp's 8 columns (lanes 4g .. 4g+3 hold them)
+                // warp's 8 columns (lanes 4g .. 4g+3 hold them).  Only those 8 starts are
+                // needed: the kept count of the columns before them (one reduction) plus a
+                // scan within the 4 lanes.
                 const uint4 bw = *(const uint4*)(smem + p.off_raw + (size_t)rs * p.raw_stage_bytes +
                                                  512u * q + 16u * lane);
                 const int cl0 = __popc(bw.x), c0 = cl0 + __popc(bw.y);
                 const int cl1 = __popc(bw.z), c1 = cl1 + __popc(bw.w);
-                const int incl = warp_inclusive_scan(c0 + c1, lane);
+                const int cnt = c0 + c1;
+                const int before = (int)__reduce_add_sync(0xffffffffu, (lane >> 2) < g ? (uint32_t)cnt : 0u);
+                int loc = cnt;
+                const int l1 = __shfl_up_sync(0xffffffffu, loc, 1);
+                if ((lane & 3) >= 1) loc += l1;
+                const int l2 = __shfl_up_sync(0xffffffffu, loc, 2);
+                if ((lane & 3) >= 2) loc += l2;
+                const int incl = before + loc;  // exact for lanes 4g .. 4g+3
                 const uint32_t vb = rst_s + 1024u + (uint32_t)q * p.val_slot;
                 const uint32_t a0 = vb + 2u * (uint32_t)(incl - c0 - c1);
                 const uint32_t a1 = a0 + 2u * (uint32_t)c0;
                 // More values than the slot holds means the bitmaps and the tile pointers
                 // disagree: report it and decode the tile as empty rather than read past it.
-                if (2u * (uint32_t)__shfl_sync(0xffffffffu, incl, 31) > p.val_slot - 16u) {
+                if (2u * __reduce_add_sync(0xffffffffu, (uint32_t)cnt) > p.val_slot - 16u) {
                     if (lane == 0) raise_status(p.status, SPW_ERR_FORMAT);
                     dec = false;
                 } else if ((lane >> 2) == g) {
