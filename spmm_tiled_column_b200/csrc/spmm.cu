@@ -18,9 +18,11 @@
 //   * When output tiles are fewer than the SMs can hold, K is split across CTAs: each
 //     stores its fp32 partial tile; the last CTA of a tile (counted with an atomic) sums
 //     the partials in K order -- deterministic -- and writes fp16.
-//   * warp 0 (producer): lane 0 TMA-loads the X tiles (MT rows x 64, fp16, 128-byte
-//     swizzle, no multicast); lane 1, independently, 1-D bulk-copies the two TCB tiles
-//     (bitmaps + packed values) of each k-step.
+//   * warp 0, lane 0 (X producer): TMA-loads the X tiles (MT rows x 64, fp16, 128-byte
+//     swizzle, no multicast).  The last warp, lane 0 (TCB producer): 1-D bulk-copies the
+//     two TCB tiles (bitmaps + packed values) of each k-step.  Two warps, not two lanes
+//     of one: divergent lanes of a warp run one path at a time, so one ring's wait
+//     (a suspended mbarrier try_wait) would hold up the other ring's issue.
 //   * warp 1 (MMA): allocates TMEM; one thread issues tcgen05.mma.kind::f16 (A = decoded
 //     W, B = X, both K-major 128B-swizzled shared memory) and commits stage releases.
 //   * Decode (spw_spmv_tc) with a threshold above zero or a column set first writes x~ to
@@ -56,7 +58,8 @@ constexpr int kTileStrips = kTileRows / kStripRows;
 constexpr int kBK = 64;                 // one TCB k-tile
 constexpr int kMaxTokens = 512;         // tokens per CTA tile (TMEM columns)
 constexpr int kDecoderWarps = 16;
-constexpr int kThreads = 32 * (2 + kDecoderWarps);      // producer, MMA, decoders
+constexpr int kTcbWarp = 2 + kDecoderWarps;             // the TCB producer's warp (the last)
+constexpr int kThreads = 32 * (3 + kDecoderWarps);      // X producer, MMA, decoders, TCB producer
 constexpr uint32_t kWStageBytes = kTileRows * kBK * 2;  // 16 KB
 constexpr int kSmemLimit = 227 * 1024;
 
@@ -270,10 +273,10 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    int x_issued = 0, r_issued = 0;  // producer lanes 0 (X) and 1 (TCB): stages armed
-    if (warp == 0) {
+    int x_issued = 0, r_issued = 0;  // lane 0 of warp 0 (X) and of the TCB warp: stages armed
+    if (warp == 0 || warp == kTcbWarp) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {  // X ring
+        if (warp == 0 && lane == 0) {  // X ring
             asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap_x) : "memory");
             const int rows = p.MT / p.nh;  // TMA box height
             int xs = 0;
@@ -293,7 +296,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 x_issued++;
                 if (++xs == SX) { xs = 0; xph ^= 1u; }
             }
-        } else if (lane == 1) {  // TCB ring: the two tiles of each k-step
+        } else if (warp == kTcbWarp && lane == 0) {  // TCB ring: the two tiles of each k-step
             int rs = 0;
             uint32_t rph = 0;
             for (int i = 0; i < n_kc; i++) {
@@ -555,15 +558,15 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             }
         }
     }
-    if (warp == 0 && *abort_flag) {
-        // Drain the copies this CTA armed (bounded), each producer lane its own ring: for
-        // each slot, the phase of its last issue.  Phases a consumer already waited for
-        // return at once.
-        for (int i = 0; lane == 0 && i < SX && i < x_issued; i++) {
+    if ((warp == 0 || warp == kTcbWarp) && *abort_flag) {
+        // Drain the copies this CTA armed (bounded), each producer its own ring: for each
+        // slot, the phase of its last issue.  Phases a consumer already waited for return
+        // at once.
+        for (int i = 0; warp == 0 && lane == 0 && i < SX && i < x_issued; i++) {
             const int last = i + ((x_issued - 1 - i) / SX) * SX;
             (void)mbar_wait(smem_u32(&x_full[i]), (uint32_t)((last / SX) & 1));
         }
-        for (int i = 0; lane == 1 && i < SR && i < r_issued; i++) {
+        for (int i = 0; warp == kTcbWarp && lane == 0 && i < SR && i < r_issued; i++) {
             const int last = i + ((r_issued - 1 - i) / SR) * SR;
             (void)mbar_wait(smem_u32(&r_full[i]), (uint32_t)((last / SR) & 1));
         }
