@@ -204,6 +204,34 @@ int spw_spmv_group(int n, const spw_format* hdrs, const void* const* d_bufs,
                    const uint32_t* const* d_act_bits, uint16_t* const* d_ys, const int* ldys,
                    int B, float threshold, void* d_ws, uint64_t ws_bytes, void* stream);
 
+/* Workspace bytes spw_spmv_ffn needs for this gate/up pair and batch (0 if the headers
+ * are invalid or their shapes differ). */
+uint64_t spw_spmv_ffn_workspace_bytes(const spw_format* hdr_gate, const spw_format* hdr_up, int B);
+
+/* Fused FFN activation for decode ("Reduced Matrix Multiplication" §4.2: H = act(X W_up),
+ * keep the high-response channels of H, multiply with the matching rows of W_down; §3.2:
+ * SiLU's saturation is where the zeros come from), in the gated form of Llama's FFN:
+ *   g_b = fp16(W_gate . x_b), u_b = fp16(W_up . x_b)   (as spw_spmv with threshold 0)
+ *   h_b[r] = fp16(SiLU(g_b[r]) * u_b[r]),  SiLU(v) = v / (1 + e^-v), computed in fp32
+ *   act bit r set iff the threshold rule keeps h_b[r] for some b (as spw_select_threshold)
+ * in one launch: the gate and up layers are one decode group, and once both layers' rows
+ * of a 64-row strip are final the warp that finished second computes that strip's h and
+ * its two column-set words.  The outputs feed the down projection directly:
+ * spw_spmv(down, h, threshold, act_bits) computes only the kept columns.
+ *   hdr_gate, hdr_up: same N (intermediate size) and K (hidden size).
+ *   d_x:  B x K fp16 input rows at ldx, used as given (no input threshold).
+ *   d_h:  B x N fp16 output at ldh >= N (written).  d_act_bits: ceil(N/32) words (written).
+ *   d_ws: spw_spmv_ffn_workspace_bytes(...) bytes, zero before the first call and left so
+ *         (split-K and pair counters); it also holds g and u.  Concurrent calls must not
+ *         share a workspace.
+ * Deterministic.  Asynchronous.  Errors: INVALID_ARG (shapes differ, bad B, null
+ * pointer, ldh < N, threshold negative, NaN or Inf), ALIGNMENT, FORMAT, BUFFER_TOO_SMALL,
+ * CUDA; device-side waits and tile checks as spw_spmv. */
+int spw_spmv_ffn(const spw_format* hdr_gate, const void* d_buf_gate, const spw_format* hdr_up,
+                 const void* d_buf_up, const uint16_t* d_x, int B, int ldx, float threshold,
+                 uint16_t* d_h, int ldh, uint32_t* d_act_bits, void* d_ws, uint64_t ws_bytes,
+                 void* stream);
+
 /* Allocation-free decode.  The pages have no counterpart to this call; it exists for
  * callers that cannot call cudaMalloc, for example code running inside a framework that
  * reserved all device memory up front and forbids further allocation, or a path that may

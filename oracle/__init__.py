@@ -71,8 +71,13 @@ def _load():
         lib.orc_select_topk.argtypes = [P, i, i, i, i, P, P]
         lib.orc_spmv.argtypes = [P, i, P, i, i, i, P, i, i, f, P, P]
         lib.orc_spmm.argtypes = [P, i, P, i, i, i, P, i, i, P, i, P]
+        lib.orc_double_to_half.argtypes = [ctypes.c_double]
+        lib.orc_double_to_half.restype = ctypes.c_uint16
+        lib.orc_round_to_half.argtypes = [P, ctypes.c_int64, P]
+        lib.orc_silu_mul.argtypes = [P, P, i, i, i, P]
         for name in ("orc_tcb_query", "orc_tcb_encode", "orc_tcb_decode",
-                     "orc_select_threshold", "orc_select_topk", "orc_spmv", "orc_spmm"):
+                     "orc_select_threshold", "orc_select_topk", "orc_spmv", "orc_spmm",
+                     "orc_round_to_half", "orc_silu_mul"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -195,6 +200,38 @@ def spmm(W: np.ndarray, mask: np.ndarray, X: np.ndarray,
     _check(_load().orc_spmm(_ptr(Wb), K, _ptr(mask), K, N, K, _ptr(Xb), M, K, _ptr(rows),
                             n_rows, _ptr(Y)), "orc_spmm")
     return Y
+
+
+def round_to_half(v: np.ndarray) -> np.ndarray:
+    """fp64 values -> binary16 (float16 array), round to nearest, ties to even."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.zeros(v.shape, dtype=np.uint16)
+    _check(_load().orc_round_to_half(_ptr(v), v.size, _ptr(out)), "orc_round_to_half")
+    return out.view(np.float16)
+
+
+def silu_mul(g: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """h = fp16(SiLU(g) * u) element-wise for fp16 B x N arrays (float16 result)."""
+    gb = _half_bits(np.atleast_2d(g))
+    ub = _half_bits(np.atleast_2d(u))
+    assert gb.shape == ub.shape
+    B, N = gb.shape
+    h = np.zeros((B, N), dtype=np.uint16)
+    _check(_load().orc_silu_mul(_ptr(gb), _ptr(ub), B, N, N, _ptr(h)), "orc_silu_mul")
+    return h.view(np.float16)
+
+
+def ffn(Wg: np.ndarray, mask_g: np.ndarray, Wu: np.ndarray, mask_u: np.ndarray,
+        x: np.ndarray, t: float = 0.0) -> tuple[np.ndarray, np.ndarray]:
+    """Fused FFN activation of a decode batch: (h float16 B x N, act_bits of h).
+
+    g and u are the gate and up products rounded once to fp16 (what the two decode calls
+    return), h = fp16(SiLU(g) * u), and the column set is the threshold rule on h."""
+    g = round_to_half(spmv(Wg, mask_g, x, 0.0, None))
+    u = round_to_half(spmv(Wu, mask_u, x, 0.0, None))
+    h = silu_mul(g, u)
+    bits, _ = select_threshold(h, t)
+    return h, bits
 
 
 def rel_err(y, y_ref) -> float:

@@ -37,6 +37,9 @@
  *   orc_select_topk      active-column set for top-k by summed |x|       [RMM] §5.1.
  *   orc_spmv             y_b = W_masked . x~_b in fp64                   [RMM] §4.2, [3LF] §1.
  *   orc_spmm             Y = X . W_masked^T in fp64 (optionally some rows) [3LF] §1, §2.1.
+ *   orc_double_to_half   IEEE-754 binary16 encoding, round to nearest, ties to even
+ *   orc_round_to_half    (and its element-wise form).
+ *   orc_silu_mul         h = fp16(SiLU(g) * u) for the gated FFN    [RMM] §4.2, §3.2.
  *
  * Pins: tests/test_oracle_*.py check every function against things fixed outside this
  * file: numpy's binary16 decoder over all 65536 bit patterns, hand-derived TCB buffers
@@ -413,5 +416,60 @@ int orc_spmm(const uint16_t* W, int ldw, const uint8_t* mask, int ld_mask, int N
             Y[(size_t)i * N + n] = acc;
         }
     }
+    return ORC_OK;
+}
+
+/* IEEE-754 binary16 encoding of v: round to nearest, ties to even; overflow to infinity,
+ * NaN to a quiet NaN with the sign kept, gradual underflow to subnormals and zero. */
+uint16_t orc_double_to_half(double v) {
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    if (isnan(v)) return (uint16_t)(sign | 0x7E00u);
+    double a = fabs(v);
+    if (isinf(a)) return (uint16_t)(sign | 0x7C00u);
+    /* a = m * 2^e with m in [0.5, 1); the binary16 exponent of a is e - 1 */
+    int e;
+    double m = frexp(a, &e);
+    if (a == 0.0) return sign;
+    int exp16 = e - 1;                      /* a in [2^exp16, 2^(exp16+1)) */
+    double q;                               /* a in units of the target's last place */
+    if (exp16 < -14) q = ldexp(a, 24);      /* subnormal: units of 2^-24 */
+    else q = ldexp(m, 11);                  /* normal: 11 significant bits, in [1024, 2048) */
+    double r = floor(q);
+    double frac = q - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    if (exp16 < -14) {
+        /* r counts 2^-24 units; 1024 of them is the smallest normal, which the bit pattern
+         * below also encodes correctly (exponent field 1, fraction 0) */
+        return (uint16_t)(sign | (uint16_t)r);
+    }
+    if (r == 2048.0) {                      /* rounding carried into the next binade */
+        r = 1024.0;
+        exp16 += 1;
+    }
+    if (exp16 > 15) return (uint16_t)(sign | 0x7C00u);
+    return (uint16_t)(sign | (uint16_t)((exp16 + 15) << 10) | (uint16_t)((int)r - 1024));
+}
+
+/* Element-wise orc_double_to_half over n values. */
+int orc_round_to_half(const double* v, int64_t n, uint16_t* out) {
+    if ((!v || !out) && n > 0) return ORC_ERR_ARG;
+    for (int64_t i = 0; i < n; i++) out[i] = orc_double_to_half(v[i]);
+    return ORC_OK;
+}
+
+/* Gated FFN activation ("Reduced Matrix Multiplication" §4.2: H = act(X W_up), then keep
+ * the high-response channels of H; §3.2: SiLU's saturation makes many of them near zero),
+ * in Llama's gated form: h[b][r] = fp16(SiLU(g[b][r]) * u[b][r]) with SiLU(v) = v / (1 +
+ * e^-v), from fp16 gate and up outputs g and u, computed in fp64 and rounded once.
+ * g, u and h are B x N at leading dimension ld. */
+int orc_silu_mul(const uint16_t* g, const uint16_t* u, int B, int N, int ld, uint16_t* h) {
+    if (!g || !u || !h || B < 0 || N < 0 || ld < N) return ORC_ERR_ARG;
+    for (int b = 0; b < B; b++)
+        for (int r = 0; r < N; r++) {
+            double gv = orc_half_to_double(g[(size_t)b * ld + r]);
+            double uv = orc_half_to_double(u[(size_t)b * ld + r]);
+            double silu = gv / (1.0 + exp(-gv));
+            h[(size_t)b * ld + r] = orc_double_to_half(silu * uv);
+        }
     return ORC_OK;
 }

@@ -71,6 +71,8 @@ SIGNATURES = {
     "spw_spmv_group": ([_I, _FP, _P, _P, _P, _P, _P, _P, _I, _F, _P, _U64, _P], _I),
     "spw_spmv_noalloc_max_scratch_bytes": ([], _U64),
     "spw_spmv_noalloc": ([_FP, _P, _P, _I, _I, _F, _P, _P, _I, _P], _I),
+    "spw_spmv_ffn_workspace_bytes": ([_FP, _FP, _I], _U64),
+    "spw_spmv_ffn": ([_FP, _P, _FP, _P, _P, _I, _I, _F, _P, _I, _P, _P, _U64, _P], _I),
 }
 
 
@@ -365,6 +367,36 @@ def spw_spmv_tc(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.0,
         ctypes.byref(h), _ptr(buf), _ptr(x2), B, ldx, float(threshold), _ptr(act_bits),
         _ptr(y2), ldy, _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
     return y
+
+
+def spw_spmv_ffn_workspace_bytes(hdr_gate, hdr_up, B: int) -> int:
+    return int(lib().spw_spmv_ffn_workspace_bytes(ctypes.byref(_hdr(hdr_gate)),
+                                                  ctypes.byref(_hdr(hdr_up)), B))
+
+
+def spw_spmv_ffn(hdr_gate, buf_gate: torch.Tensor, hdr_up, buf_up: torch.Tensor, x: torch.Tensor,
+                 threshold: float = 0.0, h: torch.Tensor | None = None,
+                 act_bits: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                 stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Fused FFN activation: h (B x N fp16) = SiLU(W_gate x) * (W_up x) and the column-set
+    words of h under the threshold rule, in one launch.  ws: a zero-initialised uint8
+    workspace of spw_spmv_ffn_workspace_bytes(hdr_gate, hdr_up, B) bytes (allocated here
+    when not given).  Returns (h, act_bits)."""
+    hg, hu = _hdr(hdr_gate), _hdr(hdr_up)
+    x2, ldx = _rows(_half(x, "x"), "x")
+    B = x2.shape[0]
+    if h is None:
+        h = torch.empty((B, hg.N), dtype=torch.float16, device=x.device)
+    h2, ldh = _rows(_half(h, "h"), "h")
+    if act_bits is None:
+        act_bits = torch.empty(((hg.N + 31) // 32,), dtype=torch.int32, device=x.device)
+    if ws is None:
+        need = spw_spmv_ffn_workspace_bytes(hg, hu, B)
+        ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=x.device)
+    _check("spw_spmv_ffn", lib().spw_spmv_ffn(
+        ctypes.byref(hg), _ptr(buf_gate), ctypes.byref(hu), _ptr(buf_up), _ptr(x2), B, ldx,
+        float(threshold), _ptr(h2), ldh, _ptr(act_bits), _ptr(ws), ws.numel(), _stream(stream)))
+    return h, act_bits
 
 
 def spw_last_device_status(stream=None) -> int:

@@ -86,6 +86,13 @@ struct SpmvParams {
     uint32_t warp_smem;
     float t;
     int neg2;  // -2, passed at run time so the address step stays a multiply-add
+    // FFN mode (spw_spmv_ffn): layers 0 and 1 are gate and up of one FFN; h = SiLU(g) * u
+    // and its column-set bits are written once both layers' rows of a strip are final.
+    uint16_t* ffn_h;      // null: not FFN mode
+    int ffn_ldh;
+    uint32_t* ffn_bits;   // ceil(N / 32) words
+    uint32_t* ffn_pairs;  // per strip: finished layers (0, 1 or 2; left at 0)
+    float ffn_t;
 };
 
 __host__ __device__ constexpr int xt_stride(int B) {
@@ -362,6 +369,54 @@ __device__ inline void load_act(const SpmvParams& p, const Cursor& c, int lane, 
     if (L.act_bits && col < L.K) aw = (__ldg(L.act_bits + (col >> 5)) >> (col & 31)) & 3u;
 }
 
+// FFN mode, after a warp wrote the final fp16 outputs of strip s of the gate or the up
+// layer: the second of the two to finish computes, for the strip's rows r and every
+// batch row b, h[b][r] = fp16(SiLU(g[b][r]) * u[b][r]) in fp32 from the fp16 outputs
+// (SiLU(v) = v / (1 + e^-v)), and the strip's two column-set words: bit r is set when the
+// threshold rule keeps h[b][r] for some b.  The outputs are read back from L2 after the
+// pair counter's acquire; the counter is reset for the next call.
+template <int B>
+__device__ void ffn_strip(const SpmvParams& p, int s, int lane) {
+    __syncwarp();  // this warp's output stores before the count (release below)
+    uint32_t old = 0;
+    if (lane == 0) old = atom_add_acq_rel_gpu(p.ffn_pairs + s, 1u);
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (old != 1u) return;
+    __syncwarp();  // every lane's loads below after lane 0's acquire
+    __threadfence();
+    const SpmvLayer& G = p.L[0];
+    const SpmvLayer& U = p.L[1];
+    const int r0 = s * kStripRows + 2 * lane;
+    bool keep0 = false, keep1 = false;
+#pragma unroll 1
+    for (int b = 0; b < B; b++) {
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            const int r = r0 + e;
+            if (r >= G.N) continue;
+            const float g = __half2float(__ushort_as_half(__ldcg(G.y + (size_t)b * G.ldy + r)));
+            const float u = __half2float(__ushort_as_half(__ldcg(U.y + (size_t)b * U.ldy + r)));
+            const uint16_t h = __half_as_ushort(__float2half_rn(g / (1.0f + expf(-g)) * u));
+            p.ffn_h[(size_t)b * p.ffn_ldh + r] = h;
+            const bool k = passes_threshold(h, p.ffn_t);
+            if (e == 0) keep0 |= k; else keep1 |= k;
+        }
+    }
+    const uint32_t m0 = __ballot_sync(0xffffffffu, keep0), m1 = __ballot_sync(0xffffffffu, keep1);
+    if (lane == 0) {
+        uint32_t w0 = 0u, w1 = 0u;  // rows 64 s .. 64 s + 31 and 64 s + 32 .. 64 s + 63
+#pragma unroll
+        for (int l = 0; l < 16; l++) {
+            w0 |= (((m0 >> l) & 1u) << (2 * l)) | (((m1 >> l) & 1u) << (2 * l + 1));
+            w1 |= (((m0 >> (l + 16)) & 1u) << (2 * l)) | (((m1 >> (l + 16)) & 1u) << (2 * l + 1));
+        }
+        const int nw = (G.N + 31) / 32;
+        if (2 * s < nw) p.ffn_bits[2 * s] = w0;
+        if (2 * s + 1 < nw) p.ffn_bits[2 * s + 1] = w1;
+        p.ffn_pairs[s] = 0u;
+    }
+}
+
 // Consumer warp gw: its tile range, decoded from its ring; partial sums flushed per strip.
 template <int B>
 __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lane) {
@@ -502,6 +557,7 @@ __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lan
         const int g_last = (int)warp_of_tile((long long)first + nk - 1, PW, T);
         const int count = g_last - g_first + 1;
         const int r0 = s * kStripRows + 2 * lane;
+        bool finished = false;  // this warp wrote the strip's final outputs (warp-uniform)
         if (count == 1) {
 #pragma unroll
             for (int b = 0; b < B; b++) {
@@ -509,6 +565,7 @@ __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lan
                 if (r0 + 1 < L.N)
                     L.y[(size_t)b * L.ldy + r0 + 1] = __half_as_ushort(__float2half_rn(acc1[b]));
             }
+            finished = true;
         } else {
             // Publish this piece: store the partials, then one release atomic per warp.
             const int idx = gw - g_first;
@@ -560,8 +617,10 @@ __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lan
                     }
                 }
                 if (lane == 0) L.counters[s] = 0u;
+                finished = true;
             }
         }
+        if (p.ffn_h && finished) ffn_strip<B>(p, s, lane);
 #pragma unroll
         for (int b = 0; b < B; b++) acc0[b] = acc1[b] = 0.0f;
     }
@@ -706,10 +765,21 @@ int launch(const Plan& pl, const SpmvParams& prm, cudaStream_t s) {
 }
 
 // Checks shared by spw_spmv and spw_spmv_group, and the launch.
+// FFN mode outputs (spw_spmv_ffn): h, its column-set words, the per-strip pair counters
+// and the threshold applied to h.
+struct FfnOut {
+    uint16_t* h;
+    int ldh;
+    uint32_t* bits;
+    uint32_t* pairs;
+    float t;
+};
+
 int decode_group_launch(int n, const spw_format* hdrs, const void* const* bufs,
                         const uint16_t* const* xs, const int* ldxs,
                         const uint32_t* const* act_bits, uint16_t* const* ys, const int* ldys,
-                        int B, float threshold, void* d_ws, uint64_t ws_bytes, cudaStream_t s) {
+                        int B, float threshold, void* d_ws, uint64_t ws_bytes, cudaStream_t s,
+                        const FfnOut* ffn = nullptr) {
     if (n < 1 || n > kMaxGroup || !hdrs || !bufs || !xs || !ldxs || !ys || !ldys)
         return SPW_ERR_INVALID_ARG;
     if (!d_ws || B < 1 || B > 16) return SPW_ERR_INVALID_ARG;
@@ -765,6 +835,13 @@ int decode_group_launch(int n, const spw_format* hdrs, const void* const* bufs,
     prm.warp_smem = pl.warp_smem;
     prm.t = threshold;
     prm.neg2 = -2;
+    if (ffn) {
+        prm.ffn_h = ffn->h;
+        prm.ffn_ldh = ffn->ldh;
+        prm.ffn_bits = ffn->bits;
+        prm.ffn_pairs = ffn->pairs;
+        prm.ffn_t = ffn->t;
+    }
     switch (B) {
 #define SPW_CASE(b) \
     case b: return launch<b>(pl, prm, s);
@@ -776,12 +853,67 @@ int decode_group_launch(int n, const spw_format* hdrs, const void* const* bufs,
     return SPW_ERR_INVALID_ARG;
 }
 
+// Workspace of spw_spmv_ffn: the two-layer decode group's section, the per-strip pair
+// counters, then the fp16 gate and up outputs (B rows of ld halves each).
+struct FfnWorkspace {
+    uint64_t group, pairs, g, u, total;
+    int ld;
+};
+
+int ffn_workspace(const spw_format* hdr_gate, const spw_format* hdr_up, int B, FfnWorkspace* w) {
+    if (!hdr_gate || !hdr_up || B < 1 || B > 16) return SPW_ERR_INVALID_ARG;
+    int rc = check_header(hdr_gate);
+    if (rc == SPW_OK) rc = check_header(hdr_up);
+    if (rc != SPW_OK) return rc;
+    if (hdr_gate->N != hdr_up->N || hdr_gate->K != hdr_up->K) return SPW_ERR_INVALID_ARG;
+    const spw_format hd[2] = {*hdr_gate, *hdr_up};
+    Plan pl;
+    rc = make_plan(2, hd, B, &pl);
+    if (rc != SPW_OK) return rc;
+    w->ld = (int)round_up_u64(hdr_gate->N, 8);
+    w->group = round_up_u64(pl.ws_bytes, 256);
+    w->pairs = round_up_u64(4ull * hdr_gate->n_strips, 256);
+    const uint64_t out = round_up_u64(2ull * (uint64_t)B * (uint64_t)w->ld, 256);
+    w->g = w->group + w->pairs;
+    w->u = w->g + out;
+    w->total = w->u + out;
+    return SPW_OK;
+}
+
 }  // namespace
 }  // namespace spw
 
 using namespace spw;
 
 extern "C" {
+
+uint64_t spw_spmv_ffn_workspace_bytes(const spw_format* hdr_gate, const spw_format* hdr_up, int B) {
+    FfnWorkspace w;
+    return ffn_workspace(hdr_gate, hdr_up, B, &w) == SPW_OK ? w.total : 0;
+}
+
+int spw_spmv_ffn(const spw_format* hdr_gate, const void* d_buf_gate, const spw_format* hdr_up,
+                 const void* d_buf_up, const uint16_t* d_x, int B, int ldx, float threshold,
+                 uint16_t* d_h, int ldh, uint32_t* d_act_bits, void* d_ws, uint64_t ws_bytes,
+                 void* stream) {
+    FfnWorkspace w;
+    const int rc = ffn_workspace(hdr_gate, hdr_up, B, &w);
+    if (rc != SPW_OK) return rc;
+    if (!d_h || !d_act_bits || !d_ws || ldh < (int)hdr_gate->N) return SPW_ERR_INVALID_ARG;
+    if (!(threshold >= 0.0f) || isinf(threshold)) return SPW_ERR_INVALID_ARG;
+    if (!aligned16(d_h) || !aligned16(d_act_bits) || !aligned16(d_ws)) return SPW_ERR_ALIGNMENT;
+    if (ws_bytes < w.total) return SPW_ERR_BUFFER_TOO_SMALL;
+    uint8_t* ws = (uint8_t*)d_ws;
+    const spw_format hd[2] = {*hdr_gate, *hdr_up};
+    const void* bufs[2] = {d_buf_gate, d_buf_up};
+    const uint16_t* xs[2] = {d_x, d_x};
+    const int ldxs[2] = {ldx, ldx};
+    uint16_t* ys[2] = {(uint16_t*)(ws + w.g), (uint16_t*)(ws + w.u)};
+    const int ldys[2] = {w.ld, w.ld};
+    const FfnOut ffn = {d_h, ldh, d_act_bits, (uint32_t*)(ws + w.group), threshold};
+    return decode_group_launch(2, hd, bufs, xs, ldxs, nullptr, ys, ldys, B, 0.0f, d_ws, w.group,
+                               (cudaStream_t)stream, &ffn);
+}
 
 uint64_t spw_spmv_workspace_bytes(const spw_format* hdr, int B) {
     return spw_spmv_group_workspace_bytes(1, hdr, B);

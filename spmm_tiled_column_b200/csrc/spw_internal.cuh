@@ -170,6 +170,13 @@ __device__ inline uint32_t atom_add_release_gpu(uint32_t* p, uint32_t v) {
     return old;
 }
 
+// Device-scope add with acquire and release semantics; returns the old value.
+__device__ inline uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 // Programmatic dependent launch: wait until the previous kernel on the stream has
 // completed and its memory is visible / allow the next kernel to begin launching.
 // Both are no-ops for a kernel launched without the programmatic attribute.

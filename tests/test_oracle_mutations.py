@@ -24,6 +24,7 @@ FORMAT_PINS = "format"
 SELECT_PINS = "select"
 PRODUCT_PINS = "products"
 HALF_PINS = "half"
+FFN_PINS = "ffn"
 
 CHILD = {
     "half": "import test_oracle_half as H; H.test_all_half_patterns_match_numpy()",
@@ -42,6 +43,10 @@ CHILD = {
                  "P.test_spmv_act_bits_restrict_columns(); P.test_identity_is_exact()\n"
                  "P.test_diagonal_is_exact(); P.test_spmm_matches_numpy_and_rows()\n"
                  "P.test_spmm_transposed_operand_would_fail()"),
+    "ffn": ("import test_oracle_ffn as Q\n"
+            "Q.test_round_to_half_matches_numpy(); Q.test_round_to_half_round_trip_and_ties()\n"
+            "Q.test_silu_mul_worked_value(); Q.test_silu_odd_part_identity()\n"
+            "Q.test_silu_limits_and_zeros()"),
 }
 
 MUTANTS = [
@@ -71,6 +76,13 @@ MUTANTS = [
      "orc_half_to_double(X[(size_t)m * ldx + (K - 1 - k)]) *", [PRODUCT_PINS]),
     ("spmv_dropped_term", "acc += orc_half_to_double(W[(size_t)n * ldw + k]) * v;",
      "if (k + 1 < K) acc += orc_half_to_double(W[(size_t)n * ldw + k]) * v;", [PRODUCT_PINS]),
+    ("silu_exponent_sign", "double silu = gv / (1.0 + exp(-gv));",
+     "double silu = gv / (1.0 + exp(gv));", [FFN_PINS]),
+    ("silu_mul_dropped_factor", "h[(size_t)b * ld + r] = orc_double_to_half(silu * uv);",
+     "h[(size_t)b * ld + r] = orc_double_to_half(silu);", [FFN_PINS]),
+    ("half_ties_away", "if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;",
+     "if (frac >= 0.5) r += 1.0;", [FFN_PINS]),
+    ("half_no_carry", "    if (r == 2048.0) {", "    if (r == 4096.0) {", [FFN_PINS]),
 ]
 
 
