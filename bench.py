@@ -317,6 +317,42 @@ def run_ours(args, rank, world, local_rank):
             per_linear[name] = {"us": round(us, 3), "GB/s": round(nb / (us * 1e-6) / 1e9, 1),
                                 "bytes": int(nb)}
 
+    # Fused FFN activation (spw_spmv_ffn): the gate and up decode plus h = SiLU(g) * u and
+    # its column set in one launch, against the same work as separate launches (grouped
+    # decode, torch's SiLU and product, spw_select_threshold).  The threshold is the
+    # median |h| of this input, so about half of the down projection's columns are kept.
+    gu = GROUPS.index(["gate", "up"])
+    _, hdrs_gu, _, xd_gu, _, _ = gdata[0][gu]
+    fws = [torch.zeros(spw.spw_spmv_ffn_workspace_bytes(hdrs_gu[0], hdrs_gu[1], 1), dtype=torch.uint8,
+                       device=dev) for _ in range(N_ROTATE)]
+    h_out = torch.empty((1, hdrs_gu[0].N), dtype=torch.float16, device=dev)
+    bits_out = torch.empty(((hdrs_gu[0].N + 31) // 32 + 3,), dtype=torch.int32, device=dev)
+    with torch.cuda.stream(stream):
+        h0, _ = spw.spw_spmv_ffn(hdrs_gu[0], gdata[0][gu][2][0], hdrs_gu[1], gdata[0][gu][2][1], xd_gu,
+                                 0.0, h_out, bits_out, fws[0])
+    stream.synchronize()
+    t_ffn = float(h0.float().abs().median().item())
+
+    def fused(r):
+        _, hdrs, bufs, xd, _, _ = gdata[r][gu]
+        spw.spw_spmv_ffn(hdrs[0], bufs[0], hdrs[1], bufs[1], xd, t_ffn, h_out, bits_out, fws[r])
+
+    def unfused(r):
+        _, hdrs, bufs, xd, ys, ws = gdata[r][gu]
+        spw.spw_spmv_group(hdrs, bufs, [xd, xd], 0.0, None, ys, ws)
+        torch.mul(torch.nn.functional.silu(ys[0]), ys[1], out=h_out)
+        spw.spw_select_threshold(h_out, t_ffn, bits_out)
+
+    fused_us = time_graphs(fused)
+    unfused_us = time_graphs(unfused)
+    gu_bytes = sum(decode_bytes(*layer[idx[n]][1:]) for n in ("gate", "up"))
+    ffn_fused = {"us": round(fused_us, 3), "GB/s": round(gu_bytes / (fused_us * 1e-6) / 1e9, 1),
+                 "separate_launches_us": round(unfused_us, 3),
+                 "speedup": round(unfused_us / fused_us, 3), "threshold": round(t_ffn, 5),
+                 "how": "spw_spmv_ffn (gate+up decode, h = SiLU(g)*u, column set of h) vs "
+                        "spw_spmv_group + torch silu/mul + spw_select_threshold; graph replays"}
+    assert spw.spw_last_device_status() == spw.SPW_OK
+
     # dense cuBLAS comparison at the same shapes (fp16 in, fp32 accumulate)
     dense = {}
     for j, name in enumerate(LAYERS[:: 1]):
@@ -454,6 +490,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk.summary(),
         "e2e": e2e,
         "dense_cublas_decode": dense,
+        "ffn_fused": ffn_fused,
         "dense_cublas_step": dense_step,
         "prefill": prefill,
     }
