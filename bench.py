@@ -353,6 +353,30 @@ def run_ours(args, rank, world, local_rank):
                         "spw_spmv_group + torch silu/mul + spw_select_threshold; graph replays"}
     assert spw.spw_last_device_status() == spw.SPW_OK
 
+    # The decoder layer's step with the fused FFN activation: [q,k,v], [o], then the
+    # gate/up pair emits h and its column set, which the down projection consumes (its
+    # input is h of this layer rather than the synthetic SiLU(g)*u of the main step).
+    dn = GROUPS.index(["down"])
+    h_host = h_out.view(torch.int16).cpu().numpy().view(np.float16)
+    down_j = idx["down"]
+    ffn_step_bytes = (sum(decode_bytes(*layer[idx[n]][1:]) for n in ("q", "k", "v", "o", "gate", "up"))
+                      + decode_bytes(layer[down_j][1], layer[down_j][2], h_host, t_ffn))
+
+    def ffn_step(r):
+        for gi in (GROUPS.index(["q", "k", "v"]), GROUPS.index(["o"])):
+            _, hdrs, bufs, xd, ys, ws = gdata[r][gi]
+            spw.spw_spmv_group(hdrs, bufs, [xd] * len(bufs), 0.0, None, ys, ws)
+        fused(r)
+        _, hdrs, bufs, _, ys, ws = gdata[r][dn]
+        spw.spw_spmv_group(hdrs, bufs, [h_out], t_ffn, [bits_out], ys, ws)
+
+    ffn_step_us = time_graphs(ffn_step)
+    ffn_fused["layer_step"] = {
+        "us": round(ffn_step_us, 3), "GB/s": round(ffn_step_bytes / (ffn_step_us * 1e-6) / 1e9, 1),
+        "bytes": int(ffn_step_bytes),
+        "how": "[q,k,v], [o], spw_spmv_ffn(gate, up), down on h with its column set; 4 launches"}
+    assert spw.spw_last_device_status() == spw.SPW_OK
+
     # dense cuBLAS comparison at the same shapes (fp16 in, fp32 accumulate)
     dense = {}
     for j, name in enumerate(LAYERS[:: 1]):
