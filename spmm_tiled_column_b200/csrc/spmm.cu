@@ -76,7 +76,9 @@ struct SpmmParams {
     int n_strips, n_ktiles;
     int MT, nh;                 // tokens per tile; MMAs per k-slice (MT / nh each)
     int n_acc;                  // independent accumulators (32 columns apart) for MT <= 32
-    int ksplit;
+    int ksplit;                 // K parts of each split tile (1: no split tiles)
+    int n_whole;                // tiles 0 .. n_whole-1 run whole; the rest are split
+    int m_tiles;                // token tiles (tile t: token tile t % m_tiles, weight rows t / m_tiles)
     int sx, sr, sw;             // X, raw-tile and decoded-weight stage counts
     uint32_t x_stage_bytes;     // MT * 128
     uint32_t raw_stage_bytes;   // 1024 + 2 * val_slot
@@ -206,18 +208,26 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * p.MT;
-    const int n0 = blockIdx.y * kTileRows;
+    // This CTA's output tile and K range: CTA c < n_whole computes tile c whole; the others
+    // compute part (c - n_whole) % ksplit of split tile n_whole + (c - n_whole) / ksplit.
+    const int cta = blockIdx.x;
+    const bool split = cta >= p.n_whole;
+    const int tile = split ? p.n_whole + (cta - p.n_whole) / p.ksplit : cta;
+    const int parts = split ? p.ksplit : 1;
+    const int kz = split ? (cta - p.n_whole) % p.ksplit : 0;
+    const int stile = tile - p.n_whole;  // index among the split tiles (when split)
+    const int mt = tile % p.m_tiles, ntile = tile / p.m_tiles;
+    const int m0 = mt * p.MT;
+    const int n0 = ntile * kTileRows;
     const int s0 = n0 / kStripRows;
     const int nk = p.n_ktiles;
-    const int kz = blockIdx.z;
-    const int k_begin = (int)((long long)kz * nk / p.ksplit);
-    const int k_end = (int)((long long)(kz + 1) * nk / p.ksplit);
+    const int k_begin = (int)((long long)kz * nk / parts);
+    const int k_end = (int)((long long)(kz + 1) * nk / parts);
     // Every role walks the CTA's k-steps from a start rotated by the weight-row tile: the
     // CTAs that share an X tile then read different k-columns of it at any moment instead
     // of all hitting the same L2 lines together.
     const int n_kc = k_end - k_begin;
-    const int k_rot = n_kc > 0 ? (int)(blockIdx.y % (unsigned)n_kc) : 0;
+    const int k_rot = n_kc > 0 ? ntile % n_kc : 0;
     auto kstep = [&](int i) { return k_begin + (i + k_rot < n_kc ? i + k_rot : i + k_rot - n_kc); };
     const int SX = p.sx, SR = p.sr;
 
@@ -473,8 +483,8 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             const int part_of = (warp - 2) >> 2;  // which 32-column chunks: j % 4 == part_of
             const int row = 32 * quarter + lane;
             const int n = n0 + row;
-            const size_t tile = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
-            float* part = p.partials + (tile * p.ksplit + kz) * (size_t)p.MT * kTileRows;
+            float* part = split ? p.partials + ((size_t)stile * p.ksplit + kz) * (size_t)p.MT * kTileRows
+                                : nullptr;
             // 32 accumulator columns per load; the allocation is a power of two >= 32, so a
             // tile of 16 tokens reads 16 valid columns and 16 unused ones.
             // accumulators written by this CTA's k-slices (each k-slice writes one of them)
@@ -489,7 +499,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     for (int c = 0; c < 32; c++) r[c] = __float_as_uint(__uint_as_float(r[c]) + __uint_as_float(r2[c]));
                 }
                 const int lim = min(32, p.MT - 32 * j);
-                if (p.ksplit > 1) {
+                if (split) {
 #pragma unroll
                     for (int c = 0; c < 32; c++)
                         if (c < lim) part[(size_t)(32 * j + c) * kTileRows + row] = __uint_as_float(r[c]);
@@ -502,7 +512,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     }
                 }
             }
-            if (p.ksplit > 1) __threadfence();  // partials before the arrival below
+            if (split) __threadfence();  // partials before the arrival below
         } else {
             flag_abort(abort_flag, p.status);
         }
@@ -510,37 +520,45 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 
     tc_fence_before();
     __syncthreads();
-    if (p.ksplit > 1 && !*abort_flag) {
+    if (split && !*abort_flag) {
         // Split-K: the last CTA of this output tile sums every partial in K order.
-        const size_t tile = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
         if (threadIdx.x == 0) {
-            const uint32_t old = atom_add_release_gpu(&p.counters[tile], 1u);
+            const uint32_t old = atom_add_release_gpu(&p.counters[stile], 1u);
             *last_flag = old == (uint32_t)(p.ksplit - 1) ? 1u : 0u;
-            if (*last_flag) p.counters[tile] = 0u;
+            if (*last_flag) p.counters[stile] = 0u;
         }
         __syncthreads();
         if (*last_flag) {
             __threadfence();
             // Four consecutive rows of one token per thread (16-byte loads), four such
-            // groups in flight; the partials are summed in split order (deterministic).
-            const float4* base = (const float4*)(p.partials + tile * p.ksplit * (size_t)p.MT * kTileRows);
+            // groups, two partials at a time: 8 loads in flight per thread.  The partials
+            // are summed in split order (deterministic).
+            const float4* base = (const float4*)(p.partials + (size_t)stile * p.ksplit * (size_t)p.MT * kTileRows);
             const int n4 = p.MT * kTileRows / 4, stride4 = p.MT * kTileRows / 4;
             for (int i0 = threadIdx.x; i0 < n4; i0 += 4 * kThreads) {
                 float4 acc[4];
 #pragma unroll
                 for (int u = 0; u < 4; u++) acc[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                for (int z = 0; z < p.ksplit; z++) {
+                for (int z0 = 0; z0 < p.ksplit; z0 += 2) {
+                    float4 v[2][4];
 #pragma unroll
-                    for (int u = 0; u < 4; u++) {
-                        const int i = i0 + u * kThreads;
-                        if (i < n4) {
-                            const float4 v = __ldcg(base + (size_t)z * stride4 + i);
-                            acc[u].x += v.x;
-                            acc[u].y += v.y;
-                            acc[u].z += v.z;
-                            acc[u].w += v.w;
+                    for (int dz = 0; dz < 2; dz++)
+#pragma unroll
+                        for (int u = 0; u < 4; u++) {
+                            const int i = i0 + u * kThreads;
+                            v[dz][u] = (z0 + dz < p.ksplit && i < n4)
+                                           ? __ldcg(base + (size_t)(z0 + dz) * stride4 + i)
+                                           : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                         }
-                    }
+#pragma unroll
+                    for (int dz = 0; dz < 2; dz++)
+#pragma unroll
+                        for (int u = 0; u < 4; u++) {
+                            acc[u].x += v[dz][u].x;
+                            acc[u].y += v[dz][u].y;
+                            acc[u].z += v[dz][u].z;
+                            acc[u].w += v[dz][u].w;
+                        }
                 }
 #pragma unroll
                 for (int u = 0; u < 4; u++) {
@@ -602,7 +620,7 @@ int get_encoder() {
 }
 
 struct SpmmPlan {
-    int MT, nh, n_acc, m_tiles, n_tiles, ksplit, sx, sr, sw, ctas_per_sm;
+    int MT, nh, n_acc, m_tiles, n_tiles, ksplit, n_whole, sx, sr, sw, ctas_per_sm;
     uint32_t x_stage_bytes, val_slot, raw_stage_bytes, tmem_cols;
     uint32_t off_w, off_raw, off_rec, off_tptr, off_bar;
     size_t smem;
@@ -614,16 +632,20 @@ struct SpmmPlan {
 int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl) {
     const int sms = device_sm_count();
     if (sms <= 0) return SPW_ERR_CUDA;
-    // Token tile (512, 256 or 128 tokens, or all M when smaller) and split-K factor from a
-    // small cost model in microseconds, per CTA wave: k-steps x max(decode ~0.7, MMA
-    // ~0.76 x MT / 512) plus, when K is split, the fp32 partial tile written and summed
-    // (~0.1 GB/ms per CTA).  One CTA per SM.
+    // Token tile (512, 256 or 128 tokens, or all M when smaller) and split-K from a small
+    // cost model in microseconds: k-steps x max(decode ~0.7, MMA ~0.76 x MT / 512) per CTA,
+    // plus, when K is split, the fp32 partial tile written and summed (~0.1 GB/ms per
+    // CTA).  One CTA per SM.  Two shapes of split: every tile in k parts (whole waves), or
+    // -- when the tiles need more than one wave but fewer than two -- the first F tiles
+    // whole and the rest in k parts that fill the SMs as the whole tiles finish (the span
+    // estimated as in-order list scheduling).
     pl->n_tiles = (int)((h->N + kTileRows - 1) / kTileRows);
     const long long slots = sms;
     const long long nk_all = h->n_ktiles;
     const long long kcap = nk_all / 2 > 0 ? (nk_all / 2 < 16 ? nk_all / 2 : 16) : 1;
     double best = 1e300;
     int best_mt_max = kMaxTokens, best_ks = 1;
+    long long best_whole = -1;  // -1: every tile in best_ks parts (or whole when best_ks == 1)
     for (int tok_max = kMaxTokens; tok_max >= 128; tok_max /= 2) {
         const int mt = (M + tok_max - 1) / tok_max;
         const int per_t = (M + mt - 1) / mt;
@@ -639,6 +661,34 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl) {
                 best = cost;
                 best_mt_max = tok_max;
                 best_ks = (int)k;
+                best_whole = -1;
+            }
+        }
+        if (tiles_t > slots && tiles_t < 2 * slots) {
+            const double step = MTd * 0.76 / 512.0 > 0.7 ? MTd * 0.76 / 512.0 : 0.7;
+            const double whole = (double)nk_all * step;     // one whole tile
+            const double wr = MTd * 512.0 / 1e5;            // one part's partial tile, written
+            for (long long mult = 1; mult <= 2; mult++) {
+                const long long S = (tiles_t - slots) * mult;  // split tiles
+                if (S > tiles_t) break;
+                const long long F = tiles_t - S;               // <= slots
+                const long long idle = slots - F;              // SMs free from the start
+                for (long long k = 2; k <= kcap && k <= 8; k++) {
+                    const double part = (double)nk_all / (double)k * step + wr;
+                    const long long Q = S * k;
+                    const long long early = idle * (long long)(whole / part);  // parts done by then
+                    double span;
+                    if (Q > early) span = whole + (double)((Q - early + slots - 1) / slots) * part;
+                    else span = idle > 0 ? (double)((Q + idle - 1) / idle) * part : whole;
+                    if (span < whole) span = whole;
+                    span += (double)k * wr;                    // the last part sums k partials
+                    if (span < best * 0.98) {
+                        best = span;
+                        best_mt_max = tok_max;
+                        best_ks = (int)k;
+                        best_whole = F;
+                    }
+                }
             }
         }
         if (M <= tok_max / 2) continue;  // smaller token caps change nothing more for small M
@@ -686,9 +736,13 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl) {
     pl->ctas_per_sm = 1;  // 576 threads: one CTA per SM
     const long long tiles = (long long)pl->m_tiles * pl->n_tiles;
     pl->ksplit = best_ks;
-    pl->ws_counters = pl->ksplit > 1 ? round_up_u64(4ull * (uint64_t)tiles, 256) : 0;
-    pl->ws_bytes = pl->ksplit > 1
-                       ? pl->ws_counters + 4ull * (uint64_t)tiles * pl->ksplit * pl->MT * kTileRows
+    // the hybrid was costed for this token tile's tile count; the uniform plans split all
+    // tiles (or none)
+    pl->n_whole = best_whole >= 0 ? (int)best_whole : (best_ks > 1 ? 0 : (int)tiles);
+    const long long n_split = tiles - pl->n_whole;
+    pl->ws_counters = n_split > 0 ? round_up_u64(4ull * (uint64_t)n_split, 256) : 0;
+    pl->ws_bytes = n_split > 0
+                       ? pl->ws_counters + 4ull * (uint64_t)n_split * pl->ksplit * pl->MT * kTileRows
                        : 0;
     pl->ws_xt = round_up_u64(pl->ws_bytes, 256);
     if (rule) pl->ws_bytes = pl->ws_xt + 2ull * (uint64_t)M * round_up_u64(h->K, 8);
@@ -755,6 +809,8 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
     prm.nh = pl.nh;
     prm.n_acc = pl.n_acc;
     prm.ksplit = pl.ksplit;
+    prm.n_whole = pl.n_whole;
+    prm.m_tiles = pl.m_tiles;
     prm.sx = pl.sx;
     prm.sr = pl.sr;
     prm.sw = pl.sw;
@@ -777,8 +833,10 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
                                           (int)pl.smem));
         attr_smem[dev] = pl.smem;
     }
-    if (pl.n_tiles > 65535 || pl.ksplit > 65535) return SPW_ERR_UNSUPPORTED;
-    const dim3 grid(pl.m_tiles, pl.n_tiles, pl.ksplit);
+    const long long tiles = (long long)pl.m_tiles * pl.n_tiles;
+    const long long ctas = pl.n_whole + (tiles - pl.n_whole) * pl.ksplit;
+    if (ctas > 0x7fffffffll) return SPW_ERR_UNSUPPORTED;
+    const dim3 grid((unsigned)ctas);
     spmm_kernel<<<grid, kThreads, pl.smem, stream>>>(tmap, prm);
     SPW_LAUNCH_CHECK();
     return SPW_OK;

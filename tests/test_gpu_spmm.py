@@ -110,3 +110,20 @@ def test_llama7b_prefill_m2048_sampled(name, s):
     ref = oracle.spmm(layer.W, layer.mask, X, rows)
     assert oracle.rel_err(Y[rows], ref) <= TOL
     assert np.isfinite(Y).all()
+
+
+@pytest.mark.parametrize("N,K,M", [(5120, 5120, 2048), (5000, 5120, 2000), (5120, 13824, 2048)])
+def test_hybrid_split_second_wave(N, K, M):
+    # 160 output tiles on 148 SMs: the plan runs the first tiles whole and splits the
+    # last ones along K so they fill the SMs as the whole tiles finish (Llama-13B
+    # attention and down shapes at M = 2048, one ragged variant); rows of every token
+    # tile are sampled, so whole and split tiles are both checked
+    W = workloads.weight(N, K, "hyb")
+    mask = workloads.random_mask(N, K, 0.5, "hyb")
+    X = workloads.normal_act(M, K, "hyb")
+    Y, ws = run(W, mask, X)
+    rows = np.sort(np.concatenate([workloads.rng("hyb-rows", N, M).choice(M, 40, replace=False),
+                                   [0, M - 1]])).astype(np.int32)
+    ref = oracle.spmm(W, mask, X, rows)
+    assert oracle.rel_err(Y[rows], ref) <= TOL
+    assert np.isfinite(Y).all()
