@@ -63,17 +63,26 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def code_sha256(src: bytes) -> str:
+    """sha256 of C/C++ source with comments and whitespace removed (string literals kept),
+    so that editing a comment does not invalidate counters taken on the same code."""
+    import hashlib
+    import re
+    tok = re.compile(rb'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"|\'(?:\\.|[^\'\\])*\'', re.S)
+    kept = tok.sub(lambda m: m.group(0) if m.group(0)[:1] in (b'"', b"'") else b" ", src)
+    return hashlib.sha256(re.sub(rb"\s+", b"", kept)).hexdigest()
+
+
 def measured_traffic():
     """Per-launch DRAM bytes of the decode kernel from the committed ncu summary, or None
-    when the kernel source changed since those counters were taken."""
-    import hashlib
+    when the kernel's code (comments aside) changed since those counters were taken."""
     path = os.path.join(ROOT, "profiles", "spmv_decode_step_traffic.json")
     try:
         rec = json.load(open(path))
         src = open(os.path.join(ROOT, rec["kernel_source"]), "rb").read()
     except (OSError, ValueError, KeyError):
         return None
-    if hashlib.sha256(src).hexdigest() != rec.get("kernel_source_sha256"):
+    if code_sha256(src) != rec.get("kernel_code_sha256"):
         return None
     return int(rec["traffic_bytes_per_launch"])
 

@@ -8,7 +8,7 @@
 // sparse weight matrices", §1, challenge 1), so unstructured tiles are decoded to dense
 // in shared memory and fed to dense MMA; the weight crosses HBM compressed.
 //
-// This library's design for B200 (one output tile per CTA):
+// This library's design for B200 (one output tile, or one K part of one, per CTA):
 //   * Output tile = 128 weight rows (two 64-row TCB strips; the MMA's M) by MT tokens or
 //     batch rows (the MMA's N: MT <= 256 in one MMA, 512 as two), K stepped by 64 (one
 //     TCB k-tile).  The fp32 accumulator, 128 lanes x MT columns, lives in TMEM.  Each
@@ -17,7 +17,11 @@
 //     form 4 independent chains instead of one; the epilogue adds them.
 //   * When output tiles are fewer than the SMs can hold, K is split across CTAs: each
 //     stores its fp32 partial tile; the last CTA of a tile (counted with an atomic) sums
-//     the partials in K order -- deterministic -- and writes fp16.
+//     the partials in K order -- deterministic -- and writes fp16.  When the tiles need
+//     more than one wave but fewer than two, only the last tiles are split, and their
+//     parts fill the SMs as the whole tiles finish.  Each CTA walks its k-steps from a
+//     start rotated by its weight-row tile, so CTAs sharing an X tile read different
+//     parts of it at any moment.
 //   * warp 0, lane 0 (X producer): TMA-loads the X tiles (MT rows x 64, fp16, 128-byte
 //     swizzle, no multicast).  The last warp, lane 0 (TCB producer): 1-D bulk-copies the
 //     two TCB tiles (bitmaps + packed values) of each k-step.  Two warps, not two lanes
@@ -30,8 +34,10 @@
 //     x~ differs from x only in dropping exact zeros, which contribute nothing, and X is
 //     read as given.
 //   * warps 2..17 (decoders, then epilogue): warp d decodes strip d/8, columns
-//     8 (d%8) .. 8 (d%8) + 7, one 16-byte chunk of each of its rows.  Lane l owns rows 2l and 2l+1 at bits q, q+1 (q = 2l mod
-//     32) of one half of each column's bitmap word; the kept rows from 2l+1 upward are the
+//     8 (d%8) .. 8 (d%8) + 7, one 16-byte chunk of each of its rows; it needs only those
+//     8 columns' value starts (one reduction over the columns before them plus a 4-lane
+//     scan).  Lane l owns rows 2l and 2l+1 at bits q, q+1 (q = 2l mod 32) of one half of
+//     each column's bitmap word; the kept rows from 2l+1 upward are the
 //     last c = popc(bits >> (q+1)) values of that half, so row 2l+1's value is at end - 2c
 //     and row 2l's just before it.  Dense rows are written as 16-byte chunks in the
 //     swizzled layout the MMA reads.  After the K loop the same warps read the fp32

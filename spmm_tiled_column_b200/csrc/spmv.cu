@@ -32,7 +32,14 @@
 //   * Split-K combine: a warp writes its fp32 partial for each strip piece into the
 //     workspace; the last contributor of a strip (counted with an atomic) sums all pieces
 //     in a fixed order (even pieces, odd pieces, then the two sums), so results are
-//     deterministic, rounds to fp16 and resets the counter.  A strip with a single contributor is written directly.
+//     deterministic, rounds to fp16 and resets the counter.  A strip with a single
+//     contributor is written directly.  No warp waits for another CTA.
+//   * Tile checks: a tile whose pointers leave the values section or whose bitmaps index
+//     more values than a stage holds is skipped and reported (SPW_ERR_FORMAT).
+//   * FFN mode (spw_spmv_ffn, "Reduced Matrix Multiplication" §4.2): the gate and up
+//     layers form one group; once both layers' rows of a strip are final, the warp that
+//     finished second computes h = SiLU(g) * u for those rows and the strip's column-set
+//     words of h.
 #include <stdlib.h>
 #include <string.h>
 
