@@ -406,6 +406,53 @@ def spw_last_device_status(stream=None) -> int:
     return code.value
 
 
+class DecodeGroup:
+    """A prepared spw_spmv_group call for a fixed set of layers and batch size.
+
+    The header array, weight pointers and workspace are built once; each call only
+    refreshes the input and output pointers and leading dimensions, so the per-call host
+    cost is one library call (serving loops that decode the same layers every step)."""
+
+    def __init__(self, hdrs, bufs, B: int, ws: torch.Tensor | None = None):
+        self.n = len(hdrs)
+        if self.n != len(bufs):
+            raise ValueError("one weight buffer per header")
+        self.B = int(B)
+        self._harr = _hdr_array(hdrs)
+        self._bufs = list(bufs)  # keeps the weights alive
+        P = ctypes.c_void_p * self.n
+        I = ctypes.c_int * self.n
+        self._pbufs = P(*[b.data_ptr() for b in bufs])
+        self._px, self._py, self._pab = P(), P(), P()
+        self._ldx, self._ldy = I(), I()
+        if ws is None:
+            need = spw_spmv_group_workspace_bytes(self._harr, self.B)
+            ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=bufs[0].device)
+        self.ws = ws
+
+    def __call__(self, xs, ys, threshold: float = 0.0, act_bits=None, stream=None):
+        """Decode into ys (one B x N_l fp16 tensor per layer) from xs (B x K_l each)."""
+        if len(xs) != self.n or len(ys) != self.n:
+            raise ValueError(f"expected {self.n} inputs and outputs")
+        for i in range(self.n):
+            x, y = xs[i], ys[i]
+            if x.dtype != torch.float16 or y.dtype != torch.float16:
+                raise TypeError("inputs and outputs must be float16")
+            self._px[i] = x.data_ptr()
+            self._ldx[i] = x.stride(0) if x.dim() == 2 and x.shape[0] > 1 else x.shape[-1]
+            self._py[i] = y.data_ptr()
+            self._ldy[i] = y.stride(0) if y.dim() == 2 and y.shape[0] > 1 else y.shape[-1]
+        ab = None
+        if act_bits is not None:
+            for i in range(self.n):
+                self._pab[i] = None if act_bits[i] is None else act_bits[i].data_ptr()
+            ab = self._pab
+        _check("spw_spmv_group", lib().spw_spmv_group(
+            self.n, self._harr, self._pbufs, self._px, self._ldx, ab, self._py, self._ldy,
+            self.B, float(threshold), _ptr(self.ws), self.ws.numel(), _stream(stream)))
+        return ys
+
+
 class SparseLinear:
     """A compressed weight with its header and per-batch decode workspaces (a holder for
     the calls above; it adds no arithmetic)."""

@@ -68,3 +68,23 @@ def test_group_rejects_bad_sizes():
     x = dev(workloads.normal_act(1, 64, "group-bad"))
     with pytest.raises(spw.SpwError):
         spw.spw_spmv_group([lin.hdr] * 9, [lin.buf] * 9, [x] * 9)
+
+
+def test_prepared_group_matches_group_call():
+    # DecodeGroup only caches the argument arrays: same launch, same bits, and it keeps
+    # working when the input and output tensors change between calls
+    shapes = [(300, 512), (128, 512), (700, 512)]
+    lins = [spw.SparseLinear(dev(workloads.weight(N, K, f"prep{i}")),
+                             dev(workloads.random_mask(N, K, 0.5, f"prep{i}")))
+            for i, (N, K) in enumerate(shapes)]
+    hdrs, bufs = [l.hdr for l in lins], [l.buf for l in lins]
+    g = spw.DecodeGroup(hdrs, bufs, 3)
+    for seed in ("a", "b"):
+        x = dev(workloads.normal_act(3, 512, "prep-x", seed))
+        ys = [torch.empty((3, N), dtype=torch.float16, device="cuda") for N, _ in shapes]
+        g([x] * 3, ys, threshold=0.1)
+        ref = spw.spw_spmv_group(hdrs, bufs, [x] * 3, 0.1)
+        torch.cuda.synchronize()
+        for y, r in zip(ys, ref):
+            np.testing.assert_array_equal(host(y).view(np.uint16), host(r).view(np.uint16))
+    assert spw.spw_last_device_status() == spw.SPW_OK
