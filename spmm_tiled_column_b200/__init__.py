@@ -138,6 +138,26 @@ def _rows(t: torch.Tensor, name: str) -> tuple[torch.Tensor, int]:
     return t, max(t.stride(0), t.shape[1])
 
 
+def _need(t: torch.Tensor, rows: int, cols: int, name: str):
+    """A 2-D view must hold at least rows x cols elements: the library reads or writes
+    that much through its pointer and cannot see the tensor's size."""
+    if t.shape[0] < rows or t.shape[1] < cols:
+        raise ValueError(f"{name} is {tuple(t.shape)}; the call needs at least {rows} x {cols}")
+
+
+def _need_buf(buf: torch.Tensor, h, name: str = "buf"):
+    if not buf.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if buf.numel() * buf.element_size() < h.bytes_total:
+        raise ValueError(f"{name} holds {buf.numel() * buf.element_size()} bytes; the format "
+                         f"header says {h.bytes_total}")
+
+
+def _need_words(a: torch.Tensor | None, n: int, name: str = "act_bits"):
+    if a is not None and a.numel() * a.element_size() < 4 * ((n + 31) // 32):
+        raise ValueError(f"{name} needs at least {(n + 31) // 32} 32-bit words")
+
+
 def _hdr(h) -> spw_format:
     if isinstance(h, spw_format):
         return h
@@ -199,6 +219,8 @@ def spw_decompress(hdr, buf: torch.Tensor, out: torch.Tensor | None = None,
     if out is None:
         out = torch.empty((h.N, h.K), dtype=torch.float16, device=buf.device)
     out2, ld = _rows(_half(out, "out"), "out")
+    _need_buf(buf, h)
+    _need(out2, h.N, h.K, "out")
     _check("spw_decompress", lib().spw_decompress(ctypes.byref(h), _ptr(buf), _ptr(out2), ld,
                                                   _stream(stream)))
     return out
@@ -258,6 +280,10 @@ def spw_spmv(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.0,
     if y is None:
         y = torch.empty((B, h.N), dtype=torch.float16, device=x.device)
     y2, ldy = _rows(_half(y, "y"), "y")
+    _need_buf(buf, h)
+    _need(x2, B, h.K, "x")
+    _need(y2, B, h.N, "y")
+    _need_words(act_bits, h.K)
     if ws is None:
         ws = torch.zeros(max(spw_spmv_workspace_bytes(h, B), 16), dtype=torch.uint8,
                          device=x.device)
@@ -288,6 +314,13 @@ def spw_spmv_group(hdrs, bufs, xs, threshold: float = 0.0, act_bits=None, ys=Non
     if ys is None:
         ys = [torch.empty((B, int(h.N)), dtype=torch.float16, device=xs[0].device) for h in harr]
     y2 = [_rows(_half(y, "y"), "y") for y in ys]
+    if len(bufs) != n or len(x2) != n or len(y2) != n or (act_bits is not None and len(act_bits) != n):
+        raise ValueError(f"expected {n} buffers, inputs and outputs (and column sets)")
+    for i, h in enumerate(harr):
+        _need_buf(bufs[i], h, f"bufs[{i}]")
+        _need(x2[i][0], B, h.K, f"xs[{i}]")
+        _need(y2[i][0], B, h.N, f"ys[{i}]")
+        _need_words(None if act_bits is None else act_bits[i], h.K, f"act_bits[{i}]")
     if ws is None:
         ws = torch.zeros(max(spw_spmv_group_workspace_bytes(hdrs, B), 16), dtype=torch.uint8,
                          device=xs[0].device)
@@ -314,6 +347,10 @@ def spw_spmv_noalloc(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float =
     if y is None:
         y = torch.empty((B, h.N), dtype=torch.float16, device=x.device)
     y2, ldy = _rows(_half(y, "y"), "y")
+    _need_buf(buf, h)
+    _need(x2, x2.shape[0], h.K, "x")
+    _need(y2, x2.shape[0], h.N, "y")
+    _need_words(act_bits, h.K)
     _check("spw_spmv_noalloc", lib().spw_spmv_noalloc(
         ctypes.byref(h), _ptr(buf), _ptr(x2), B, ldx, float(threshold), _ptr(act_bits),
         _ptr(y2), ldy, _stream(stream)))
@@ -334,6 +371,9 @@ def spw_spmm(hdr, buf: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = N
     if Y is None:
         Y = torch.empty((M, h.N), dtype=torch.float16, device=X.device)
     Y2, ldy = _rows(_half(Y, "Y"), "Y")
+    _need_buf(buf, h)
+    _need(X2, M, h.K, "X")
+    _need(Y2, M, h.N, "Y")
     need = spw_spmm_workspace_bytes(h, M)
     if ws is None and need:
         ws = torch.zeros(need, dtype=torch.uint8, device=X.device)
@@ -360,6 +400,10 @@ def spw_spmv_tc(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.0,
     if y is None:
         y = torch.empty((B, h.N), dtype=torch.float16, device=x.device)
     y2, ldy = _rows(_half(y, "y"), "y")
+    _need_buf(buf, h)
+    _need(x2, B, h.K, "x")
+    _need(y2, B, h.N, "y")
+    _need_words(act_bits, h.K)
     need = spw_spmv_tc_workspace_bytes(h, B)
     if ws is None and need:
         ws = torch.zeros(need, dtype=torch.uint8, device=x.device)
@@ -388,8 +432,13 @@ def spw_spmv_ffn(hdr_gate, buf_gate: torch.Tensor, hdr_up, buf_up: torch.Tensor,
     if h is None:
         h = torch.empty((B, hg.N), dtype=torch.float16, device=x.device)
     h2, ldh = _rows(_half(h, "h"), "h")
+    _need_buf(buf_gate, hg, "buf_gate")
+    _need_buf(buf_up, hu, "buf_up")
+    _need(x2, B, hg.K, "x")
+    _need(h2, B, hg.N, "h")
     if act_bits is None:
         act_bits = torch.empty(((hg.N + 31) // 32,), dtype=torch.int32, device=x.device)
+    _need_words(act_bits, hg.N)
     if ws is None:
         need = spw_spmv_ffn_workspace_bytes(hg, hu, B)
         ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=x.device)
@@ -419,6 +468,10 @@ class DecodeGroup:
             raise ValueError("one weight buffer per header")
         self.B = int(B)
         self._harr = _hdr_array(hdrs)
+        for i, h in enumerate(self._harr):
+            _need_buf(bufs[i], h, f"bufs[{i}]")
+        self._K = [int(h.K) for h in self._harr]
+        self._N = [int(h.N) for h in self._harr]
         self._bufs = list(bufs)  # keeps the weights alive
         P = ctypes.c_void_p * self.n
         I = ctypes.c_int * self.n
@@ -438,6 +491,12 @@ class DecodeGroup:
             x, y = xs[i], ys[i]
             if x.dtype != torch.float16 or y.dtype != torch.float16:
                 raise TypeError("inputs and outputs must be float16")
+            if not (x.is_cuda and y.is_cuda):
+                raise ValueError("inputs and outputs must be CUDA tensors")
+            xr = x.shape[0] if x.dim() == 2 else 1
+            yr = y.shape[0] if y.dim() == 2 else 1
+            if xr < self.B or x.shape[-1] < self._K[i] or yr < self.B or y.shape[-1] < self._N[i]:
+                raise ValueError(f"layer {i}: x needs {self.B} x {self._K[i]}, y {self.B} x {self._N[i]}")
             self._px[i] = x.data_ptr()
             self._ldx[i] = x.stride(0) if x.dim() == 2 and x.shape[0] > 1 else x.shape[-1]
             self._py[i] = y.data_ptr()
@@ -445,6 +504,7 @@ class DecodeGroup:
         ab = None
         if act_bits is not None:
             for i in range(self.n):
+                _need_words(act_bits[i], self._K[i], f"act_bits[{i}]")
                 self._pab[i] = None if act_bits[i] is None else act_bits[i].data_ptr()
             ab = self._pab
         _check("spw_spmv_group", lib().spw_spmv_group(

@@ -88,3 +88,26 @@ def test_prepared_group_matches_group_call():
         for y, r in zip(ys, ref):
             np.testing.assert_array_equal(host(y).view(np.uint16), host(r).view(np.uint16))
     assert spw.spw_last_device_status() == spw.SPW_OK
+
+
+def test_bindings_check_tensor_sizes():
+    # the library cannot see tensor sizes, so the bindings compare them with the header
+    # before any launch: short inputs, outputs, weight buffers or column sets are refused
+    (W, mask, lin), = make([(200, 304)], "sizes")
+    x = dev(workloads.normal_act(2, 304, "sizes"))
+    with pytest.raises(ValueError):
+        spw.spw_spmv(lin.hdr, lin.buf, x[:, :296].contiguous())
+    with pytest.raises(ValueError):
+        spw.spw_spmv(lin.hdr, lin.buf, x, y=torch.empty((2, 199), dtype=torch.float16, device="cuda"))
+    with pytest.raises(ValueError):
+        spw.spw_spmv(lin.hdr, lin.buf[:-16], x)
+    with pytest.raises(ValueError):
+        spw.spw_spmv(lin.hdr, lin.buf, x, act_bits=torch.zeros(9, dtype=torch.int32, device="cuda"))
+    with pytest.raises(ValueError):
+        spw.spw_spmm(lin.hdr, lin.buf, x, torch.empty((1, 200), dtype=torch.float16, device="cuda"))
+    g = spw.DecodeGroup([lin.hdr], [lin.buf], 2)
+    with pytest.raises(ValueError):
+        g([x], [torch.empty((1, 200), dtype=torch.float16, device="cuda")])
+    ok = g([x], [torch.empty((2, 200), dtype=torch.float16, device="cuda")])
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(ok[0]), host(lin.spmv(x)))

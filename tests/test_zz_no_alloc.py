@@ -49,7 +49,7 @@ def test_noalloc_matches_spmv_twice(B, a):
 def test_noalloc_rejects_oversized_requests():
     # A header for a 65536 x 4096 weight: its batch-16 workspace exceeds the fixed
     # scratch, so the call must be refused on the host before anything is launched or
-    # read (the small buffers below are never touched).
+    # read (the zero buffers below, sized as the header says, are never touched).
     N, K = 65536, 4096
     h = spw.spw_format()
     h.magic, h.version, h.N, h.K, h.TN, h.TK = 0x31424354, 1, N, K, 64, 64
@@ -62,7 +62,7 @@ def test_noalloc_rejects_oversized_requests():
     h.nnz, h.max_tile_units = 8 * T, 1
     limit = spw.lib().spw_spmv_noalloc_max_scratch_bytes()
     assert spw.spw_spmv_workspace_bytes(h, 16) > limit
-    buf = torch.zeros(1024, dtype=torch.uint8, device="cuda")
+    buf = torch.zeros(h.bytes_total, dtype=torch.uint8, device="cuda")
     x = torch.zeros((16, K), dtype=torch.float16, device="cuda")
     y = torch.zeros((16, N), dtype=torch.float16, device="cuda")
     with pytest.raises(spw.SpwError) as e:
