@@ -254,12 +254,27 @@ int spw_spmv_noalloc(const spw_format* hdr, const void* d_buf, const uint16_t* d
                      int ldx, float threshold, const uint32_t* d_act_bits, uint16_t* d_y, int ldy,
                      void* stream);
 
-/* Workspace bytes spw_spmm needs for M rows of X on the current device: 0 when the output
- * tiles fill the GPU (d_ws may then be NULL); otherwise K is split across CTAs and the
- * workspace holds per-tile arrival counters (its first bytes: zero before the first call,
- * left zero by every call that completes) and fp32 partial tiles.  0 for an invalid
+/* Workspace bytes spw_spmm needs for M rows of X on the current device: 0 when no output
+ * tile is split along K (d_ws may then be NULL); otherwise the workspace holds an arrival
+ * counter per split tile (its first bytes: zero before the first call, left zero by every
+ * call that completes) and fp32 partial tiles.  Tiles are split when the output tiles
+ * would leave SMs idle: all of them when they fill less than a wave, the last ones when
+ * they need more than one wave but fewer than two (see spw_spmm_plan).  0 for an invalid
  * header or M < 1. */
 uint64_t spw_spmm_workspace_bytes(const spw_format* hdr, int M);
+
+/* The launch plan spw_spmm uses for this format and M on a device with sm_count SMs
+ * (sm_count <= 0: the current device).  token_tile tokens (a multiple of 16) per output
+ * tile, token_tiles x weight_tiles output tiles of 128 weight rows; the first
+ * whole_tiles tiles run whole and the others in k_parts parts along K (k_parts = 1: no
+ * split); ctas = whole_tiles + (tiles - whole_tiles) * k_parts; workspace_bytes as
+ * spw_spmm_workspace_bytes.  Host only, no launch.  Errors: INVALID_ARG, FORMAT, CUDA
+ * (no device and sm_count <= 0). */
+typedef struct {
+    int32_t token_tile, token_tiles, weight_tiles, k_parts, whole_tiles, ctas;
+    uint64_t workspace_bytes;
+} spw_spmm_plan_info;
+int spw_spmm_plan(const spw_format* hdr, int M, int sm_count, spw_spmm_plan_info* out);
 
 /* Prefill SpMM ([SPDP] Tensor-Core SpMM; [3LF] §1: tensor cores take only 2:4 sparsity,
  * so unstructured tiles are decoded to dense in shared memory and fed to dense MMA):

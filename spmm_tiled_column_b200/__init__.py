@@ -50,6 +50,13 @@ class spw_format(ctypes.Structure):
 
 
 _FP = ctypes.POINTER(spw_format)
+
+
+class spw_spmm_plan_info(ctypes.Structure):
+    _fields_ = [("token_tile", ctypes.c_int32), ("token_tiles", ctypes.c_int32),
+                ("weight_tiles", ctypes.c_int32), ("k_parts", ctypes.c_int32),
+                ("whole_tiles", ctypes.c_int32), ("ctas", ctypes.c_int32),
+                ("workspace_bytes", ctypes.c_uint64)]
 SIGNATURES = {
     "spw_status_string": ([_I], ctypes.c_char_p),
     "spw_version": ([], _I),
@@ -72,6 +79,7 @@ SIGNATURES = {
     "spw_spmv_noalloc_max_scratch_bytes": ([], _U64),
     "spw_spmv_noalloc": ([_FP, _P, _P, _I, _I, _F, _P, _P, _I, _P], _I),
     "spw_spmv_ffn_workspace_bytes": ([_FP, _FP, _I], _U64),
+    "spw_spmm_plan": ([_FP, _I, _I, ctypes.POINTER(spw_spmm_plan_info)], _I),
     "spw_spmv_ffn": ([_FP, _P, _FP, _P, _P, _I, _I, _F, _P, _I, _P, _P, _U64, _P], _I),
 }
 
@@ -381,6 +389,14 @@ def spw_spmm(hdr, buf: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = N
         ctypes.byref(h), _ptr(buf), _ptr(X2), M, ldx, _ptr(Y2), ldy, _ptr(ws),
         0 if ws is None else ws.numel(), _stream(stream)))
     return Y
+
+
+def spw_spmm_plan(hdr, M: int, sm_count: int = 0) -> dict:
+    """The launch plan of spw_spmm for M tokens on sm_count SMs (0: the current device)."""
+    info = spw_spmm_plan_info()
+    _check("spw_spmm_plan", lib().spw_spmm_plan(ctypes.byref(_hdr(hdr)), int(M), int(sm_count),
+                                                ctypes.byref(info)))
+    return {name: getattr(info, name) for name, _ in info._fields_}
 
 
 def spw_spmv_tc_workspace_bytes(hdr, B: int) -> int:

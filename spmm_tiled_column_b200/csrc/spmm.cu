@@ -635,8 +635,9 @@ struct SpmmPlan {
 };
 
 // Token tile, split-K factor, stage counts and shared-memory layout for M rows of X.
-int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl) {
-    const int sms = device_sm_count();
+// sm_count > 0 plans for that many SMs (spw_spmm_plan); 0 asks the current device.
+int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_count = 0) {
+    const int sms = sm_count > 0 ? sm_count : device_sm_count();
     if (sms <= 0) return SPW_ERR_CUDA;
     // Token tile (512, 256 or 128 tokens, or all M when smaller) and split-K from a small
     // cost model in microseconds: k-steps x max(decode ~0.7, MMA ~0.76 x MT / 512) per CTA,
@@ -854,6 +855,24 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
 using namespace spw;
 
 extern "C" {
+
+int spw_spmm_plan(const spw_format* hdr, int M, int sm_count, spw_spmm_plan_info* out) {
+    if (!out || M < 1) return SPW_ERR_INVALID_ARG;
+    const int rc = check_header(hdr);
+    if (rc != SPW_OK) return rc;
+    SpmmPlan pl;
+    const int prc = make_spmm_plan(hdr, M, false, &pl, sm_count);
+    if (prc != SPW_OK) return prc;
+    const long long tiles = (long long)pl.m_tiles * pl.n_tiles;
+    out->token_tile = pl.MT;
+    out->token_tiles = pl.m_tiles;
+    out->weight_tiles = pl.n_tiles;
+    out->k_parts = pl.ksplit;
+    out->whole_tiles = pl.n_whole;
+    out->ctas = (int32_t)(pl.n_whole + (tiles - pl.n_whole) * pl.ksplit);
+    out->workspace_bytes = pl.ws_bytes;
+    return SPW_OK;
+}
 
 uint64_t spw_spmm_workspace_bytes(const spw_format* hdr, int M) {
     if (check_header(hdr) != SPW_OK || M < 1) return 0;

@@ -113,3 +113,33 @@ def test_host_validation_without_gpu(spw):
     assert L.spw_format_read(good, 10, None, s) == 1
     # device status
     assert L.spw_last_device_status(s, None) == 1
+
+
+def test_tensor_core_decode_and_ffn_host_validation_without_gpu(spw):
+    L = spw.lib()
+    h = valid_header(spw)
+    P = ctypes.c_void_p
+    good, odd, s = P(0x10000), P(0x10008), P(0)
+    ws_n = ctypes.c_uint64(1 << 20)
+    # tensor-core decode: every argument error is found before any device call
+    bad = valid_header(spw)
+    bad.version = 2
+    assert L.spw_spmv_tc(ctypes.byref(bad), good, good, 1, 128, 0.0, None, good, 128, good, ws_n, s) == 4
+    for B in (0, 17):
+        assert L.spw_spmv_tc(ctypes.byref(h), good, good, B, 128, 0.0, None, good, 128, good, ws_n, s) == 1
+    assert L.spw_spmv_tc(ctypes.byref(h), None, good, 1, 128, 0.0, None, good, 128, good, ws_n, s) == 1
+    for t in (-1.0, float("nan"), float("inf")):
+        assert L.spw_spmv_tc(ctypes.byref(h), good, good, 1, 128, t, None, good, 128, good, ws_n, s) == 1
+    assert L.spw_spmv_tc(ctypes.byref(h), good, good, 2, 132, 0.0, None, good, 128, good, ws_n, s) == 1
+    assert L.spw_spmv_tc(ctypes.byref(h), good, good, 1, 128, 0.0, None, good, 127, good, ws_n, s) == 1
+    assert L.spw_spmv_tc(ctypes.byref(h), good, odd, 1, 128, 0.0, None, good, 128, good, ws_n, s) == 2
+    # fused FFN: header, batch and gate/up shape checks come first
+    other = valid_header(spw, N=192)
+    args = (good, good, 1, 128, 0.0, good, 128, good, good, ws_n, s)
+    assert L.spw_spmv_ffn(None, good, ctypes.byref(h), *args) == 1
+    assert L.spw_spmv_ffn(ctypes.byref(h), good, ctypes.byref(bad), *args) == 4
+    assert L.spw_spmv_ffn(ctypes.byref(h), good, ctypes.byref(other), *args) == 1
+    for B in (0, 17):
+        assert L.spw_spmv_ffn(ctypes.byref(h), good, ctypes.byref(h), good, good, B, 128, 0.0,
+                              good, 128, good, good, ws_n, s) == 1
+    assert L.spw_spmv_ffn_workspace_bytes(ctypes.byref(h), ctypes.byref(other), 1) == 0
