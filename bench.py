@@ -87,6 +87,19 @@ def measured_traffic():
     return int(rec["traffic_bytes_per_launch"])
 
 
+def job_rate(ms_local: float, bytes_per_step: int, steps: int, world: int, device) -> tuple:
+    """Whole-job rate of N replicas: the slowest rank's time (a MAX all-reduce over the
+    process group when world > 1) and every rank's bytes.  Returns (ms, GB/s)."""
+    ms = float(ms_local)
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        tt = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    return ms, bytes_per_step * steps * world / (ms * 1e-3) / 1e9
+
+
 def decode_bytes(W, mask, x, t):
     """Algorithmic bytes of one decode call: values + bitmap words of the active columns,
     activations read, outputs written."""
@@ -271,14 +284,7 @@ def run_ours(args, rank, world, local_rank):
         stream.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
-    total_bytes = step_bytes * args.steps * world
-    gbs = total_bytes / (ms * 1e-3) / 1e9
+    ms, gbs = job_rate(e0.elapsed_time(e1), step_bytes, args.steps, world, dev)
     per_rank_gbs = gbs / world
     assert spw.spw_last_device_status() == spw.SPW_OK
 
@@ -496,14 +502,8 @@ def run_ours(args, rank, world, local_rank):
                 e2e_step(i % N_ROTATE)
             b.record(stream)
         stream.synchronize()
-        ems = a.elapsed_time(b)
-        if world > 1:
-            import torch.distributed as dist
-            tt = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
-        ebytes = step_bytes * e2e_steps * world
-        e2e = {"value": round(ebytes / (ems * 1e-3) / 1e9, 2), "unit": "GB/s",
+        ems, egbs = job_rate(a.elapsed_time(b), step_bytes, e2e_steps, world, dev)
+        e2e = {"value": round(egbs, 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(ems / e2e_steps, 4),
                "how": "per step: one pinned H2D of the 4 group inputs, the 4 grouped decodes "
