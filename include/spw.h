@@ -171,7 +171,8 @@ uint64_t spw_spmv_workspace_bytes(const spw_format* hdr, int B);
  *   y_b[n] = sum_k W[n,k] mask[n,k] x~_b[k],  b < B, n < N,
  *   x~_b[k] = x_b[k] if k is in I, x_b[k] != 0 and not |x_b[k]| < threshold, else 0,
  * with I = the columns set in d_act_bits, or every column when d_act_bits is NULL.
- * Columns with no surviving entry in any row are skipped.  fp32 accumulation, one
+ * Columns with no surviving entry in any row cost no decode work (their weight bytes
+ * are still read with the tile's whole-tile copy).  fp32 accumulation, one
  * round-to-nearest-even to fp16 at the end.  x: B x K fp16 (row stride ldx); y: B x N
  * fp16 (row stride ldy).  1 <= B <= 16; threshold finite and >= 0.
  * Workspace: d_ws of at least spw_spmv_workspace_bytes(hdr, B) bytes.  Its first
