@@ -2,6 +2,8 @@
 """Benchmark of the sparse-weight decode / prefill path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --sweep decode|prefill|taxonomy [--quick] [--out FILE]
+    python bench.py --case spmv|spmm|tc|ffn [--layer L] [--batch B] [--act A] [--m M] ...
 
 A step is one decode pass over the seven pruned linear layers of one Llama-7B decoder
 layer (q, k, v, o: 4096 x 4096; gate, up: 11008 x 4096; down: 4096 x 11008), fp16
@@ -16,11 +18,20 @@ the 126 MB L2), so weight bytes come from HBM.
 
 value = algorithmic bytes / time (GB/s): per linear, the values and bitmap words of the
 active columns plus the activations read and the outputs written.  Prefill (spw_spmm at
-M = 2048) and the dense cuBLAS comparisons are extra keys of the same JSON line.
+M = 2048, graph-replayed over rotated operands), the dense cuBLAS comparisons (fp32
+accumulation, no fp16 reduced-precision reductions), the decode time against a plain
+copy of the same bytes (the three-layer-format page's Fig. 5) and the bytes per weight
+of dense / CSR / TCB storage (its Fig. 3) are extra keys of the same JSON line.
 
 --impl reference times the fp64 CPU oracle (this path's reference implementation) on
-the host, on a bounded sample of the same workload.  N > 1 GPUs run replicas (one
-process per GPU via torchrun, no collective on the data path).
+one pinned host core: each step is a bounded sample of the same workload (the decode of
+one of the layer's linears, in turn).  N > 1 GPUs run replicas (one process per GPU via
+torchrun, no collective on the data path).
+
+--sweep times the parity-test configurations that are not bench lines (Llama-7B and
+Llama-13B decode and prefill sweeps, the GEMM-taxonomy shapes), one JSON line per point.
+--case runs one decode or prefill case in a loop, for profilers (ncu -s/-c select
+launches) and quick timing.
 """
 from __future__ import annotations
 
@@ -52,6 +63,52 @@ WORKLOAD = ("Llama-7B decoder-layer decode, batch 1: 7 pruned linears (q,k,v,o 4
             "input, o has its own; down input SiLU(g)*u with the smallest 50% zeroed; one "
             "grouped decode launch per shared input ([q,k,v],[o],[gate,up],[down]) with the "
             "threshold selection fused in")
+
+
+L2_BYTES = 126 * 2**20
+
+
+def run_config(world: int) -> dict:
+    """The workload description, identical on both arms."""
+    return {"workload": WORKLOAD, "global_batch": world, "parallelism": "replicas",
+            "launch_overlap": "programmatic dependent launch between consecutive decode kernels",
+            "l2": f"inputs larger than L2: {N_ROTATE} device copies of the layer's compressed "
+                  "weights rotated (about 7x the 126 MB L2)"}
+
+
+def host_cpu_info() -> dict:
+    model = "unknown"
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
+class pinned_one_core:
+    """Run the block on one host core (the first one this process may use)."""
+
+    def __enter__(self):
+        self.old = None
+        self.core = None
+        try:
+            self.old = os.sched_getaffinity(0)
+            self.core = min(self.old)
+            os.sched_setaffinity(0, {self.core})
+        except (AttributeError, OSError):
+            pass
+        return self.core
+
+    def __exit__(self, *exc):
+        if self.old is not None:
+            try:
+                os.sched_setaffinity(0, self.old)
+            except OSError:
+                pass
+        return False
 
 
 def peaks():
@@ -185,25 +242,61 @@ class Clocks:
 # ------------------------------------------------------------------ CPU oracle arm
 
 def oracle_decode_sample(seconds=12.0, layers=None):
-    """Time the fp64 oracle on whole decode steps of the same workload (one thread)."""
+    """Time the fp64 oracle on whole decode steps of the same workload (one thread,
+    pinned to one host core)."""
     import oracle
     layers = layers if layers is not None else make_layer()
     step_bytes = sum(decode_bytes(W, m, x, t) for _, W, m, x, t in layers)
-    # warm the library once on the smallest linear
-    name, W, m, x, t = layers[0]
-    oracle.spmv(W, m, x, t)
-    done, t0 = 0, time.perf_counter()
-    while True:
-        for _, W, m, x, t in layers:
-            oracle.spmv(W, m, x, t)
-        done += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
+    info = host_cpu_info()
+    with pinned_one_core() as core:
+        # warm the library once on the smallest linear
+        name, W, m, x, t = layers[0]
+        oracle.spmv(W, m, x, t)
+        done, t0 = 0, time.perf_counter()
+        while True:
+            for _, W, m, x, t in layers:
+                oracle.spmv(W, m, x, t)
+            done += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
     return {"value": round(step_bytes * done / el / 1e9, 4), "unit": "GB/s", "cores": 1,
-            "kind": "oracle",
+            "kind": "oracle", **info, "pinned_core": core,
             "sample": f"{done} full decode steps (7 linears, batch 1) in {el:.1f} s, "
-                      "single-threaded fp64 C oracle"}, el / done
+                      f"single-threaded fp64 C oracle on host core {core} of {info['nproc']} "
+                      f"({info['cpu_model']})"}, el / done
+
+
+def reference_arm(args, world):
+    """The oracle as it stands, timed on one pinned host core.  Step i is a bounded sample
+    of the same workload: the oracle decode of linear i mod 7 of the layer (batch 1)."""
+    import oracle
+    layers = make_layer()
+    info = host_cpu_info()
+    with pinned_one_core() as core:
+        for i in range(args.warmup):
+            _, W, m, x, t = layers[i % len(layers)]
+            oracle.spmv(W, m, x, t)
+        total, nbytes = 0.0, 0
+        for i in range(args.steps):
+            _, W, m, x, t = layers[i % len(layers)]
+            t0 = time.perf_counter()
+            oracle.spmv(W, m, x, t)
+            total += time.perf_counter() - t0
+            nbytes += decode_bytes(W, m, x, t)
+    value = nbytes / total / 1e9
+    sample = (f"{args.steps} steps, each the fp64 C oracle's decode of one of the layer's 7 "
+              f"linears in turn (batch 1), after {args.warmup} untimed; one thread on host core "
+              f"{core} of {info['nproc']} ({info['cpu_model']})")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": run_config(world),
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1,
+                             "kind": "oracle", "sample": sample, **info, "pinned_core": core},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -215,6 +308,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     hbm_peak, tc_peak, tc_sust, peak_src = peaks()
+    # the dense cuBLAS bar accumulates in fp32 throughout (no fp16 split-K reductions)
+    torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction = False
 
     def to_dev(a):
         a = np.ascontiguousarray(a)
@@ -510,17 +605,32 @@ def run_ours(args, rank, world, local_rank):
                       "through prepared DecodeGroup calls (Python binding -> C-ABI "
                       "spw_spmv_group), one D2H of the 7 outputs; eager launches on one stream"}
 
-    prefill = None
+    prefill, prefill_detail = None, None
     try:
-        prefill = run_prefill(args, dev, stream, tc_peak, peak_src)
+        prefill, prefill_detail = run_prefill(args, dev, stream, tc_peak, peak_src)
     except Exception as exc:  # the prefill leg must not hide the decode number
         prefill = {"unavailable": f"{type(exc).__name__}: {exc}"[:300]}
+
+    # Decode time against a plain copy of the same bytes (the launch's compressed
+    # weights), per grouped launch: the three-layer-format page's comparison of global
+    # memory access with on-chip decoding (Fig. 5).
+    decode_vs_read = {}
+    for gi, group in enumerate(GROUPS):
+        _, hdrs, _, _, _, _ = gdata[0][gi]
+        nb = sum(int(h.bytes_total) for h in hdrs)
+        cus = copy_us(nb, dev, stream)
+        key = "+".join(group)
+        decode_vs_read[key] = {"weight_bytes": nb, "copy_us": round(cus, 3),
+                               "decode_us": per_group[key]["us"],
+                               "decode_over_copy": round(per_group[key]["us"] / cus, 3)}
+    storage = storage_bytes_per_weight(dev)
 
     avg_launch_us = ms * 1e3 / (args.steps * len(GROUPS))
     achieved = per_rank_gbs
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4), "traffic": measured_traffic(),
-            "traffic_source": "profiles/spmv_decode_step_traffic_llama7b_b1.md (ncu, per launch)",
+            "traffic_source": "profiles/spmv_decode_step_traffic.json (ncu dram bytes per launch; "
+                              "null when the decode kernel's code changed since the capture)",
             "kernel": "spw::spmv_kernel<1>", "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
             "avg_launch_us": round(avg_launch_us, 3),
             "per_group_launch": per_group,
@@ -530,10 +640,7 @@ def run_ours(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "global_batch": world, "parallelism": "replicas",
-                   "launch_overlap": "programmatic dependent launch between consecutive decode kernels",
-                   "l2": f"inputs larger than L2: {N_ROTATE} device copies of the layer rotated "
-                         f"({N_ROTATE * sum(l.buf.numel() for l in base) / 1e9:.2f} GB)"},
+        "config": run_config(world),
         "roofline": roof,
         "gpu_launches": args.steps * len(GROUPS),
         "clocks": clk.summary(),
@@ -542,57 +649,401 @@ def run_ours(args, rank, world, local_rank):
         "ffn_fused": ffn_fused,
         "dense_cublas_step": dense_step,
         "prefill": prefill,
+        "prefill_detail": prefill_detail,
+        "decode_vs_plain_copy": decode_vs_read,
+        "storage_bytes_per_weight": storage,
     }
     return result, layer
 
 
+def graph_us(calls, stream, reps=20, warm=3):
+    """Median microseconds per call: one CUDA graph replays calls[0..R-1] (R rotated
+    operand sets), timed with CUDA events on the launching stream."""
+    import torch
+    R = len(calls)
+    with torch.cuda.stream(stream):
+        for c in calls:
+            c()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for c in calls:
+            c()
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            g.replay()
+    times = []
+    for _ in range(reps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+        stream.synchronize()
+        times.append(a.elapsed_time(b) * 1e3 / R)
+    del g
+    return float(statistics.median(times))
+
+
 def run_prefill(args, dev, stream, tc_peak, peak_src):
+    """spw_spmm at M = 2048 on the q, gate and down shapes against cuBLAS on the dense
+    masked weight, both replayed from CUDA graphs over 3 rotated operand sets (weights,
+    X and Y together exceed L2).  Returns (flat record, per-shape detail)."""
     import torch
     import spmm_tiled_column_b200 as spw
-    M = 2048
-    out = {}
+    M, R = 2048, 3
+    flat, detail = {"M": M}, {}
     for name in ("q", "gate", "down"):
         N, K = workloads.LLAMA7B_LAYERS[name]
         lin = workloads.pruned_layer(name, N, K, SPARSITY, "bench-prefill")
         W = torch.from_numpy(lin.W.view(np.int16)).to(dev).view(torch.float16)
         mask = torch.from_numpy(lin.mask).to(dev)
         sl = spw.SparseLinear(W, mask)
-        X = torch.randn((M, K), device=dev, dtype=torch.float16)
-        Y = torch.empty((M, N), device=dev, dtype=torch.float16)
-        sl.spmm(X, Y)
-        torch.cuda.synchronize()
-        reps = 20
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                sl.spmm(X, Y)
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(reps):
-                sl.spmm(X, Y)
-            b.record(stream)
-        stream.synchronize()
-        us = a.elapsed_time(b) * 1e3 / reps
-        Wd = W * mask.to(torch.float16)
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                torch.nn.functional.linear(X, Wd)
-            a.record(stream)
-            for _ in range(reps):
-                torch.nn.functional.linear(X, Wd)
-            b.record(stream)
-        stream.synchronize()
-        dus = a.elapsed_time(b) * 1e3 / reps
+        bufs = [sl.buf] + [sl.buf.clone() for _ in range(R - 1)]
+        g = torch.Generator(device=dev).manual_seed(2048 + N + K)
+        Xs = [torch.randn((M, K), device=dev, dtype=torch.float16, generator=g) for _ in range(R)]
+        Ys = [torch.empty((M, N), device=dev, dtype=torch.float16) for _ in range(R)]
+        need = spw.spw_spmm_workspace_bytes(sl.hdr, M)
+        wss = [torch.zeros(need, dtype=torch.uint8, device=dev) if need else None for _ in range(R)]
+        us = graph_us([(lambda r=r: spw.spw_spmm(sl.hdr, bufs[r], Xs[r], Ys[r], wss[r]))
+                       for r in range(R)], stream)
+        assert spw.spw_last_device_status() == spw.SPW_OK
+        Wd0 = W * mask.to(torch.float16)
+        Wds = [Wd0] + [Wd0.clone() for _ in range(R - 1)]
+        dus = graph_us([(lambda r=r: torch.matmul(Xs[r], Wds[r].t(), out=Ys[r])) for r in range(R)],
+                       stream)
         flops = 2.0 * M * N * K
-        out[name] = {"M": M, "N": N, "K": K, "us": round(us, 2),
-                     "TFLOP/s_executed": round(flops / (us * 1e-6) / 1e12, 1),
-                     "TFLOP/s_useful": round(2.0 * M * lin.mask.sum() / (us * 1e-6) / 1e12, 1),
-                     "tensor_frac": round(flops / (us * 1e-6) / 1e12 / tc_peak, 4),
-                     "dense_cublas_us": round(dus, 2),
-                     "dense_cublas_TFLOP/s": round(flops / (dus * 1e-6) / 1e12, 1),
-                     "speedup_vs_dense": round(dus / us, 3)}
-    out["peak"] = {"TFLOP/s": tc_peak, "source": f"{peak_src} bf16_tflops (fp16 dense rate equals bf16)"}
+        ex = flops / (us * 1e-6) / 1e12
+        detail[name] = {"M": M, "N": N, "K": K, "us": round(us, 2),
+                        "TFLOP/s_executed": round(ex, 1),
+                        "TFLOP/s_useful": round(2.0 * M * int(lin.mask.sum()) / (us * 1e-6) / 1e12, 1),
+                        "tensor_frac": round(ex / tc_peak, 4), "dense_cublas_us": round(dus, 2),
+                        "dense_cublas_TFLOP/s": round(flops / (dus * 1e-6) / 1e12, 1),
+                        "speedup_vs_dense": round(dus / us, 3)}
+        flat.update({f"{name}_us": round(us, 2), f"{name}_tflops_executed": round(ex, 1),
+                     f"{name}_tensor_frac": round(ex / tc_peak, 4),
+                     f"{name}_cublas_us": round(dus, 2), f"{name}_vs_cublas": round(dus / us, 3)})
+        del bufs, Xs, Ys, Wds, Wd0, sl, wss
+        torch.cuda.empty_cache()
+    detail["peak"] = {"TFLOP/s": tc_peak,
+                      "source": f"{peak_src} bf16_tflops (fp16 dense rate equals bf16)",
+                      "how": "graph replays over 3 rotated operand sets; cuBLAS via torch.matmul "
+                             "with fp16 reduced-precision reductions disabled"}
+    flat["peak_tflops"] = tc_peak
+    return flat, detail
+
+
+def storage_bytes_per_weight(dev):
+    """Bytes per weight slot of a 4096 x 4096 layer stored dense (fp16), as CSR (fp16
+    values, int32 column indices, int32 row pointers), as CSR with 16-bit column indices,
+    and as TCB v1 (bytes_total from spw_format_query), at 40-80 % magnitude pruning: the
+    three-layer-format page's storage comparison (Fig. 3) for this format."""
+    import torch
+    import spmm_tiled_column_b200 as spw
+    N = K = 4096
+    W = workloads.weight(N, K, "storage")
+    out = {}
+    for s in (0.4, 0.5, 0.6, 0.7, 0.8):
+        mask = workloads.magnitude_mask(W, s)
+        nnz = int(np.count_nonzero(mask))
+        nbytes, _ = spw.spw_format_query(torch.from_numpy(mask).to(dev))
+        out[f"{int(s * 100)}%"] = {"dense": 2.0,
+                                   "csr_int32": round((6 * nnz + 4 * (N + 1)) / (N * K), 4),
+                                   "csr_int16": round((4 * nnz + 4 * (N + 1)) / (N * K), 4),
+                                   "tcb_v1": round(nbytes / (N * K), 4)}
     return out
+
+
+def copy_us(nbytes, dev, stream):
+    """Time of a plain device-to-device copy of nbytes (cudaMemcpyAsync through torch:
+    reads nbytes and writes nbytes), over rotated buffers larger than L2."""
+    import torch
+    n = max(16, nbytes)
+    R = max(2, -(-3 * L2_BYTES // (2 * n)))
+    src = [torch.ones(n, dtype=torch.uint8, device=dev) for _ in range(R)]
+    dst = [torch.empty(n, dtype=torch.uint8, device=dev) for _ in range(R)]
+    us = graph_us([(lambda r=r: dst[r].copy_(src[r])) for r in range(R)], stream)
+    del src, dst
+    return us
+
+
+# ------------------------------------------------------------------ sweeps (--sweep)
+
+def _dev(a: np.ndarray):
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float16:
+        return torch.from_numpy(a.view(np.int16)).cuda().view(torch.float16)
+    return torch.from_numpy(a).cuda()
+
+
+def _copies(nbytes: int, cap: int = 24) -> int:
+    return max(2, min(cap, -(-3 * L2_BYTES // max(nbytes, 1))))
+
+
+class _SweepLayer:
+    """One pruned weight on the device: rotated compressed copies for the sparse side and
+    dense masked copies for cuBLAS, each set together larger than 3x the L2."""
+
+    def __init__(self, W: np.ndarray, mask: np.ndarray, dense: bool = True):
+        import torch
+        import spmm_tiled_column_b200 as spw
+        self.W, self.mask = W, mask
+        self.N, self.K = W.shape
+        self.lin = spw.SparseLinear(_dev(W), _dev(mask))
+        R = _copies(self.lin.buf.numel())
+        self.bufs = [self.lin.buf] + [self.lin.buf.clone() for _ in range(R - 1)]
+        self.dense = None
+        if dense:
+            d0 = _dev(np.where(mask.astype(bool), W, np.float16(0)).astype(np.float16))
+            self.dense = [d0] + [d0.clone() for _ in range(_copies(d0.numel() * 2) - 1)]
+        torch.cuda.synchronize()
+
+
+def _sweep_decode_point(layer, x, t, stream, act_bits=None) -> dict:
+    import torch
+    import spmm_tiled_column_b200 as spw
+    B = x.shape[0]
+    xd = _dev(x)
+    ws = [torch.zeros(max(16, spw.spw_spmv_workspace_bytes(layer.lin.hdr, B)), dtype=torch.uint8,
+                      device="cuda") for _ in layer.bufs]
+    ys = [torch.empty((B, layer.N), dtype=torch.float16, device="cuda") for _ in layer.bufs]
+    us = graph_us([(lambda r=r: spw.spw_spmv(layer.lin.hdr, layer.bufs[r], xd, t, act_bits, ys[r],
+                                             ws[r])) for r in range(len(layer.bufs))], stream)
+    assert spw.spw_last_device_status() == spw.SPW_OK
+    out = {"sparse_us": round(us, 3)}
+    if B >= 4:  # the tensor-core decode path as well
+        need = spw.spw_spmv_tc_workspace_bytes(layer.lin.hdr, B)
+        tws = [torch.zeros(max(16, need), dtype=torch.uint8, device="cuda") for _ in layer.bufs]
+        out["tc_us"] = round(graph_us([(lambda r=r: spw.spw_spmv_tc(
+            layer.lin.hdr, layer.bufs[r], xd, t, act_bits, ys[r], tws[r]))
+            for r in range(len(layer.bufs))], stream), 3)
+        assert spw.spw_last_device_status() == spw.SPW_OK
+    if layer.dense is not None:
+        yd = [torch.empty((B, layer.N), dtype=torch.float16, device="cuda") for _ in layer.dense]
+        dus = graph_us([(lambda r=r: torch.matmul(xd, layer.dense[r].t(), out=yd[r]))
+                        for r in range(len(layer.dense))], stream)
+        out.update({"dense_us": round(dus, 3), "speedup": round(dus / us, 3)})
+    return out
+
+
+def _sweep_prefill_point(layer, M, stream) -> dict:
+    import torch
+    import spmm_tiled_column_b200 as spw
+    X = [_dev(workloads.normal_act(M, layer.K, "sweep-prefill", M, layer.K, r)) for r in range(2)]
+    Y = [torch.empty((M, layer.N), dtype=torch.float16, device="cuda") for _ in range(2)]
+    us = graph_us([(lambda r=r: spw.spw_spmm(layer.lin.hdr, layer.bufs[r % len(layer.bufs)], X[r],
+                                             Y[r])) for r in range(2)], stream, reps=10)
+    assert spw.spw_last_device_status() == spw.SPW_OK
+    out = {"sparse_us": round(us, 2)}
+    if layer.dense is not None:
+        dus = graph_us([(lambda r=r: torch.matmul(X[r], layer.dense[r % len(layer.dense)].t(),
+                                                  out=Y[r])) for r in range(2)], stream, reps=10)
+        out.update({"dense_us": round(dus, 2), "speedup": round(dus / us, 3)})
+    return out
+
+
+def _emit(rec: dict, fh):
+    line = json.dumps(rec)
+    print(line, flush=True)
+    if fh:
+        fh.write(line + "\n")
+        fh.flush()
+
+
+def sweep_decode(quick: bool, fh, stream):
+    """Llama-7B linears (q, gate, down) at 50 % and Llama-13B linears at 40-80 % weight
+    sparsity, crossed with activation sparsity (the smallest floor(a K) entries of every
+    batch row zeroed) and batch B in {1, 4, 16}; each point also reports the decode time
+    against a plain copy of the compressed bytes (Fig. 5 of the three-layer-format page)."""
+    import torch
+    hbm = peaks()[0]
+    cases = [("7b", n, workloads.LLAMA7B_LAYERS[n], [0.5], [0.0, 0.3, 0.5, 0.7])
+             for n in ("q", "gate", "down")]
+    s13 = [0.5] if quick else [0.4, 0.5, 0.6, 0.7, 0.8]
+    cases += [("13b", n, sh, s13, [0.0, 0.5, 0.9] if not quick else [0.0, 0.5])
+              for n, sh in workloads.LLAMA13B_SHAPES.items()]
+    batches = [1, 16] if quick else [1, 4, 16]
+    for fam, name, (N, K), sps, acts in cases:
+        W = workloads.weight(N, K, "sweep", fam, name)
+        for s in sps:
+            mask = workloads.magnitude_mask(W, s)
+            layer = _SweepLayer(W, mask)
+            cp_us = copy_us(int(layer.lin.hdr.bytes_total), "cuda", stream)
+            for B in batches:
+                for a in acts:
+                    x, t = workloads.decode_act(name, B, K, a, "sweep", fam, B)
+                    r = _sweep_decode_point(layer, x, 0.0, stream)
+                    byts = decode_bytes(W, mask, x, 0.0)
+                    r.update({"kind": "decode", "family": fam, "layer": name, "N": N, "K": K,
+                              "sparsity": s, "act_sparsity": a, "B": B, "bytes": byts,
+                              "GB/s": round(byts / r["sparse_us"] / 1e3, 1),
+                              "hbm_frac": round(byts / r["sparse_us"] / 1e3 / hbm, 4),
+                              "copy_us": round(cp_us, 3),
+                              "decode_over_copy": round(r["sparse_us"] / cp_us, 3)})
+                    _emit(r, fh)
+            del layer
+            torch.cuda.empty_cache()
+
+
+def sweep_prefill(quick: bool, fh, stream):
+    """The same shapes at 50/60/70 % weight sparsity and M in {512, 2048}."""
+    import torch
+    tc = peaks()[1]
+    shapes = [("7b", n, workloads.LLAMA7B_LAYERS[n]) for n in ("q", "gate", "down")]
+    if not quick:
+        shapes += [("13b", n, sh) for n, sh in workloads.LLAMA13B_SHAPES.items()]
+    for fam, name, (N, K) in shapes:
+        W = workloads.weight(N, K, "sweep", fam, name)
+        for s in ([0.5] if quick else [0.5, 0.6, 0.7]):
+            mask = workloads.magnitude_mask(W, s)
+            layer = _SweepLayer(W, mask)
+            nnz = int(np.count_nonzero(mask))
+            for M in ([2048] if quick else [512, 2048]):
+                r = _sweep_prefill_point(layer, M, stream)
+                ex = 2.0 * M * N * K / r["sparse_us"] / 1e6
+                r.update({"kind": "prefill", "family": fam, "layer": name, "N": N, "K": K,
+                          "sparsity": s, "M": M, "TFLOP/s_executed": round(ex, 1),
+                          "tensor_frac": round(ex / tc, 4),
+                          "TFLOP/s_useful": round(2.0 * M * nnz / r["sparse_us"] / 1e6, 1)})
+                _emit(r, fh)
+            del layer
+            torch.cuda.empty_cache()
+
+
+def sweep_taxonomy(quick: bool, fh, stream):
+    """The GEMM-centric taxonomy shapes of "Beyond FLOPs" on the Llama-7B FFN: width-pruned
+    N (gate/up 11008 -> 8256, 5504; down's K likewise) in decode and prefill, token-reduced
+    M in {2048, 1024, 512}, and the K-reduced down projection keeping 25/50/75 % of its
+    inputs by top-k |activation| ("Reduced Matrix Multiplication" §4.2, §5.1): on the dense
+    side a gather of the kept weight columns (timed separately) plus cuBLAS on the reduced
+    K, on the sparse side top-k selection plus spw_spmv with that column set on the full
+    compressed layer."""
+    import torch
+    import spmm_tiled_column_b200 as spw
+    hbm, tc = peaks()[0], peaks()[1]
+    for w in ([8256] if quick else [8256, 5504]):
+        for name, (N, K) in (("gate", (w, 4096)), ("down", (4096, w))):
+            W = workloads.weight(N, K, "sweep-width", name, w)
+            mask = workloads.magnitude_mask(W, 0.5)
+            layer = _SweepLayer(W, mask)
+            x, _ = workloads.decode_act(name, 1, K, 0.0, "sweep-width", w)
+            r = _sweep_decode_point(layer, x, 0.0, stream)
+            byts = decode_bytes(W, mask, x, 0.0)
+            r.update({"kind": "width_decode", "layer": name, "N": N, "K": K, "sparsity": 0.5,
+                      "B": 1, "bytes": byts, "GB/s": round(byts / r["sparse_us"] / 1e3, 1),
+                      "hbm_frac": round(byts / r["sparse_us"] / 1e3 / hbm, 4)})
+            _emit(r, fh)
+            for M in ([2048] if quick else [2048, 1024, 512]):
+                r = _sweep_prefill_point(layer, M, stream)
+                ex = 2.0 * M * N * K / r["sparse_us"] / 1e6
+                r.update({"kind": "width_prefill", "layer": name, "N": N, "K": K,
+                          "sparsity": 0.5, "M": M, "TFLOP/s_executed": round(ex, 1),
+                          "tensor_frac": round(ex / tc, 4)})
+                _emit(r, fh)
+            del layer
+            torch.cuda.empty_cache()
+    N, K = workloads.LLAMA7B_LAYERS["down"]
+    W = workloads.weight(N, K, "sweep-kred")
+    mask = workloads.magnitude_mask(W, 0.5)
+    layer = _SweepLayer(W, mask)
+    x = workloads.silu_gate_up_act(1, K, "sweep-kred")
+    xd = _dev(x)
+    Wd = layer.dense[0]
+    for keep in ([0.5] if quick else [0.25, 0.5, 0.75]):
+        k = int(round(keep * K))
+        bits = torch.empty((-(-K // 32)) + 3, dtype=torch.int32, device="cuda")
+        idx = torch.empty(k, dtype=torch.int32, device="cuda")
+        spw.spw_select_topk(xd, k, bits, idx)
+        torch.cuda.synchronize()
+        sel_us = graph_us([lambda: spw.spw_select_topk(xd, k, bits, idx)], stream)
+        rec = _sweep_decode_point(layer, x, 0.0, stream, act_bits=bits)
+        il = idx.long()
+        Wg = [Wd.index_select(1, il).contiguous() for _ in range(_copies(N * k * 2))]
+        xg = xd.index_select(1, il).contiguous()
+        gather_us = graph_us([lambda r=r: Wd.index_select(1, il) for r in range(2)], stream)
+        yg = [torch.empty((1, N), dtype=torch.float16, device="cuda") for _ in Wg]
+        gemm_us = graph_us([(lambda r=r: torch.matmul(xg, Wg[r].t(), out=yg[r]))
+                            for r in range(len(Wg))], stream)
+        act = np.zeros(K, dtype=bool)
+        act[idx.cpu().numpy()] = True
+        xk = np.where(act[None, :], x, np.float16(0)).astype(np.float16)
+        byts = decode_bytes(W, mask, xk, 0.0)
+        rec.update({"kind": "k_reduced_down", "N": N, "K": K, "keep": keep, "k": k,
+                    "topk_select_us": round(sel_us, 3), "dense_gather_us": round(gather_us, 3),
+                    "dense_gemm_reduced_K_us": round(gemm_us, 3), "bytes": byts,
+                    "GB/s": round(byts / rec["sparse_us"] / 1e3, 1),
+                    "select_plus_decode_us": round(sel_us + rec["sparse_us"], 3)})
+        rec["speedup_vs_gather_plus_gemm"] = round((gather_us + gemm_us) / rec["sparse_us"], 3)
+        _emit(rec, fh)
+        del Wg
+
+
+def run_sweep(args):
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("the sweeps need a CUDA device")
+    torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction = False
+    fh = open(args.out, "a") if args.out else None
+    stream = torch.cuda.Stream()
+    {"decode": sweep_decode, "prefill": sweep_prefill, "taxonomy": sweep_taxonomy}[args.sweep](
+        args.quick, fh, stream)
+    return 0
+
+
+# ------------------------------------------------------------------ one case (--case)
+
+def run_case(args):
+    """One decode or prefill case of the seeded Llama-7B layers in a loop: --warmup untimed
+    calls, then --reps calls timed with CUDA events on the launching stream (L2-warm: the
+    same operands every call).  Meant for profilers, which select launches with -s / -c."""
+    import torch
+    import spmm_tiled_column_b200 as spw
+    N, K = workloads.LLAMA7B_LAYERS[args.layer]
+    stream = torch.cuda.current_stream()
+    if args.case == "ffn":  # the gate/up pair of one layer, whatever --layer says
+        N, K = workloads.LLAMA7B_LAYERS["gate"]
+        gate = workloads.pruned_layer("gate", N, K, args.sparsity, "profile")
+        up = workloads.pruned_layer("up", N, K, args.sparsity, "profile")
+        lg = spw.SparseLinear(_dev(gate.W), _dev(gate.mask))
+        lu = spw.SparseLinear(_dev(up.W), _dev(up.mask))
+        xd = _dev(workloads.normal_act(args.batch, K, "profile"))
+        h = torch.empty((args.batch, N), dtype=torch.float16, device="cuda")
+        bits = torch.empty(((N + 31) // 32,), dtype=torch.int32, device="cuda")
+        ws = torch.zeros(spw.spw_spmv_ffn_workspace_bytes(lg.hdr, lu.hdr, args.batch),
+                         dtype=torch.uint8, device="cuda")
+        run = lambda: spw.spw_spmv_ffn(lg.hdr, lg.buf, lu.hdr, lu.buf, xd, args.t, h, bits, ws)  # noqa: E731
+    else:
+        layer = workloads.pruned_layer(args.layer, N, K, args.sparsity, "profile")
+        lin = spw.SparseLinear(_dev(layer.W), _dev(layer.mask))
+        if args.case == "spmm":
+            X = _dev(workloads.normal_act(args.m, K, "profile"))
+            Y = torch.empty((args.m, N), dtype=torch.float16, device="cuda")
+            run = lambda: lin.spmm(X, Y)  # noqa: E731
+        else:
+            x, t = workloads.decode_act(args.layer, args.batch, K, args.act, "profile")
+            xd = _dev(x)
+            y = torch.empty((args.batch, N), dtype=torch.float16, device="cuda")
+            thr = t if args.use_threshold else 0.0
+            if args.case == "tc":
+                ws = torch.zeros(max(spw.spw_spmv_tc_workspace_bytes(lin.hdr, args.batch), 16),
+                                 dtype=torch.uint8, device="cuda")
+                run = lambda: spw.spw_spmv_tc(lin.hdr, lin.buf, xd, thr, None, y, ws)  # noqa: E731
+            else:
+                run = lambda: lin.spmv(xd, thr, None, y)  # noqa: E731
+    for _ in range(args.warmup):
+        run()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.reps):
+        run()
+    b.record(stream)
+    torch.cuda.synchronize()
+    assert spw.spw_last_device_status() == spw.SPW_OK
+    print(f"{args.case} {args.layer} {N}x{K} sparsity={args.sparsity} B={args.batch} M={args.m} "
+          f"act={args.act}: {a.elapsed_time(b) * 1e3 / args.reps:.2f} us per call (L2-warm loop)")
+    return 0
 
 
 def main():
@@ -602,7 +1053,24 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", choices=["decode", "prefill", "taxonomy"], default=None)
+    ap.add_argument("--quick", action="store_true", help="--sweep: a few points of each sweep")
+    ap.add_argument("--out", default=None, help="--sweep: also append the JSON lines to this file")
+    ap.add_argument("--case", choices=["spmv", "spmm", "tc", "ffn"], default=None)
+    ap.add_argument("--layer", default="q", choices=sorted(workloads.LLAMA7B_LAYERS))
+    ap.add_argument("--sparsity", type=float, default=0.5)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--act", type=float, default=0.0, help="--case: activation sparsity")
+    ap.add_argument("--use-threshold", action="store_true",
+                    help="--case spmv/tc: pass the activation threshold instead of 0")
+    ap.add_argument("--m", type=int, default=2048, help="--case spmm: tokens")
+    ap.add_argument("--t", type=float, default=0.0, help="--case ffn: threshold on h")
+    ap.add_argument("--reps", type=int, default=10, help="--case: timed calls")
     args = ap.parse_args()
+    if args.sweep:
+        return run_sweep(args)
+    if args.case:
+        return run_case(args)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
 
@@ -613,18 +1081,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        steps = max(1, args.steps)
-        per_step_s = None
-        cpu, per_step_s = oracle_decode_sample(seconds=min(60.0, max(5.0, 0.06 * steps)))
-        line = {"impl": "reference", "metric": METRIC, "value": cpu["value"], "unit": "GB/s",
-                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": round(per_step_s * 1e3, 3), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": WORKLOAD, "parallelism": "host, 1 thread"},
-                "cpu_baseline": cpu,
-                "e2e": {"value": cpu["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
+        print(json.dumps(reference_arm(args, world)), flush=True)
         return 0
 
     if world > 1:

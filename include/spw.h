@@ -115,6 +115,18 @@ int spw_version(void);
  * compressed at load time and left alone).  Returns the previous setting. */
 int spw_set_launch_overlap(int enable);
 
+/* Limit of the product kernels' bounded pipeline waits, in SM clock cycles (process-wide).
+ * The default, about one second (2e9 cycles), is far above any normal wait, which ends
+ * within microseconds; a wait that runs out makes the kernel stop, drain the copies and
+ * tensor-core operations it has in flight, free its tensor memory, report SPW_ERR_TIMEOUT
+ * through spw_last_device_status and return.  A smaller limit exists so that tests can
+ * drive that path on purpose: a few hundred cycles is shorter than a weight copy from
+ * HBM, so the first wait of the next call gives up.  The drain waits keep the default
+ * limit whatever is set here.  cycles = 0 (or above the default) restores the default.
+ * Takes effect at the next launch.  Returns the previous limit in cycles.  No page has a
+ * counterpart; it serves failure detection only. */
+uint64_t spw_set_wait_limit_cycles(uint64_t cycles);
+
 /* Size of the TCB v1 buffer for an N x K mask (device uint8, row stride ld_mask bytes,
  * nonzero = kept).  [SPDP] format; layout above.  Writes bytes_total and nnz (host
  * pointers).  Synchronises `stream`.  Allocates 16 bytes of device scratch (offline).

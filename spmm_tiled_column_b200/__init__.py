@@ -61,6 +61,7 @@ SIGNATURES = {
     "spw_status_string": ([_I], ctypes.c_char_p),
     "spw_version": ([], _I),
     "spw_set_launch_overlap": ([_I], _I),
+    "spw_set_wait_limit_cycles": ([_U64], _U64),
     "spw_format_query": ([_P, _I, _I, _I, _P, _P, _P], _I),
     "spw_compress": ([_P, _I, _P, _I, _I, _I, _P, _U64, _FP, _P], _I),
     "spw_format_read": ([_P, _U64, _FP, _P], _I),
@@ -179,6 +180,13 @@ def spw_set_launch_overlap(enable: bool) -> bool:
     """Enable/disable programmatic launch overlap of consecutive spw_spmv calls (see
     include/spw.h for the one condition it needs); returns the previous setting."""
     return bool(lib().spw_set_launch_overlap(1 if enable else 0))
+
+
+def spw_set_wait_limit_cycles(cycles: int) -> int:
+    """Set the limit of the kernels' bounded pipeline waits in SM cycles (0: the default,
+    about one second); returns the previous limit.  A test hook for the timeout path (see
+    include/spw.h)."""
+    return int(lib().spw_set_wait_limit_cycles(int(cycles)))
 
 
 # ------------------------------------------------------------------ format

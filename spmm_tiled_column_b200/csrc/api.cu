@@ -11,10 +11,10 @@ namespace {
 // Device status word: nonzero after a bounded device wait ran out (SPW_ERR_TIMEOUT).
 __device__ int g_device_status;
 
-constexpr int kMaxDevices = 64;
 std::atomic<int> g_launch_overlap{0};
-int* g_status_ptr[kMaxDevices];
-int g_sm_count[kMaxDevices];
+std::atomic<long long> g_wait_limit{0};  // 0: the default, spw::kWaitLimitCycles
+int* g_status_ptr[spw::kMaxDevices];
+int g_sm_count[spw::kMaxDevices];
 std::mutex g_mutex;
 
 }  // namespace
@@ -47,6 +47,11 @@ int device_sm_count() {
 }
 
 bool launch_overlap() { return g_launch_overlap.load(std::memory_order_relaxed) != 0; }
+
+long long wait_limit_cycles() {
+    const long long v = g_wait_limit.load(std::memory_order_relaxed);
+    return v > 0 ? v : kWaitLimitCycles;
+}
 
 int check_header(const spw_format* h) {
     if (!h) return SPW_ERR_INVALID_ARG;
@@ -86,6 +91,13 @@ int spw_version(void) { return 100; }
 
 int spw_set_launch_overlap(int enable) {
     return g_launch_overlap.exchange(enable ? 1 : 0) != 0;
+}
+
+uint64_t spw_set_wait_limit_cycles(uint64_t cycles) {
+    const long long v = cycles == 0 || cycles > (uint64_t)spw::kWaitLimitCycles
+                            ? 0ll : (long long)cycles;
+    const long long old = g_wait_limit.exchange(v);
+    return (uint64_t)(old > 0 ? old : spw::kWaitLimitCycles);
 }
 
 int spw_format_read(const void* d_buf, uint64_t buf_bytes, spw_format* hdr_out, void* stream) {

@@ -179,7 +179,7 @@ int spw_select_topk(const uint16_t* d_x, int B, int K, int ldx, int k, uint32_t*
     if (!aligned16(d_act_bits) || ((uintptr_t)d_idx & 3u)) return SPW_ERR_ALIGNMENT;
     if (K > kTopkMaxK) return SPW_ERR_UNSUPPORTED;
     const size_t smem = (size_t)K * sizeof(unsigned long long);
-    static bool attr_set[64];
+    static bool attr_set[kMaxDevices];
     int dev = 0;
     SPW_CUDA_TRY(cudaGetDevice(&dev));
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {

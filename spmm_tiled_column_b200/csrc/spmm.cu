@@ -91,6 +91,7 @@ struct SpmmParams {
     uint32_t val_slot;          // bytes per strip's values slot (incl. 16 bytes of slack)
     uint32_t tmem_cols;
     uint32_t off_w, off_raw, off_rec, off_tptr, off_bar;  // dynamic smem offsets
+    long long wait_limit;       // pipeline waits, in SM cycles (drains use the fixed limit)
 };
 
 // ------------------------------------------------------------------ tcgen05 helpers
@@ -160,12 +161,15 @@ __device__ inline void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0,
 }
 
 // Bounded wait that also gives up when another warp has flagged an abort.
-__device__ inline bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
+// A limit shorter than the default polls with the non-blocking test (see mbar_wait).
+__device__ inline bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                     long long limit) {
+    const bool blocking = limit >= kWaitLimitCycles;
+    if (blocking && mbar_try_wait(bar, parity)) return true;
     const long long start = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!(blocking ? mbar_try_wait(bar, parity) : mbar_test_wait(bar, parity))) {
         if (*abort_flag) return false;
-        if (clock64() - start > kWaitLimitCycles) return false;
+        if (clock64() - start > limit) return false;
     }
     return true;
 }
@@ -300,7 +304,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             for (int i = 0; i < n_kc; i++) {
                 const int kt = kstep(i);
                 // X tile: rows m0..m0+MT-1, columns 64 kt.. (zero fill outside X)
-                if (i >= SX && !wait_or_abort(smem_u32(&x_empty[xs]), xph ^ 1u, abort_flag)) {
+                if (i >= SX && !wait_or_abort(smem_u32(&x_empty[xs]), xph ^ 1u, abort_flag, p.wait_limit)) {
                     flag_abort(abort_flag, p.status);
                     break;
                 }
@@ -317,7 +321,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             uint32_t rph = 0;
             for (int i = 0; i < n_kc; i++) {
                 const int kt = kstep(i);
-                if (i >= SR && !wait_or_abort(smem_u32(&r_empty[rs]), rph ^ 1u, abort_flag)) {
+                if (i >= SR && !wait_or_abort(smem_u32(&r_empty[rs]), rph ^ 1u, abort_flag, p.wait_limit)) {
                     flag_abort(abort_flag, p.status);
                     break;
                 }
@@ -358,8 +362,8 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         uint32_t xph = 0, wph = 0;
         bool ok = true;
         for (int i = 0; i < n_kc && ok; i++) {
-            ok = __all_sync(0xffffffffu, wait_or_abort(smem_u32(&x_full[xs]), xph, abort_flag));
-            ok = ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_full[ws]), wph, abort_flag));
+            ok = __all_sync(0xffffffffu, wait_or_abort(smem_u32(&x_full[xs]), xph, abort_flag, p.wait_limit));
+            ok = ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_full[ws]), wph, abort_flag, p.wait_limit));
             if (!ok) {
                 if (lane == 0) flag_abort(abort_flag, p.status);
                 break;
@@ -389,7 +393,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         if (lane == 0) {
             umma_commit(smem_u32(acc_full));
             umma_commit(smem_u32(drain));
-            (void)mbar_wait(smem_u32(drain), 0);  // every issued MMA has completed
+            (void)mbar_drain(smem_u32(drain), 0);  // every issued MMA has completed
         }
         __syncwarp();
     } else {
@@ -408,7 +412,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         uint32_t rph = 0, wph = 0;
         for (int i = 0; i < n_kc; i++) {
             // every lane waits; __all_sync keeps the outcome warp-uniform
-            if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&r_full[rs]), rph, abort_flag))) {
+            if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&r_full[rs]), rph, abort_flag, p.wait_limit))) {
                 flag_abort(abort_flag, p.status);
                 break;
             }
@@ -434,9 +438,19 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 const uint32_t vb = rst_s + 1024u + (uint32_t)q * p.val_slot;
                 const uint32_t a0 = vb + 2u * (uint32_t)(incl - c0 - c1);
                 const uint32_t a1 = a0 + 2u * (uint32_t)c0;
-                // More values than the slot holds means the bitmaps and the tile pointers
-                // disagree: report it and decode the tile as empty rather than read past it.
-                if (2u * __reduce_add_sync(0xffffffffu, (uint32_t)cnt) > p.val_slot - 16u) {
+                // The tile's packed values fill u1 - u0 16-byte units (0 when the producer
+                // rejected the range), so its bitmaps must count between 8 (u1 - u0) - 7
+                // and 8 (u1 - u0) kept weights.  Anything else means the bitmaps and the
+                // tile pointers disagree: report it and decode the tile as empty rather
+                // than read values that belong to no column.
+                const int kt = kstep(i);
+                const uint32_t u0 = tptr[q * (nk + 1) + kt], u1 = tptr[q * (nk + 1) + kt + 1];
+                const uint32_t units = u1 >= u0 && u1 <= p.values_units &&
+                                               (uint64_t)(u1 - u0) * 16u <= p.val_slot - 16u
+                                           ? u1 - u0
+                                           : 0u;
+                const uint32_t total = __reduce_add_sync(0xffffffffu, (uint32_t)cnt);
+                if ((total + 7u) >> 3 != units) {
                     if (lane == 0) raise_status(p.status, SPW_ERR_FORMAT);
                     dec = false;
                 } else if ((lane >> 2) == g) {
@@ -447,7 +461,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             }
             __syncwarp();
             if (i >= SW &&
-                !__all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_empty[ws]), wph ^ 1u, abort_flag))) {
+                !__all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_empty[ws]), wph ^ 1u, abort_flag, p.wait_limit))) {
                 flag_abort(abort_flag, p.status);
                 break;
             }
@@ -482,7 +496,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 
         // ------------------------------------------------------------ epilogue
         const bool acc_ready =
-            __all_sync(0xffffffffu, !*abort_flag && wait_or_abort(smem_u32(acc_full), 0, abort_flag));
+            __all_sync(0xffffffffu, !*abort_flag && wait_or_abort(smem_u32(acc_full), 0, abort_flag, p.wait_limit));
         if (acc_ready) {
             tc_fence_after();
             const int quarter = warp & 3;       // TMEM lanes this warp may access
@@ -588,11 +602,11 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         // at once.
         for (int i = 0; warp == 0 && lane == 0 && i < SX && i < x_issued; i++) {
             const int last = i + ((x_issued - 1 - i) / SX) * SX;
-            (void)mbar_wait(smem_u32(&x_full[i]), (uint32_t)((last / SX) & 1));
+            (void)mbar_drain(smem_u32(&x_full[i]), (uint32_t)((last / SX) & 1));
         }
         for (int i = 0; warp == kTcbWarp && lane == 0 && i < SR && i < r_issued; i++) {
             const int last = i + ((r_issued - 1 - i) / SR) * SR;
-            (void)mbar_wait(smem_u32(&r_full[i]), (uint32_t)((last / SR) & 1));
+            (void)mbar_drain(smem_u32(&r_full[i]), (uint32_t)((last / SR) & 1));
         }
     }
     __syncthreads();
@@ -830,11 +844,12 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
     prm.off_rec = pl.off_rec;
     prm.off_tptr = pl.off_tptr;
     prm.off_bar = pl.off_bar;
+    prm.wait_limit = wait_limit_cycles();
 
-    static size_t attr_smem[64];
+    static size_t attr_smem[kMaxDevices];
     int dev = 0;
     SPW_CUDA_TRY(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= 64) return SPW_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SPW_ERR_CUDA;
     if (attr_smem[dev] < pl.smem) {
         SPW_CUDA_TRY(cudaFuncSetAttribute(spmm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)pl.smem));

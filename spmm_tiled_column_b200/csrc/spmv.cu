@@ -55,12 +55,19 @@ constexpr int kDefaultCtasPerSm = 2;
 constexpr int kMaxStages = 4;
 constexpr int kMinStages = 2;
 constexpr int kCtaHeader = 128;  // CTA-wide words before the consumer regions
-// Per-consumer header: full mbarriers at 0, empty mbarriers at 32, column records at 128
-// (64 x 16 bytes), x~ at 1152 (64 columns x xt_stride(B) halves).
+// Per-consumer header: full mbarriers at 0, empty mbarriers at 32, each stage's tile size
+// (16-byte units, written by the producer) at 64, then the column records and x~.  A
+// record is 8 bytes per half-column: {the half's 32 bitmap bits, the shared-memory
+// address just past that half's packed values}.  The low halves (rows 0-31) sit at
+// kRecLoOff, the high halves at kRecHiOff, both in column-position order, so the 16 bytes
+// at position 2j are the records of columns 2j and 2j+1; the high block is offset by 16
+// bytes so that the two half-warps' 16-byte reads of one pair fall in different banks.
 constexpr int kFullOff = 0;
 constexpr int kEmptyOff = 32;
-constexpr int kRecOff = 128;
-constexpr int kXtOff = 1152;
+constexpr int kUnitsOff = 64;
+constexpr int kRecLoOff = 128;
+constexpr int kRecHiOff = kRecLoOff + 64 * 8 + 16;
+constexpr int kXtOff = kRecHiOff + 64 * 8;  // 64 columns x xt_stride(B) halves
 constexpr int kSmemPerSm = 227 * 1024;
 constexpr uint32_t kStageValsOff = 512;  // stage: 64 bitmap words, then packed values
 
@@ -86,6 +93,7 @@ struct SpmvParams {
     SpmvLayer L[kMaxGroup];
     int n_layers;
     int* status;
+    long long wait_limit;  // pipeline waits, in SM cycles (drains use the fixed limit)
     int n_tiles;      // all layers
     int total_warps;  // working consumer warps
     int stages;
@@ -110,85 +118,99 @@ __host__ __device__ constexpr uint32_t warp_header_bytes(int B) {
     return (uint32_t)((kXtOff + 64 * 2 * xt_stride(B) + 127) / 128 * 128);
 }
 
+// Column pairs decoded per group: the loads of a group are issued before its
+// multiply-adds (x~ of a group is 16 to 64 bytes, read with 16-byte loads).
+__host__ __device__ constexpr int pair_group(int B) { return B <= 2 ? 4 : B <= 4 ? 2 : 1; }
+
 __host__ __device__ inline long long warp_of_tile(long long t, long long total_warps,
                                                   long long n_tiles) {
     return ((t + 1) * total_warps - 1) / n_tiles;
 }
-
-// Columns decoded per group: the loads of a whole group are issued before its
-// multiply-adds, so a warp has 2 * kGroup independent load chains in flight.
-constexpr int kGroup = 4;
 
 // Split a 32-bit word into its two fp16 halves (register halves, no shifts).
 __device__ inline void split_halves(uint32_t w, uint16_t& lo, uint16_t& hi) {
     asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(w));
 }
 
-// acc[b] += a * x[b] for N batch rows when flag != 0: one predicate, N predicated fused
-// multiply-adds (fp16 inputs, fp32 accumulator, one rounding).  A skipped product never
-// touches acc, so a value that belongs to another row (possibly Inf/NaN) cannot leak in.
+// acc[b] += a * x[b] for N batch rows when bits & bit != 0: one lop3 that writes the
+// predicate directly, then N predicated fused multiply-adds (fp16 inputs, fp32
+// accumulator, one rounding).  A skipped product never touches acc, so a value that
+// belongs to another row (possibly Inf/NaN) cannot leak in.
 template <int N>
-__device__ inline void fma_rows_chunk(uint32_t flag, uint16_t a, const uint16_t* x, float* acc);
+__device__ inline void fma_rows_chunk(uint32_t bits, uint32_t bit, uint16_t a, const uint16_t* x,
+                                      float* acc);
 
 template <>
-__device__ inline void fma_rows_chunk<1>(uint32_t flag, uint16_t a, const uint16_t* x, float* acc) {
-    asm("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %1, 0;\n\t"
-        "@p fma.rn.f32.f16 %0, %2, %3, %0;\n\t}"
+__device__ inline void fma_rows_chunk<1>(uint32_t bits, uint32_t bit, uint16_t a, const uint16_t* x,
+                                         float* acc) {
+    asm("{\n\t.reg .pred p, q;\n\t.reg .b32 t;\n\t"
+        "setp.ne.b32 q, 1, 0;\n\t"
+        "lop3.and.b32 t|p, %2, %3, 0, 0xc0, q;\n\t"
+        "@p fma.rn.f32.f16 %0, %4, %1, %0;\n\t}"
         : "+f"(acc[0])
-        : "r"(flag), "h"(a), "h"(x[0]));
+        : "h"(x[0]), "r"(bits), "r"(bit), "h"(a));
 }
 
 template <>
-__device__ inline void fma_rows_chunk<2>(uint32_t flag, uint16_t a, const uint16_t* x, float* acc) {
-    asm("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t"
-        "@p fma.rn.f32.f16 %0, %3, %4, %0;\n\t"
-        "@p fma.rn.f32.f16 %1, %3, %5, %1;\n\t}"
+__device__ inline void fma_rows_chunk<2>(uint32_t bits, uint32_t bit, uint16_t a, const uint16_t* x,
+                                         float* acc) {
+    asm("{\n\t.reg .pred p, q;\n\t.reg .b32 t;\n\t"
+        "setp.ne.b32 q, 1, 0;\n\t"
+        "lop3.and.b32 t|p, %4, %5, 0, 0xc0, q;\n\t"
+        "@p fma.rn.f32.f16 %0, %6, %2, %0;\n\t"
+        "@p fma.rn.f32.f16 %1, %6, %3, %1;\n\t}"
         : "+f"(acc[0]), "+f"(acc[1])
-        : "r"(flag), "h"(a), "h"(x[0]), "h"(x[1]));
+        : "h"(x[0]), "h"(x[1]), "r"(bits), "r"(bit), "h"(a));
 }
 
 template <>
-__device__ inline void fma_rows_chunk<4>(uint32_t flag, uint16_t a, const uint16_t* x, float* acc) {
-    asm("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "@p fma.rn.f32.f16 %0, %5, %6, %0;\n\t"
-        "@p fma.rn.f32.f16 %1, %5, %7, %1;\n\t"
-        "@p fma.rn.f32.f16 %2, %5, %8, %2;\n\t"
-        "@p fma.rn.f32.f16 %3, %5, %9, %3;\n\t}"
+__device__ inline void fma_rows_chunk<4>(uint32_t bits, uint32_t bit, uint16_t a, const uint16_t* x,
+                                         float* acc) {
+    asm("{\n\t.reg .pred p, q;\n\t.reg .b32 t;\n\t"
+        "setp.ne.b32 q, 1, 0;\n\t"
+        "lop3.and.b32 t|p, %8, %9, 0, 0xc0, q;\n\t"
+        "@p fma.rn.f32.f16 %0, %10, %4, %0;\n\t"
+        "@p fma.rn.f32.f16 %1, %10, %5, %1;\n\t"
+        "@p fma.rn.f32.f16 %2, %10, %6, %2;\n\t"
+        "@p fma.rn.f32.f16 %3, %10, %7, %3;\n\t}"
         : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
-        : "r"(flag), "h"(a), "h"(x[0]), "h"(x[1]), "h"(x[2]), "h"(x[3]));
+        : "h"(x[0]), "h"(x[1]), "h"(x[2]), "h"(x[3]), "r"(bits), "r"(bit), "h"(a));
 }
 
 template <>
-__device__ inline void fma_rows_chunk<8>(uint32_t flag, uint16_t a, const uint16_t* x, float* acc) {
-    asm("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %8, 0;\n\t"
-        "@p fma.rn.f32.f16 %0, %9, %10, %0;\n\t"
-        "@p fma.rn.f32.f16 %1, %9, %11, %1;\n\t"
-        "@p fma.rn.f32.f16 %2, %9, %12, %2;\n\t"
-        "@p fma.rn.f32.f16 %3, %9, %13, %3;\n\t"
-        "@p fma.rn.f32.f16 %4, %9, %14, %4;\n\t"
-        "@p fma.rn.f32.f16 %5, %9, %15, %5;\n\t"
-        "@p fma.rn.f32.f16 %6, %9, %16, %6;\n\t"
-        "@p fma.rn.f32.f16 %7, %9, %17, %7;\n\t}"
-        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3]), "+f"(acc[4]), "+f"(acc[5]),
-          "+f"(acc[6]), "+f"(acc[7])
-        : "r"(flag), "h"(a), "h"(x[0]), "h"(x[1]), "h"(x[2]), "h"(x[3]), "h"(x[4]), "h"(x[5]),
-          "h"(x[6]), "h"(x[7]));
+__device__ inline void fma_rows_chunk<8>(uint32_t bits, uint32_t bit, uint16_t a, const uint16_t* x,
+                                         float* acc) {
+    asm("{\n\t.reg .pred p, q;\n\t.reg .b32 t;\n\t"
+        "setp.ne.b32 q, 1, 0;\n\t"
+        "lop3.and.b32 t|p, %16, %17, 0, 0xc0, q;\n\t"
+        "@p fma.rn.f32.f16 %0, %18, %8, %0;\n\t"
+        "@p fma.rn.f32.f16 %1, %18, %9, %1;\n\t"
+        "@p fma.rn.f32.f16 %2, %18, %10, %2;\n\t"
+        "@p fma.rn.f32.f16 %3, %18, %11, %3;\n\t"
+        "@p fma.rn.f32.f16 %4, %18, %12, %4;\n\t"
+        "@p fma.rn.f32.f16 %5, %18, %13, %5;\n\t"
+        "@p fma.rn.f32.f16 %6, %18, %14, %6;\n\t"
+        "@p fma.rn.f32.f16 %7, %18, %15, %7;\n\t}"
+        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3]), "+f"(acc[4]), "+f"(acc[5]), "+f"(acc[6]), "+f"(acc[7])
+        : "h"(x[0]), "h"(x[1]), "h"(x[2]), "h"(x[3]), "h"(x[4]), "h"(x[5]), "h"(x[6]), "h"(x[7]), "r"(bits), "r"(bit), "h"(a));
 }
+
 
 // Any batch width as chunks of 8, 4, 2 and 1 rows.
 template <int B>
-__device__ inline void fma_rows(uint32_t flag, uint16_t a, const uint16_t* x, float* acc) {
+__device__ inline void fma_rows(uint32_t bits, uint32_t bit, uint16_t a, const uint16_t* x,
+                                float* acc) {
     if constexpr (B >= 8) {
-        fma_rows_chunk<8>(flag, a, x, acc);
-        if constexpr (B > 8) fma_rows<B - 8>(flag, a, x + 8, acc + 8);
+        fma_rows_chunk<8>(bits, bit, a, x, acc);
+        if constexpr (B > 8) fma_rows<B - 8>(bits, bit, a, x + 8, acc + 8);
     } else if constexpr (B >= 4) {
-        fma_rows_chunk<4>(flag, a, x, acc);
-        if constexpr (B > 4) fma_rows<B - 4>(flag, a, x + 4, acc + 4);
+        fma_rows_chunk<4>(bits, bit, a, x, acc);
+        if constexpr (B > 4) fma_rows<B - 4>(bits, bit, a, x + 4, acc + 4);
     } else if constexpr (B >= 2) {
-        fma_rows_chunk<2>(flag, a, x, acc);
-        if constexpr (B > 2) fma_rows<B - 2>(flag, a, x + 2, acc + 2);
+        fma_rows_chunk<2>(bits, bit, a, x, acc);
+        if constexpr (B > 2) fma_rows<B - 2>(bits, bit, a, x + 2, acc + 2);
     } else {
-        fma_rows_chunk<1>(flag, a, x, acc);
+        fma_rows_chunk<1>(bits, bit, a, x, acc);
     }
 }
 
@@ -225,32 +247,42 @@ __device__ inline void load_xg(const uint16_t* xt, int j, uint16_t (&xv)[G][B]) 
         for (int b = 0; b < B; b++) xv[c][b] = h[c * XS + b];
 }
 
-// G compacted active columns of one tile, branch-free.  rec2 points at this lane's 8 bytes
-// of each 16-byte column record: {32 bitmap bits of the lane's half, shared-memory address
-// just past that half's packed values}.  Every lane loads its two candidate values whether
-// or not its bits are set (both addresses stay inside the stage), and the predicated
+// 2 PG column positions of one tile, branch-free.  recp points at this lane's half of
+// the records (low or high block): the 16 bytes at position 2j hold columns 2j and 2j+1.
+// Every lane loads its two candidate values whether or not its bits are set (both
+// addresses stay inside the stage: the lowest is 2 bytes below the tile's first value,
+// in the bitmap block, the highest the tile's last value), and the predicated
 // multiply-adds keep only the products of kept rows.
-template <int B, int G>
-__device__ inline void decode_cols(const uint2* rec2, const uint16_t* xt, int j, int sh, int neg2,
-                                   uint32_t bit0, uint32_t bit1, float* acc0, float* acc1) {
-    uint2 r[G];
+template <int B, int PG>
+__device__ inline void decode_pairs(const uint4* recp, const uint16_t* xt, int j, int sh, int neg2,
+                                    uint32_t bit0, uint32_t bit1, float* acc0, float* acc1) {
+    constexpr int G = 2 * PG;
+    uint4 r[PG];
     uint16_t xv[G][B];
 #pragma unroll
-    for (int c = 0; c < G; c++) r[c] = rec2[2 * (j + c)];
+    for (int g = 0; g < PG; g++) r[g] = recp[(j >> 1) + g];
     load_xg<B, G>(xt, j, xv);
+    uint32_t bits[G], end[G];
+#pragma unroll
+    for (int g = 0; g < PG; g++) {
+        bits[2 * g] = r[g].x;
+        end[2 * g] = r[g].y;
+        bits[2 * g + 1] = r[g].z;
+        end[2 * g + 1] = r[g].w;
+    }
     uint16_t v0[G], v1[G];
 #pragma unroll
     for (int c = 0; c < G; c++) {
-        const int above = __popc(r[c].x >> sh);  // kept rows from 2l+1 up in this half
-        uint32_t a;                             // row 2l+1's value: end - 2 * above
-        asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(a) : "r"(above), "r"(neg2), "r"(r[c].y));
+        const int above = __popc(bits[c] >> sh);  // kept rows from 2l+1 up in this half
+        uint32_t a;                               // row 2l+1's value: end - 2 * above
+        asm("mad.lo.s32 %0, %1, %2, %3;" : "=r"(a) : "r"(above), "r"(neg2), "r"(end[c]));
         v1[c] = lds_u16(a);
         v0[c] = lds_u16(a - 2u);
     }
 #pragma unroll
     for (int c = 0; c < G; c++) {
-        fma_rows<B>(r[c].x & bit0, v0[c], xv[c], acc0);
-        fma_rows<B>(r[c].x & bit1, v1[c], xv[c], acc1);
+        fma_rows<B>(bits[c], bit0, v0[c], xv[c], acc0);
+        fma_rows<B>(bits[c], bit1, v1[c], xv[c], acc1);
     }
 }
 
@@ -329,7 +361,7 @@ __device__ void produce(const SpmvParams& p, unsigned char* regions, int W, int 
             nu1 = __ldg(tp + 1);
         }
         const int slot = r % S;
-        if (r >= S && !mbar_wait(reg_s + kEmptyOff + 8 * slot, (uint32_t)((r / S - 1) & 1))) {
+        if (r >= S && !mbar_wait(reg_s + kEmptyOff + 8 * slot, (uint32_t)((r / S - 1) & 1), p.wait_limit)) {
             raise_status(p.status, SPW_ERR_TIMEOUT);
             ok = false;
             continue;
@@ -340,6 +372,9 @@ __device__ void produce(const SpmvParams& p, unsigned char* regions, int W, int 
             raise_status(p.status, SPW_ERR_FORMAT);
             vbytes = 0;
         }
+        // The tile's size for the consumer's bitmap check (published by the arrive below).
+        *(volatile uint32_t*)(regions + (size_t)lane * p.warp_smem + kUnitsOff + 4 * slot) =
+            (uint32_t)(vbytes >> 4);
         const uint32_t bar = reg_s + kFullOff + 8 * slot;
         const uint32_t st = reg_s + HDR + (uint32_t)slot * p.stage_bytes;
         mbar_arrive_expect_tx(bar, 512u + (uint32_t)vbytes);
@@ -351,7 +386,7 @@ __device__ void produce(const SpmvParams& p, unsigned char* regions, int W, int 
         u1 = nu1;
     }
     for (int r = issued > S ? issued - S : 0; r < issued; r++)
-        (void)mbar_wait(reg_s + kFullOff + 8 * (r % S), (uint32_t)((r / S) & 1));
+        (void)mbar_drain(reg_s + kFullOff + 8 * (r % S), (uint32_t)((r / S) & 1));
 }
 
 // Activations of tile columns 2l and 2l+1 for every batch row (one 32-bit load per row
@@ -428,13 +463,16 @@ __device__ void ffn_strip(const SpmvParams& p, int s, int lane) {
 template <int B>
 __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lane) {
     constexpr int XS = xt_stride(B);
+    constexpr int PG = pair_group(B);
     constexpr uint32_t HDR = warp_header_bytes(B);
     const int T = p.n_tiles, PW = p.total_warps, S = p.stages;
     if (gw >= PW) return;  // warps are independent: no block-wide barrier follows
     const int t_begin = (int)((long long)gw * T / PW);
     const int ntiles = (int)((long long)(gw + 1) * T / PW) - t_begin;
     const uint32_t reg_s = smem_u32(reg);
-    uint4* rec = (uint4*)(reg + kRecOff);
+    uint2* rec_lo = (uint2*)(reg + kRecLoOff);
+    uint2* rec_hi = (uint2*)(reg + kRecHiOff);
+    const uint4* recp = (const uint4*)(reg + (lane < 16 ? kRecLoOff : kRecHiOff));
     uint16_t* xt = (uint16_t*)(reg + kXtOff);
     const uint32_t ltmask = lanemask_lt();
     // This lane's rows 2l and 2l+1 sit at bits q and q+1 of the low (lanes 0-15) or high
@@ -442,10 +480,8 @@ __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lan
     const int q = 2 * (lane & 15);
     const int sh = q + 1;
     const uint32_t bit0 = 1u << q, bit1 = 2u << q;
-    const uint2* rec2 = (const uint2*)rec + (lane < 16 ? 0 : 1);  // this half's 8 bytes
     const int neg2 = p.neg2;
-    // Largest value count a stage holds (the slack after it serves the branch-free loads).
-    const int cap = (int)((p.stage_bytes - kStageValsOff - 16u) / 2u);
+    const bool zero_t = p.t == 0.0f;  // the rule is then "v != 0": one test on the bits
 
     // Activations, column sets, outputs and the workspace only after the previous kernel
     // on the stream is complete.
@@ -472,39 +508,43 @@ __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lan
         const SpmvLayer& L = p.L[cur.l];
         const uint32_t st_s = reg_s + HDR + (uint32_t)slot * p.stage_bytes;
         // Warp-uniform outcome: the ballots below need every lane.
-        if (!__all_sync(0xffffffffu, mbar_wait(reg_s + kFullOff + 8 * slot, phase))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(reg_s + kFullOff + 8 * slot, phase, p.wait_limit))) {
             raise_status(p.status, SPW_ERR_TIMEOUT);
             return;  // the producer drains the copies still in flight
         }
 
+        const uint4 bw = *(const uint4*)(reg + HDR + (size_t)slot * p.stage_bytes + 16 * lane);
+        const uint32_t units = *(const volatile uint32_t*)(reg + kUnitsOff + 4 * slot);
+        // Column starts within the tile's values (all 64 columns, in column order).
+        const int cl0 = __popc(bw.x), c0 = cl0 + __popc(bw.y);
+        const int cl1 = __popc(bw.z), c1 = cl1 + __popc(bw.w);
+        const int incl = warp_inclusive_scan(c0 + c1, lane);
+        // The tile's packed values fill `units` 16-byte units, so its bitmaps must count
+        // between 8 units - 7 and 8 units kept weights (the padding is under 8 halves).
+        // Anything else means the bitmaps and the tile pointers disagree: report it and
+        // decode the tile as empty rather than read values that belong to no column.
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        const bool ok = (uint32_t)(total + 7) >> 3 == units;  // warp-uniform
+        if (!ok && lane == 0) raise_status(p.status, SPW_ERR_FORMAT);
+
         // Threshold rule and column set for columns 2l and 2l+1.
         const int col = cur.kt * kTileCols + 2 * lane;
-        const bool in0 = col < L.K && (ac & 1u), in1 = col + 1 < L.K && (ac & 2u);
+        const bool in0 = ok && col < L.K && (ac & 1u), in1 = ok && col + 1 < L.K && (ac & 2u);
         uint16_t xa[B], xb[B];
         bool any0 = false, any1 = false;
 #pragma unroll
         for (int b = 0; b < B; b++) {
             uint16_t lo, hi;
             split_halves(xc[b], lo, hi);
-            const bool p0 = in0 && passes_threshold(lo, p.t);
-            const bool p1 = in1 && passes_threshold(hi, p.t);
+            const bool p0 = in0 && (zero_t ? (lo & 0x7fffu) != 0u : passes_threshold(lo, p.t));
+            const bool p1 = in1 && (zero_t ? (hi & 0x7fffu) != 0u : passes_threshold(hi, p.t));
             xa[b] = p0 ? lo : (uint16_t)0;
             xb[b] = p1 ? hi : (uint16_t)0;
             any0 |= p0;
             any1 |= p1;
         }
-        const uint4 bw = *(const uint4*)(reg + HDR + (size_t)slot * p.stage_bytes + 16 * lane);
-        // Column starts within the tile's values (all 64 columns, in column order).
-        const int cl0 = __popc(bw.x), c0 = cl0 + __popc(bw.y);
-        const int cl1 = __popc(bw.z), c1 = cl1 + __popc(bw.w);
-        const int incl = warp_inclusive_scan(c0 + c1, lane);
-        // A lane's columns index values below incl.  More than a stage holds means the
-        // bitmaps and the tile pointers disagree: report it and skip those columns rather
-        // than read beyond the stage.
-        const bool fits = incl <= cap;
-        if (!fits) raise_status(p.status, SPW_ERR_FORMAT);
-        any0 = fits && any0 && (bw.x | bw.y) != 0u;
-        any1 = fits && any1 && (bw.z | bw.w) != 0u;
+        any0 = any0 && (bw.x | bw.y) != 0u;
+        any1 = any1 && (bw.z | bw.w) != 0u;
         const uint32_t m0 = __ballot_sync(0xffffffffu, any0);
         const uint32_t m1 = __ballot_sync(0xffffffffu, any1);
         const int n_act = __popc(m0) + __popc(m1);
@@ -513,38 +553,60 @@ __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lan
             const uint32_t vb = st_s + kStageValsOff;
             const uint32_t a0 = vb + 2u * (uint32_t)(incl - c0 - c1);
             const uint32_t a1 = a0 + 2u * (uint32_t)c0;
-            // Records at their column positions when every column is active (fully
-            // unrolled decode); otherwise the active columns are compacted, in column
-            // order, and padded with empty records to a group multiple.
-            const bool all = B <= 4 && n_act == 64;  // wider batches keep the loop (registers)
-            const int pos0 = all ? 2 * lane : __popc(m0 & ltmask) + __popc(m1 & ltmask);
-            const int pos1 = pos0 + ((all || any0) ? 1 : 0);
-            if (any0) {
-                rec[pos0] = make_uint4(bw.x, a0 + 2u * (uint32_t)cl0, bw.y, a0 + 2u * (uint32_t)c0);
+            const uint2 lo0 = make_uint2(bw.x, a0 + 2u * (uint32_t)cl0);
+            const uint2 hi0 = make_uint2(bw.y, a0 + 2u * (uint32_t)c0);
+            const uint2 lo1 = make_uint2(bw.z, a1 + 2u * (uint32_t)cl1);
+            const uint2 hi1 = make_uint2(bw.w, a1 + 2u * (uint32_t)c1);
+            if (B <= 4 && n_act == 64) {
+                // Every column active: records in column order (lane l writes the pair
+                // 2l, 2l+1 of each half with one 16-byte store) and a fully unrolled decode.
+                *(uint4*)(rec_lo + 2 * lane) = make_uint4(lo0.x, lo0.y, lo1.x, lo1.y);
+                *(uint4*)(rec_hi + 2 * lane) = make_uint4(hi0.x, hi0.y, hi1.x, hi1.y);
+                if constexpr (B == 1) {
+                    *(uint32_t*)(xt + 2 * lane) = (uint32_t)xa[0] | ((uint32_t)xb[0] << 16);
+                } else {
 #pragma unroll
-                for (int b = 0; b < B; b++) xt[pos0 * XS + b] = xa[b];
-            }
-            if (any1) {
-                rec[pos1] = make_uint4(bw.z, a1 + 2u * (uint32_t)cl1, bw.w, a1 + 2u * (uint32_t)c1);
-#pragma unroll
-                for (int b = 0; b < B; b++) xt[pos1 * XS + b] = xb[b];
-            }
-            if constexpr (B <= 4) {
-                if (all) {
-                    __syncwarp();
-#pragma unroll
-                    for (int j = 0; j < 64; j += kGroup)
-                        decode_cols<B, kGroup>(rec2, xt, j, sh, neg2, bit0, bit1, acc0, acc1);
-                }
-            }
-            if (!all) {
-                const int n_pad = (n_act + kGroup - 1) & ~(kGroup - 1);
-                if (lane < n_pad - n_act) {
-                    rec[n_act + lane] = make_uint4(0u, vb, 0u, vb);
+                    for (int b = 0; b < B; b++) {
+                        xt[(2 * lane) * XS + b] = xa[b];
+                        xt[(2 * lane + 1) * XS + b] = xb[b];
+                    }
                 }
                 __syncwarp();
-                for (int j = 0; j < n_pad; j += kGroup)
-                    decode_cols<B, kGroup>(rec2, xt, j, sh, neg2, bit0, bit1, acc0, acc1);
+                if constexpr (B <= 4) {
+#pragma unroll
+                    for (int j = 0; j < 64; j += 2 * PG)
+                        decode_pairs<B, PG>(recp, xt, j, sh, neg2, bit0, bit1, acc0, acc1);
+                }
+            } else {
+                // Active columns compacted in column order; an odd count is padded with an
+                // empty column (no bits: its multiply-adds never fire).
+                const int pos0 = __popc(m0 & ltmask) + __popc(m1 & ltmask);
+                const int pos1 = pos0 + (any0 ? 1 : 0);
+                if (any0) {
+                    rec_lo[pos0] = lo0;
+                    rec_hi[pos0] = hi0;
+#pragma unroll
+                    for (int b = 0; b < B; b++) xt[pos0 * XS + b] = xa[b];
+                }
+                if (any1) {
+                    rec_lo[pos1] = lo1;
+                    rec_hi[pos1] = hi1;
+#pragma unroll
+                    for (int b = 0; b < B; b++) xt[pos1 * XS + b] = xb[b];
+                }
+                if ((n_act & 1) && lane == 0) {
+                    rec_lo[n_act] = make_uint2(0u, vb);
+                    rec_hi[n_act] = make_uint2(0u, vb);
+                }
+                __syncwarp();
+                const int n_cols = (n_act + 1) & ~1;
+                int j = 0;
+                for (; j + 2 * PG <= n_cols; j += 2 * PG)
+                    decode_pairs<B, PG>(recp, xt, j, sh, neg2, bit0, bit1, acc0, acc1);
+                if constexpr (PG > 1) {
+                    for (; j < n_cols; j += 2)
+                        decode_pairs<B, 1>(recp, xt, j, sh, neg2, bit0, bit1, acc0, acc1);
+                }
             }
         }
         pin_acc<B>(acc0, acc1);
@@ -670,9 +732,9 @@ struct Plan {
     uint64_t ws_bytes;
 };
 
-// Occupancy knobs: consumer warps per CTA and CTAs per SM.  SPW_SPMV_WARPS and
-// SPW_SPMV_CTAS_PER_SM override the defaults (a tuning aid; both change only the launch
-// shape, never the work done).
+// Occupancy knobs: consumer warps per CTA, CTAs per SM and stages per warp.
+// SPW_SPMV_WARPS, SPW_SPMV_CTAS_PER_SM and SPW_SPMV_STAGES override the defaults (a
+// tuning aid; they change only the launch shape, never the work done).
 int env_int(const char* name, int dflt, int lo, int hi) {
     const char* v = getenv(name);
     if (!v || !*v) return dflt;
@@ -710,7 +772,8 @@ int make_plan(int n, const spw_format* h, int B, Plan* pl) {
         if (stages >= kMinStages) break;
     }
     if (stages < kMinStages) return SPW_ERR_UNSUPPORTED;
-    if (stages > kMaxStages) stages = kMaxStages;
+    const int max_stages = env_int("SPW_SPMV_STAGES", kMaxStages, kMinStages, kMaxStages);
+    if (stages > max_stages) stages = max_stages;
     pl->grid = sms * pl->ctas_per_sm;
     pl->total_warps = (long long)pl->grid * pl->warps;
     if (pl->total_warps > T) pl->total_warps = T;  // one tile or more per working warp
@@ -742,10 +805,10 @@ int make_plan(int n, const spw_format* h, int B, Plan* pl) {
 
 template <int B>
 int launch(const Plan& pl, const SpmvParams& prm, cudaStream_t s) {
-    static size_t attr_smem[64];
+    static size_t attr_smem[kMaxDevices];
     int dev = 0;
     SPW_CUDA_TRY(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= 64) return SPW_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SPW_ERR_CUDA;
     if (attr_smem[dev] < pl.smem) {
         SPW_CUDA_TRY(cudaFuncSetAttribute(spmv_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)pl.smem));
@@ -789,16 +852,11 @@ int decode_group_launch(int n, const spw_format* hdrs, const void* const* bufs,
                         const FfnOut* ffn = nullptr) {
     if (n < 1 || n > kMaxGroup || !hdrs || !bufs || !xs || !ldxs || !ys || !ldys)
         return SPW_ERR_INVALID_ARG;
-    if (!d_ws || B < 1 || B > 16) return SPW_ERR_INVALID_ARG;
-    if (!(threshold >= 0.0f) || isinf(threshold)) return SPW_ERR_INVALID_ARG;
+    if (!d_ws) return SPW_ERR_INVALID_ARG;
     for (int l = 0; l < n; l++) {
-        const int rc = check_header(&hdrs[l]);
+        const int rc = check_decode_args(&hdrs[l], bufs[l], xs[l], B, ldxs[l], threshold,
+                                         act_bits ? act_bits[l] : nullptr, ys[l], ldys[l]);
         if (rc != SPW_OK) return rc;
-        if (!bufs[l] || !xs[l] || !ys[l]) return SPW_ERR_INVALID_ARG;
-        if (!ld_ok(ldxs[l], (int)hdrs[l].K, B) || ldys[l] < (int)hdrs[l].N) return SPW_ERR_INVALID_ARG;
-        const uint32_t* ab = act_bits ? act_bits[l] : nullptr;
-        if (!aligned16(bufs[l]) || !aligned16(xs[l]) || !aligned16(ys[l]) || !aligned16(ab))
-            return SPW_ERR_ALIGNMENT;
     }
     if (!aligned16(d_ws)) return SPW_ERR_ALIGNMENT;
     Plan pl;
@@ -842,6 +900,7 @@ int decode_group_launch(int n, const spw_format* hdrs, const void* const* bufs,
     prm.warp_smem = pl.warp_smem;
     prm.t = threshold;
     prm.neg2 = -2;
+    prm.wait_limit = wait_limit_cycles();
     if (ffn) {
         prm.ffn_h = ffn->h;
         prm.ffn_ldh = ffn->ldh;
@@ -888,6 +947,20 @@ int ffn_workspace(const spw_format* hdr_gate, const spw_format* hdr_up, int B, F
 }
 
 }  // namespace
+
+int check_decode_args(const spw_format* hdr, const void* buf, const uint16_t* x, int B, int ldx,
+                      float threshold, const uint32_t* act_bits, const uint16_t* y, int ldy) {
+    const int rc = check_header(hdr);
+    if (rc != SPW_OK) return rc;
+    if (B < 1 || B > 16) return SPW_ERR_INVALID_ARG;
+    if (!(threshold >= 0.0f) || isinf(threshold)) return SPW_ERR_INVALID_ARG;
+    if (!buf || !x || !y) return SPW_ERR_INVALID_ARG;
+    if (!ld_ok(ldx, (int)hdr->K, B) || ldy < (int)hdr->N) return SPW_ERR_INVALID_ARG;
+    if (!aligned16(buf) || !aligned16(x) || !aligned16(y) || !aligned16(act_bits))
+        return SPW_ERR_ALIGNMENT;
+    return SPW_OK;
+}
+
 }  // namespace spw
 
 using namespace spw;

@@ -14,7 +14,7 @@ namespace {
 constexpr uint64_t kNoAllocScratchBytes = 8ull << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-void* g_noalloc_ptr[64];  // device address of the array, per device ordinal
+void* g_noalloc_ptr[spw::kMaxDevices];  // device address of the array, per device ordinal
 std::mutex g_noalloc_mutex;
 
 // Device address of g_noalloc_scratch on the current device.  In host code the array's
@@ -22,7 +22,7 @@ std::mutex g_noalloc_mutex;
 // lookup runs once per device, with that device current.
 void* noalloc_scratch_address() {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= spw::kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
     if (!g_noalloc_ptr[dev]) {
         void* ptr = nullptr;
@@ -41,9 +41,10 @@ uint64_t spw_spmv_noalloc_max_scratch_bytes(void) { return kNoAllocScratchBytes;
 int spw_spmv_noalloc(const spw_format* hdr, const void* d_buf, const uint16_t* d_x, int B,
                      int ldx, float threshold, const uint32_t* d_act_bits, uint16_t* d_y, int ldy,
                      void* stream) {
-    const int rc = spw::check_header(hdr);
+    // Every argument check of spw_spmv first: a bad argument returns before anything is
+    // put on the stream.
+    const int rc = spw::check_decode_args(hdr, d_buf, d_x, B, ldx, threshold, d_act_bits, d_y, ldy);
     if (rc != SPW_OK) return rc;
-    if (B < 1 || B > 16) return SPW_ERR_INVALID_ARG;
     const uint64_t need = spw_spmv_workspace_bytes(hdr, B);
     if (need == 0) return SPW_ERR_UNSUPPORTED;  // no launch plan for this format and batch
     if (need > kNoAllocScratchBytes) return SPW_ERR_UNSUPPORTED;

@@ -49,8 +49,12 @@ __device__ inline void raise_status(int* status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
 
-// Upper bound, in SM clock cycles, on every spin-wait in the library's kernels.
-// About one second at the B200's 1.9 GHz clock; normal waits end within microseconds.
+// Upper bound, in SM clock cycles, on the spin-waits of the library's kernels: about one
+// second at the B200's 1.9 GHz clock; normal waits end within microseconds.  Kernels take
+// the limit of their pipeline waits as a launch parameter (spw_set_wait_limit_cycles can
+// shorten it to exercise the timeout path); the waits that drain copies and MMAs after an
+// abort always use this fixed limit, so that no asynchronous copy can still be writing
+// shared memory when a CTA exits.
 constexpr long long kWaitLimitCycles = 2000000000ll;
 
 // ------------------------------------------------------------------ PTX primitives
@@ -94,15 +98,43 @@ __device__ inline bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return done != 0;
 }
 
-// Wait for the phase with the given parity to complete, giving up after
-// kWaitLimitCycles.  Returns false on timeout (the caller reports it and unwinds).
-__device__ inline bool mbar_wait(uint32_t bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Non-blocking test of the same phase condition.
+__device__ inline bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait for the phase with the given parity to complete, giving up after `limit` cycles.
+// Returns false on timeout (the caller reports it and unwinds).  try_wait may suspend the
+// thread until the phase completes (up to a hardware time window), which is the cheap way
+// to wait but would let a short wait finish whatever the limit; a limit shorter than the
+// default (set only to exercise the timeout path) therefore polls with test_wait.
+__device__ inline bool mbar_wait(uint32_t bar, uint32_t parity, long long limit) {
+    if (limit >= kWaitLimitCycles) {
+        if (mbar_try_wait(bar, parity)) return true;
+        const long long start = clock64();
+        while (!mbar_try_wait(bar, parity)) {
+            if (clock64() - start > limit) return false;
+        }
+        return true;
+    }
     const long long start = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - start > kWaitLimitCycles) return false;
+    while (!mbar_test_wait(bar, parity)) {
+        if (clock64() - start > limit) return false;
     }
     return true;
+}
+
+// Drain wait after an abort (or at exit): always the fixed limit.
+__device__ inline bool mbar_drain(uint32_t bar, uint32_t parity) {
+    return mbar_wait(bar, parity, kWaitLimitCycles);
 }
 
 // One-dimensional bulk copy global -> shared (this CTA), completing on an mbarrier.
@@ -212,6 +244,10 @@ __device__ inline int warp_inclusive_scan(int v, int lane) {
 // ------------------------------------------------------------------ host helpers
 namespace spw {
 
+// Per-device host state (status-word address, SM count, kernel attributes) is kept for
+// device ordinals below this.
+constexpr int kMaxDevices = 64;
+
 inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 // Row stride rule for fp16 operands: multiple of 8 elements unless the operand has a
@@ -230,8 +266,17 @@ int* device_status_ptr();
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 
+// Host-side checks of a decode call's arguments, shared by every decode entry point:
+// header, batch, null pointers, alignment, leading dimensions and threshold.  Returns
+// SPW_OK or the status the call must return; touches no device state.
+int check_decode_args(const spw_format* hdr, const void* buf, const uint16_t* x, int B, int ldx,
+                      float threshold, const uint32_t* act_bits, const uint16_t* y, int ldy);
+
 // Process-wide switch set by spw_set_launch_overlap.
 bool launch_overlap();
+
+// Limit of the kernels' pipeline waits, in SM cycles (spw_set_wait_limit_cycles).
+long long wait_limit_cycles();
 
 }  // namespace spw
 

@@ -53,6 +53,16 @@ def test_status_strings_and_version(spw):
     assert L.spw_status_string(99).decode() == "unknown spw status"
 
 
+def test_wait_limit_setting(spw):
+    # The timeout hook is host state: 0 and values above the default (2e9 cycles) restore
+    # the default; each call returns the previous limit.
+    L = spw.lib()
+    assert L.spw_set_wait_limit_cycles(0) == 2_000_000_000
+    assert L.spw_set_wait_limit_cycles(5000) == 2_000_000_000
+    assert L.spw_set_wait_limit_cycles(3 * 10**9) == 5000
+    assert L.spw_set_wait_limit_cycles(0) == 2_000_000_000
+
+
 def valid_header(spw, N=128, K=128):
     h = spw.spw_format()
     h.magic, h.version, h.N, h.K, h.TN, h.TK = 0x31424354, 1, N, K, 64, 64

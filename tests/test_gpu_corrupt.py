@@ -1,7 +1,8 @@
 """Per-tile buffer checks in the product kernels.
 
 A buffer whose header is valid but whose sections disagree -- a tile whose bitmaps claim
-more kept weights than any tile may hold, or tile pointers outside the values section --
+more kept weights than any tile may hold, a tile whose bitmaps claim a few more kept
+weights than its own values hold, or tile pointers outside the values section --
 must come back as SPW_ERR_FORMAT from spw_last_device_status, with every access kept
 inside the buffer and the stages, and the next call on a consistent buffer (same
 workspace) must be correct again: the split-K counters are left at zero."""
@@ -31,6 +32,18 @@ def corrupted(lin, what):
     if what == "bitmaps":
         # tile 0: all 64 x 64 bits set, far more kept weights than max_tile_units allows
         buf[h.off_bitmaps:h.off_bitmaps + 512] = 0xFF
+    elif what == "overclaim":
+        # tile 0: 16 more bits set than its values hold -- still far fewer than a stage
+        # holds, so only the count against the tile's own size can catch it
+        words = buf[h.off_bitmaps:h.off_bitmaps + 512].view(torch.int64)
+        bits = words.cpu().numpy().view(np.uint64)
+        added = 0
+        for w in range(64):
+            for r in range(64):
+                if added < 16 and not (int(bits[w]) >> r) & 1:
+                    bits[w] = np.uint64(int(bits[w]) | (1 << r))
+                    added += 1
+        buf[h.off_bitmaps:h.off_bitmaps + 512] = torch.from_numpy(bits.view(np.uint8).copy()).cuda()
     else:
         # tile 0's end (= tile 1's start) far past the values section
         T = h.n_strips * h.n_ktiles
@@ -44,7 +57,7 @@ def status():
     return spw.spw_last_device_status()
 
 
-@pytest.mark.parametrize("what", ["bitmaps", "tileptr"])
+@pytest.mark.parametrize("what", ["bitmaps", "overclaim", "tileptr"])
 @pytest.mark.parametrize("B", [1, 8])
 def test_decode_reports_format_and_recovers(what, B):
     W, mask, lin = layer()
@@ -58,7 +71,7 @@ def test_decode_reports_format_and_recovers(what, B):
     assert oracle.rel_err(host(y).astype(np.float64), oracle.spmv(W, mask, x, 0.0, None)) <= TOL
 
 
-@pytest.mark.parametrize("what", ["bitmaps", "tileptr"])
+@pytest.mark.parametrize("what", ["bitmaps", "overclaim", "tileptr"])
 def test_tensor_core_decode_reports_format_and_recovers(what):
     W, mask, lin = layer()
     assert status() == spw.SPW_OK
@@ -72,7 +85,7 @@ def test_tensor_core_decode_reports_format_and_recovers(what):
     assert oracle.rel_err(host(y).astype(np.float64), oracle.spmv(W, mask, x, 0.0, None)) <= TOL
 
 
-@pytest.mark.parametrize("what", ["bitmaps", "tileptr"])
+@pytest.mark.parametrize("what", ["bitmaps", "overclaim", "tileptr"])
 def test_prefill_reports_format_and_recovers(what):
     W, mask, lin = layer()
     assert status() == spw.SPW_OK

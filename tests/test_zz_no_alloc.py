@@ -34,16 +34,48 @@ def test_noalloc_matches_spmv_twice(B, a):
         want = host(lin.spmv(xd)).astype(np.float64)
         y = torch.full((B, N), float("nan"), dtype=torch.float16, device="cuda")
         h = lin.hdr
+        torch.cuda.synchronize()
+        torch_before = torch.cuda.memory_allocated()
+        free_before, _ = torch.cuda.mem_get_info()  # cudaMemGetInfo
         rc = spw.lib().spw_spmv_noalloc(
             ctypes.byref(h), ctypes.c_void_p(lin.buf.data_ptr()), ctypes.c_void_p(xd.data_ptr()),
             B, xd.stride(0), 0.0, None, ctypes.c_void_p(y.data_ptr()), N,
             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
         assert rc == spw.SPW_OK, spw.status_string(rc)
         torch.cuda.synchronize()
+        # The call itself allocates nothing: neither through torch's allocator nor on the
+        # device (the first call's one-time work -- the array's address lookup and loading
+        # the kernels -- is done by then, so the second call is the one to check).
+        assert torch.cuda.memory_allocated() == torch_before
+        if call == 1:
+            assert torch.cuda.mem_get_info()[0] == free_before
         assert spw.spw_last_device_status() == spw.SPW_OK
         got = host(y).astype(np.float64)
         assert oracle.rel_err(got, want) <= TOL
         assert oracle.rel_err(got, oracle.spmv(layer.W, layer.mask, x)) <= TOL
+
+
+def test_noalloc_bad_argument_launches_nothing():
+    # An argument spw_spmv would reject (here a misaligned output pointer) is rejected
+    # before the counter clear is queued: the stream sees no work from the call.
+    N, K = 256, 512
+    layer = workloads.pruned_layer("tiny", N, K, 0.5, "noalloc-bad")
+    lin = spw.SparseLinear(dev(layer.W), dev(layer.mask))
+    x = dev(workloads.normal_act(1, K, "noalloc-bad"))
+    y = torch.zeros((1, N + 8), dtype=torch.float16, device="cuda")
+    s = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    h = lin.hdr
+    rc = spw.lib().spw_spmv_noalloc(
+        ctypes.byref(h), ctypes.c_void_p(lin.buf.data_ptr()), ctypes.c_void_p(x.data_ptr()),
+        1, K, 0.0, None, ctypes.c_void_p(y.data_ptr() + 2), N, ctypes.c_void_p(s.cuda_stream))
+    assert rc == spw.SPW_ERR_ALIGNMENT
+    rc = spw.lib().spw_spmv_noalloc(
+        ctypes.byref(h), ctypes.c_void_p(lin.buf.data_ptr()), ctypes.c_void_p(x.data_ptr()),
+        1, K, -1.0, None, ctypes.c_void_p(y.data_ptr()), N, ctypes.c_void_p(s.cuda_stream))
+    assert rc == spw.SPW_ERR_INVALID_ARG
+    assert s.query()  # nothing was queued
+    assert int(torch.count_nonzero(y)) == 0
 
 
 def test_noalloc_rejects_oversized_requests():
