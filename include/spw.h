@@ -278,13 +278,20 @@ uint64_t spw_spmm_workspace_bytes(const spw_format* hdr, int M);
 
 /* The launch plan spw_spmm uses for this format and M on a device with sm_count SMs
  * (sm_count <= 0: the current device).  token_tile tokens (a multiple of 16) per output
- * tile, token_tiles x weight_tiles output tiles of 128 weight rows; the first
- * whole_tiles tiles run whole and the others in k_parts parts along K (k_parts = 1: no
- * split); ctas = whole_tiles + (tiles - whole_tiles) * k_parts; workspace_bytes as
- * spw_spmm_workspace_bytes.  Host only, no launch.  Errors: INVALID_ARG, FORMAT, CUDA
- * (no device and sm_count <= 0). */
+ * tile, token_tiles x weight_tiles output tiles of 128 weight rows -- or, when cta_pair
+ * is 1, of 256 weight rows each computed by a cluster of two CTAs on an SM pair (one
+ * tcgen05 cta_group::2 MMA: each CTA decodes its 128 rows and loads half the token
+ * tile, so X crosses L2 half as often); the first whole_tiles tiles run whole and the
+ * others in k_parts parts along K (k_parts = 1: no split); ctas = (whole_tiles + (tiles
+ * - whole_tiles) * k_parts) * (cta_pair ? 2 : 1); workspace_bytes as
+ * spw_spmm_workspace_bytes.  Pair mode is used only when the environment sets
+ * SPW_SPMM_PAIR=1, and then for M >= 256 and N > 128 (with sm_count > 0 it assumes
+ * sm_count / 2 SM pairs).  Host only, no launch.
+ * Errors: INVALID_ARG, FORMAT, CUDA (no device and sm_count <= 0). */
 typedef struct {
     int32_t token_tile, token_tiles, weight_tiles, k_parts, whole_tiles, ctas;
+    int32_t cta_pair;  /* 1: each tile is 256 weight rows on an SM pair (two CTAs) */
+    int32_t reserved;  /* 0 */
     uint64_t workspace_bytes;
 } spw_spmm_plan_info;
 int spw_spmm_plan(const spw_format* hdr, int M, int sm_count, spw_spmm_plan_info* out);

@@ -56,6 +56,7 @@ class spw_spmm_plan_info(ctypes.Structure):
     _fields_ = [("token_tile", ctypes.c_int32), ("token_tiles", ctypes.c_int32),
                 ("weight_tiles", ctypes.c_int32), ("k_parts", ctypes.c_int32),
                 ("whole_tiles", ctypes.c_int32), ("ctas", ctypes.c_int32),
+                ("cta_pair", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("workspace_bytes", ctypes.c_uint64)]
 SIGNATURES = {
     "spw_status_string": ([_I], ctypes.c_char_p),

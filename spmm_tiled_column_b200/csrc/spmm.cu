@@ -50,6 +50,7 @@
 // the CUDA-core decode (spmv.cu) skips dropped weights instead.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -59,7 +60,9 @@
 namespace spw {
 namespace {
 
-constexpr int kTileRows = 128;          // weight rows per CTA tile (the MMA's M)
+constexpr int kTileRows = 128;          // weight rows per CTA tile (the MMA's M, or half of it)
+constexpr int kPeerSlots = 8;           // pair mode: the peer's stage-ready ring (on the leader)
+constexpr uint32_t kRecBytesPerWarp = 160;  // a decoder warp's column records (see the decoders)
 constexpr int kTileStrips = kTileRows / kStripRows;
 constexpr int kBK = 64;                 // one TCB k-tile
 constexpr int kMaxTokens = 512;         // tokens per CTA tile (TMEM columns)
@@ -135,6 +138,78 @@ __device__ inline void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 
+// ---- SM-pair (cta_group::2) helpers: a cluster of two CTAs computes one 256-row tile;
+// CTA rank 0 issues the MMAs for both.
+__device__ inline uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ inline uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+// Every thread of both CTAs (no thread may leave early): orders everything before it in
+// either CTA before everything after it in both.
+__device__ inline void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ inline void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Waits with cluster-scope acquire (for arrivals made by the other CTA of the pair).
+__device__ inline bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+__device__ inline bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ inline void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                     uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on the barrier at this offset in both CTAs of the pair once the MMAs issued so
+// far have completed.
+__device__ inline void umma_commit_pair_both(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(bar)
+        : "memory");
+}
+__device__ inline void umma_commit_pair_local(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
 __device__ inline void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -168,6 +243,19 @@ __device__ inline bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int
     if (blocking && mbar_try_wait(bar, parity)) return true;
     const long long start = clock64();
     while (!(blocking ? mbar_try_wait(bar, parity) : mbar_test_wait(bar, parity))) {
+        if (*abort_flag) return false;
+        if (clock64() - start > limit) return false;
+    }
+    return true;
+}
+
+// The same for a barrier the other CTA of a pair arrives on (cluster-scope acquire).
+__device__ inline bool wait_or_abort_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             long long limit) {
+    const bool blocking = limit >= kWaitLimitCycles;
+    if (blocking && mbar_try_wait_cluster(bar, parity)) return true;
+    const long long start = clock64();
+    while (!(blocking ? mbar_try_wait_cluster(bar, parity) : mbar_test_wait_cluster(bar, parity))) {
         if (*abort_flag) return false;
         if (clock64() - start > limit) return false;
     }
@@ -211,6 +299,14 @@ __global__ void __launch_bounds__(256) rule_kernel(const uint16_t* __restrict__ 
     *(uint4*)(xt + (size_t)b * ld + k0) = w;
 }
 
+// PAIR: a cluster of two CTAs on an SM pair computes one 256-weight-row tile.  Each CTA
+// decodes its own 128 rows (the MMA's A, split by rows) and TMA-loads its own half of the
+// token tile (the MMA's B, split by tokens); CTA rank 0 issues tcgen05.mma.cta_group::2
+// for both, whose accumulator halves land in each CTA's own tensor memory.  The other
+// CTA's MMA warp relays "my X and W stages are ready" to rank 0 with a cluster-scope
+// arrive; rank 0's commits release the stages in both CTAs.  Per output element the X
+// tile crosses L2 half as often as with one CTA per 128-row tile.
+template <bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ SpmmParams p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -220,15 +316,17 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // This CTA's output tile and K range: CTA c < n_whole computes tile c whole; the others
     // compute part (c - n_whole) % ksplit of split tile n_whole + (c - n_whole) / ksplit.
-    const int cta = blockIdx.x;
+    const uint32_t rank = PAIR ? cluster_rank() : 0u;  // 0: issues the pair's MMAs
+    const int cta = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // the (pair's) tile slot
     const bool split = cta >= p.n_whole;
     const int tile = split ? p.n_whole + (cta - p.n_whole) / p.ksplit : cta;
     const int parts = split ? p.ksplit : 1;
     const int kz = split ? (cta - p.n_whole) % p.ksplit : 0;
-    const int stile = tile - p.n_whole;  // index among the split tiles (when split)
+    // index of this CTA's 128-row output half among the split ones (when split)
+    const int stile = PAIR ? 2 * (tile - p.n_whole) + (int)rank : tile - p.n_whole;
     const int mt = tile % p.m_tiles, ntile = tile / p.m_tiles;
     const int m0 = mt * p.MT;
-    const int n0 = ntile * kTileRows;
+    const int n0 = ntile * (PAIR ? 2 * kTileRows : kTileRows) + kTileRows * (int)rank;
     const int s0 = n0 / kStripRows;
     const int nk = p.n_ktiles;
     const int k_begin = (int)((long long)kz * nk / parts);
@@ -251,7 +349,8 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     uint64_t* w_empty = w_full + SW;
     uint64_t* acc_full = w_empty + SW;
     uint64_t* drain = acc_full + 1;
-    uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+    uint64_t* peer_ready = drain + 1;  // PAIR, on rank 0: the other CTA's stages are ready
+    uint32_t* tmem_slot = (uint32_t*)(peer_ready + kPeerSlots);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     volatile uint32_t* last_flag = (volatile uint32_t*)(tmem_slot + 2);
     uint32_t* tptr = (uint32_t*)(smem + p.off_tptr);
@@ -271,6 +370,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         }
         mbar_init(smem_u32(acc_full), 1);
         mbar_init(smem_u32(drain), 1);
+        for (int i = 0; i < kPeerSlots; i++) mbar_init(smem_u32(&peer_ready[i]), 1);
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
@@ -281,16 +381,31 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         const int s = s0 + j;
         tptr[i] = (s < p.n_strips) ? __ldg(p.tileptr + (size_t)s * nk + kt) : 0u;
     }
-    if (warp == 1) {  // TMEM allocation (whole warp)
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_u32(tmem_slot)),
-                     "r"(p.tmem_cols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if (warp == 1) {  // TMEM allocation (whole warp; in pair mode warp 1 of both CTAs)
+        if constexpr (PAIR) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(tmem_slot)),
+                         "r"(p.tmem_cols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(tmem_slot)),
+                         "r"(p.tmem_cols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync_all();  // both CTAs' barriers exist before any remote arrive
     tc_fence_after();
+    // Pair mode: an abort in either CTA stops both (the flag is also set in the other CTA).
+    const uint32_t peer_abort = PAIR ? map_to_rank(smem_u32((const void*)abort_flag), rank ^ 1u) : 0u;
+    auto abort_both = [&]() {
+        flag_abort(abort_flag, p.status);
+        if constexpr (PAIR) asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer_abort), "r"(1) : "memory");
+    };
     const uint32_t tmem = *tmem_slot;
 
     int x_issued = 0, r_issued = 0;  // lane 0 of warp 0 (X) and of the TCB warp: stages armed
@@ -298,21 +413,24 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         // ------------------------------------------------------------ producer
         if (warp == 0 && lane == 0) {  // X ring
             asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmap_x) : "memory");
-            const int rows = p.MT / p.nh;  // TMA box height
+            // Per MMA h the token rows m0 + h rows .. +rows; in pair mode this CTA loads
+            // its half of them (the MMA's B is split by tokens across the pair).
+            const int rows = p.MT / p.nh;
+            const int crows = PAIR ? rows / 2 : rows;  // TMA box height
             int xs = 0;
             uint32_t xph = 0;
             for (int i = 0; i < n_kc; i++) {
                 const int kt = kstep(i);
                 // X tile: rows m0..m0+MT-1, columns 64 kt.. (zero fill outside X)
                 if (i >= SX && !wait_or_abort(smem_u32(&x_empty[xs]), xph ^ 1u, abort_flag, p.wait_limit)) {
-                    flag_abort(abort_flag, p.status);
+                    abort_both();
                     break;
                 }
                 const uint32_t xbar = smem_u32(&x_full[xs]);
                 mbar_arrive_expect_tx(xbar, p.x_stage_bytes);
                 for (int h = 0; h < p.nh; h++)
-                    tma_load_2d(sbase + (uint32_t)xs * p.x_stage_bytes + (uint32_t)(h * rows * 128),
-                                &tmap_x, kt * kBK, m0 + h * rows, xbar);
+                    tma_load_2d(sbase + (uint32_t)xs * p.x_stage_bytes + (uint32_t)(h * crows * 128),
+                                &tmap_x, kt * kBK, m0 + h * rows + (int)rank * crows, xbar);
                 x_issued++;
                 if (++xs == SX) { xs = 0; xph ^= 1u; }
             }
@@ -322,7 +440,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             for (int i = 0; i < n_kc; i++) {
                 const int kt = kstep(i);
                 if (i >= SR && !wait_or_abort(smem_u32(&r_empty[rs]), rph ^ 1u, abort_flag, p.wait_limit)) {
-                    flag_abort(abort_flag, p.status);
+                    abort_both();
                     break;
                 }
                 const uint32_t rbar = smem_u32(&r_full[rs]);
@@ -354,18 +472,25 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 if (++rs == SR) { rs = 0; rph ^= 1u; }
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 && (!PAIR || rank == 0)) {
         // ------------------------------------------------------------ MMA issuer
-        const uint32_t idesc = idesc_f16(kTileRows, p.MT / p.nh);
-        const uint32_t half_cols = (uint32_t)(p.MT / p.nh);
+        // (pair mode: rank 0, for both CTAs: M = 256, A and B halves in each CTA)
+        const uint32_t idesc = idesc_f16(PAIR ? 2 * kTileRows : kTileRows, p.MT / p.nh);
+        const uint32_t half_cols = (uint32_t)(p.MT / p.nh);           // the MMA's N per h
+        const uint32_t brows = PAIR ? half_cols / 2 : half_cols;       // this CTA's B rows per h
         int xs = 0, ws = 0;
         uint32_t xph = 0, wph = 0;
         bool ok = true;
         for (int i = 0; i < n_kc && ok; i++) {
             ok = __all_sync(0xffffffffu, wait_or_abort(smem_u32(&x_full[xs]), xph, abort_flag, p.wait_limit));
             ok = ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_full[ws]), wph, abort_flag, p.wait_limit));
+            if constexpr (PAIR)
+                ok = ok && __all_sync(0xffffffffu,
+                                      wait_or_abort_cluster(smem_u32(&peer_ready[i % kPeerSlots]),
+                                                            (uint32_t)((i / kPeerSlots) & 1), abort_flag,
+                                                            p.wait_limit));
             if (!ok) {
-                if (lane == 0) flag_abort(abort_flag, p.status);
+                if (lane == 0) abort_both();
                 break;
             }
             if (lane == 0) {
@@ -379,41 +504,83 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     const uint32_t acc = p.n_acc > 1 ? 32u * (uint32_t)(slice % p.n_acc) : 0u;
                     const uint32_t first = p.n_acc > 1 ? (uint32_t)(slice < p.n_acc) : (uint32_t)(slice == 0);
                     for (int h = 0; h < p.nh; h++) {
-                        const uint64_t bdesc = umma_desc_sw128(xa + half_cols * 128u * h + 32u * j);
-                        umma_f16(tmem + acc + half_cols * h, adesc, bdesc, idesc, first ? 0u : 1u);
+                        const uint64_t bdesc = umma_desc_sw128(xa + brows * 128u * h + 32u * j);
+                        if constexpr (PAIR)
+                            umma_f16_pair(tmem + acc + half_cols * h, adesc, bdesc, idesc, first ? 0u : 1u);
+                        else
+                            umma_f16(tmem + acc + half_cols * h, adesc, bdesc, idesc, first ? 0u : 1u);
                     }
                 }
-                umma_commit(smem_u32(&x_empty[xs]));
-                umma_commit(smem_u32(&w_empty[ws]));
+                if constexpr (PAIR) {
+                    umma_commit_pair_both(smem_u32(&x_empty[xs]));
+                    umma_commit_pair_both(smem_u32(&w_empty[ws]));
+                } else {
+                    umma_commit(smem_u32(&x_empty[xs]));
+                    umma_commit(smem_u32(&w_empty[ws]));
+                }
             }
             __syncwarp();
             if (++xs == SX) { xs = 0; xph ^= 1u; }
             if (++ws == SW) { ws = 0; wph ^= 1u; }
         }
         if (lane == 0) {
-            umma_commit(smem_u32(acc_full));
-            umma_commit(smem_u32(drain));
+            if constexpr (PAIR) {
+                umma_commit_pair_both(smem_u32(acc_full));
+                umma_commit_pair_local(smem_u32(drain));
+            } else {
+                umma_commit(smem_u32(acc_full));
+                umma_commit(smem_u32(drain));
+            }
             (void)mbar_drain(smem_u32(drain), 0);  // every issued MMA has completed
         }
         __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ pair relay (rank 1)
+        // Once this CTA's X stage has landed and its decoders have filled the W stage of a
+        // k-step, tell rank 0 (cluster-scope release); rank 0's commits free both stages.
+        const uint32_t ready0 = map_to_rank(smem_u32(&peer_ready[0]), 0u);
+        int xs = 0, ws = 0;
+        uint32_t xph = 0, wph = 0;
+        for (int i = 0; i < n_kc; i++) {
+            bool ok = __all_sync(0xffffffffu, wait_or_abort(smem_u32(&x_full[xs]), xph, abort_flag, p.wait_limit));
+            ok = ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_full[ws]), wph, abort_flag, p.wait_limit));
+            if (!ok) {
+                if (lane == 0) abort_both();
+                break;
+            }
+            if (lane == 0) mbar_arrive_cluster(ready0 + 8u * (uint32_t)(i % kPeerSlots));
+            __syncwarp();
+            if (++xs == SX) { xs = 0; xph ^= 1u; }
+            if (++ws == SW) { ws = 0; wph ^= 1u; }
+        }
     } else {
         // ------------------------------------------------------------ decoders
         const int d = warp - 2;          // 0..15
         const int q = d >> 3;            // strip within the tile
         const int g = d & 7;             // 8-column group: one 16-byte chunk per row
         const bool strip_ok = s0 + q < p.n_strips;
-        uint4* rec = (uint4*)(smem + p.off_rec + 128u * d);  // 8 columns x 16 bytes
+        // The warp's 8 column records, 8 bytes per half-column {bits, end of the half's
+        // values}: the low halves (rows 0-31) at kRecLo, the high halves at kRecHi, so the
+        // 16 bytes at pair p hold columns 2p and 2p+1; the high block sits 16 bytes off so
+        // that the two half-warps' reads of one pair fall in different banks.
+        constexpr uint32_t kRecLo = 0, kRecHi = 80;
+        unsigned char* rec = smem + p.off_rec + kRecBytesPerWarp * d;
         const int qb = 2 * (lane & 15);  // this lane's rows sit at bits qb, qb+1 of one half
         const int sh = qb + 1;
         const uint32_t bit0 = 1u << qb, bit1 = 2u << qb;
-        const uint2* rec2 = (const uint2*)rec + (lane < 16 ? 0 : 1);
-        const uint32_t nl0 = 64u * q + 2u * lane, nl1 = nl0 + 1u;  // local W rows
+        const uint4* recp = (const uint4*)(rec + (lane < 16 ? kRecLo : kRecHi));
+        const uint32_t nl0 = 64u * q + 2u * lane;  // local W rows nl0, nl0 + 1
+        // Stores of the dense rows: the first store of lanes 4m..4m+3 writes their even row
+        // when m is even and their odd row when m is odd (the second store the other), so
+        // the 8 lanes of each quarter-warp write 8 distinct swizzled chunk positions.
+        const uint32_t swap = ((uint32_t)lane >> 2) & 1u;
+        const uint32_t rowA = nl0 + swap, rowB = nl0 + 1u - swap;
         int rs = 0, ws = 0;
         uint32_t rph = 0, wph = 0;
         for (int i = 0; i < n_kc; i++) {
             // every lane waits; __all_sync keeps the outcome warp-uniform
             if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&r_full[rs]), rph, abort_flag, p.wait_limit))) {
-                flag_abort(abort_flag, p.status);
+                abort_both();
                 break;
             }
             const uint32_t rst_s = sbase + p.off_raw + (uint32_t)rs * p.raw_stage_bytes;
@@ -454,15 +621,16 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     if (lane == 0) raise_status(p.status, SPW_ERR_FORMAT);
                     dec = false;
                 } else if ((lane >> 2) == g) {
-                    const int j = 2 * (lane & 3);
-                    rec[j] = make_uint4(bw.x, a0 + 2u * (uint32_t)cl0, bw.y, a1);
-                    rec[j + 1] = make_uint4(bw.z, a1 + 2u * (uint32_t)cl1, bw.w, a1 + 2u * (uint32_t)c1);
+                    const uint32_t pp = 16u * (uint32_t)(lane & 3);  // pair: columns 2(l&3), +1
+                    *(uint4*)(rec + kRecLo + pp) =
+                        make_uint4(bw.x, a0 + 2u * (uint32_t)cl0, bw.z, a1 + 2u * (uint32_t)cl1);
+                    *(uint4*)(rec + kRecHi + pp) = make_uint4(bw.y, a1, bw.w, a1 + 2u * (uint32_t)c1);
                 }
             }
             __syncwarp();
             if (i >= SW &&
                 !__all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_empty[ws]), wph ^ 1u, abort_flag, p.wait_limit))) {
-                flag_abort(abort_flag, p.status);
+                abort_both();
                 break;
             }
             unsigned char* wst = smem + p.off_w + (uint32_t)ws * kWStageBytes;
@@ -470,19 +638,25 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 uint32_t o0[4] = {0u, 0u, 0u, 0u}, o1[4] = {0u, 0u, 0u, 0u};
                 if (dec) {
 #pragma unroll
-                    for (int c = 0; c < 8; c++) {
-                        const uint2 r = rec2[2 * c];
-                        uint32_t a;
-                        asm("mad.lo.s32 %0, %1, -2, %2;" : "=r"(a) : "r"(__popc(r.x >> sh)), "r"(r.y));
-                        const uint32_t v1 = lds_u16(a), v0 = lds_u16(a - 2u);
-                        const uint32_t sft = 16u * (uint32_t)(c & 1);
-                        o0[c >> 1] |= ((r.x & bit0) ? v0 : 0u) << sft;
-                        o1[c >> 1] |= ((r.x & bit1) ? v1 : 0u) << sft;
+                    for (int pr = 0; pr < 4; pr++) {
+                        const uint4 r = recp[pr];
+                        const uint32_t bits[2] = {r.x, r.z}, end[2] = {r.y, r.w};
+#pragma unroll
+                        for (int e = 0; e < 2; e++) {
+                            uint32_t a;
+                            asm("mad.lo.s32 %0, %1, -2, %2;" : "=r"(a) : "r"(__popc(bits[e] >> sh)), "r"(end[e]));
+                            const uint32_t v1 = lds_u16(a), v0 = lds_u16(a - 2u);
+                            const uint32_t sft = 16u * (uint32_t)e;
+                            o0[pr] |= ((bits[e] & bit0) ? v0 : 0u) << sft;
+                            o1[pr] |= ((bits[e] & bit1) ? v1 : 0u) << sft;
+                        }
                     }
                 }
+                const uint4 wA = swap ? make_uint4(o1[0], o1[1], o1[2], o1[3]) : make_uint4(o0[0], o0[1], o0[2], o0[3]);
+                const uint4 wB = swap ? make_uint4(o0[0], o0[1], o0[2], o0[3]) : make_uint4(o1[0], o1[1], o1[2], o1[3]);
                 const uint32_t chunk = (uint32_t)g;
-                *(uint4*)(wst + nl0 * 128u + ((chunk ^ (nl0 & 7u)) << 4)) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-                *(uint4*)(wst + nl1 * 128u + ((chunk ^ (nl1 & 7u)) << 4)) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+                *(uint4*)(wst + rowA * 128u + ((chunk ^ (rowA & 7u)) << 4)) = wA;
+                *(uint4*)(wst + rowB * 128u + ((chunk ^ (rowB & 7u)) << 4)) = wB;
             }
             fence_proxy_async_smem();  // generic-proxy stores -> tensor-core reads
             __syncwarp();
@@ -534,13 +708,18 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             }
             if (split) __threadfence();  // partials before the arrival below
         } else {
-            flag_abort(abort_flag, p.status);
+            abort_both();
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (split && !*abort_flag) {
+    // One decision for the whole CTA: in pair mode the other CTA may raise the flag at
+    // any moment, and every thread must take the same side of the barriers below.
+    volatile int* aborted = (volatile int*)(tmem_slot + 3);
+    if (threadIdx.x == 0) *aborted = *abort_flag;
+    __syncthreads();
+    if (split && !*aborted) {
         // Split-K: the last CTA of this output tile sums every partial in K order.
         if (threadIdx.x == 0) {
             const uint32_t old = atom_add_release_gpu(&p.counters[stile], 1u);
@@ -610,11 +789,20 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         }
     }
     __syncthreads();
+    // Pair mode: rank 0's MMAs read both CTAs' shared memory and write both tensor
+    // memories; neither CTA frees either until both are past this point (rank 0 has
+    // drained its MMAs by then, rank 1 has read its accumulator or given up).
+    if constexpr (PAIR) cluster_sync_all();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                     "r"(p.tmem_cols)
-                     : "memory");
+        if constexpr (PAIR)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                         "r"(p.tmem_cols)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                         "r"(p.tmem_cols)
+                         : "memory");
     }
 }
 
@@ -640,6 +828,7 @@ int get_encoder() {
 }
 
 struct SpmmPlan {
+    bool pair;  // 256-row tiles on SM pairs (tcgen05 cta_group::2)
     int MT, nh, n_acc, m_tiles, n_tiles, ksplit, n_whole, sx, sr, sw, ctas_per_sm;
     uint32_t x_stage_bytes, val_slot, raw_stage_bytes, tmem_cols;
     uint32_t off_w, off_raw, off_rec, off_tptr, off_bar;
@@ -648,11 +837,60 @@ struct SpmmPlan {
     uint64_t ws_xt;  // decode with a rule: offset of x~ (B rows of K rounded up to 8)
 };
 
+// Clusters of two CTAs (one per SM, the most shared memory) that can be resident at once
+// on the current device: the SM pairs available to pair-mode tiles.  0 when the query
+// fails (pair mode is then not used).
+int device_pair_slots() {
+    static int cache[kMaxDevices];
+    static bool done[kMaxDevices];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev]) {
+        int n = 0;
+        if (cudaFuncSetAttribute(spmm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemLimit) == cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2);
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = kSmemLimit;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n, spmm_kernel<true>, &cfg) != cudaSuccess) n = 0;
+        }
+        (void)cudaGetLastError();
+        cache[dev] = n;
+        done[dev] = true;
+    }
+    return cache[dev];
+}
+
 // Token tile, split-K factor, stage counts and shared-memory layout for M rows of X.
-// sm_count > 0 plans for that many SMs (spw_spmm_plan); 0 asks the current device.
-int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_count = 0) {
+// sm_count > 0 plans for that many SMs (spw_spmm_plan; pair mode then assumes sm_count / 2
+// SM pairs); 0 asks the current device.  allow_pair: the prefill may use 256-row tiles on
+// SM pairs (not the tensor-core decode, whose batches are too narrow for X traffic to
+// matter).  Pair mode is off unless SPW_SPMM_PAIR=1: on B200 it measured 5-9 % slower
+// than one CTA per 128-row tile at M = 2048 (q 102.7 vs 95.3 us), since the kernel is
+// bound by shared-memory bandwidth (decoder traffic, X writes, MMA operand reads) rather
+// than by the L2 traffic of X that it halves.
+int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_count = 0,
+                   bool allow_pair = false) {
     const int sms = sm_count > 0 ? sm_count : device_sm_count();
     if (sms <= 0) return SPW_ERR_CUDA;
+    pl->pair = false;
+    if (allow_pair && !rule && M >= 256 && h->N > (uint32_t)kTileRows) {
+        const char* e = getenv("SPW_SPMM_PAIR");
+        const bool env_on = e && e[0] == '1';
+        const int pairs = env_on ? (sm_count > 0 ? sm_count / 2 : device_pair_slots()) : 0;
+        pl->pair = pairs > 0;
+    }
+    const int tile_rows = pl->pair ? 2 * kTileRows : kTileRows;
     // Token tile (512, 256 or 128 tokens, or all M when smaller) and split-K from a small
     // cost model in microseconds: k-steps x max(decode ~0.7, MMA ~0.76 x MT / 512) per CTA,
     // plus, when K is split, the fp32 partial tile written and summed (~0.1 GB/ms per
@@ -660,8 +898,8 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
     // -- when the tiles need more than one wave but fewer than two -- the first F tiles
     // whole and the rest in k parts that fill the SMs as the whole tiles finish (the span
     // estimated as in-order list scheduling).
-    pl->n_tiles = (int)((h->N + kTileRows - 1) / kTileRows);
-    const long long slots = sms;
+    pl->n_tiles = (int)((h->N + tile_rows - 1) / tile_rows);
+    const long long slots = pl->pair ? (sm_count > 0 ? sm_count / 2 : device_pair_slots()) : sms;
     const long long nk_all = h->n_ktiles;
     const long long kcap = nk_all / 2 > 0 ? (nk_all / 2 < 16 ? nk_all / 2 : 16) : 1;
     double best = 1e300;
@@ -718,7 +956,7 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
     const int per = (M + pl->m_tiles - 1) / pl->m_tiles;
     pl->nh = per > 256 ? 2 : 1;
     pl->MT = (int)round_up_u64((uint64_t)per, 16u * pl->nh);  // each MMA's N a multiple of 16
-    pl->x_stage_bytes = (uint32_t)pl->MT * 128u;
+    pl->x_stage_bytes = (uint32_t)pl->MT * (pl->pair ? 64u : 128u);  // this CTA's share of X
     pl->n_acc = pl->MT <= 32 ? 4 : 1;
     uint32_t cols = 32;
     while (cols < (uint32_t)(pl->n_acc > 1 ? 32 * pl->n_acc : pl->MT)) cols <<= 1;
@@ -735,9 +973,9 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
         const uint32_t off_w = (uint32_t)sx * pl->x_stage_bytes;
         const uint32_t off_raw = off_w + (uint32_t)sw * kWStageBytes;
         const uint32_t off_rec = off_raw + (uint32_t)sr * pl->raw_stage_bytes;
-        const uint32_t off_tptr = off_rec + 128u * kDecoderWarps;
+        const uint32_t off_tptr = off_rec + kRecBytesPerWarp * kDecoderWarps;
         const uint32_t off_bar = (uint32_t)round_up_u64(off_tptr + tptr_bytes, 8);
-        const uint32_t bar_bytes = 8u * (2 * sx + 2 * sr + 2 * sw + 2) + 16u;
+        const uint32_t bar_bytes = 8u * (2 * sx + 2 * sr + 2 * sw + 2 + kPeerSlots) + 16u;
         const size_t total = (size_t)off_bar + bar_bytes + 1024;  // + base alignment slack
         if (total <= (size_t)kSmemLimit) {
             pl->sx = sx;
@@ -760,7 +998,8 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
     // the hybrid was costed for this token tile's tile count; the uniform plans split all
     // tiles (or none)
     pl->n_whole = best_whole >= 0 ? (int)best_whole : (best_ks > 1 ? 0 : (int)tiles);
-    const long long n_split = tiles - pl->n_whole;
+    // split-K counters and partial tiles per 128-row output half (two per pair tile)
+    const long long n_split = (tiles - pl->n_whole) * (pl->pair ? 2 : 1);
     pl->ws_counters = n_split > 0 ? round_up_u64(4ull * (uint64_t)n_split, 256) : 0;
     pl->ws_bytes = n_split > 0
                        ? pl->ws_counters + 4ull * (uint64_t)n_split * pl->ksplit * pl->MT * kTileRows
@@ -776,7 +1015,7 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
                uint64_t ws_bytes, cudaStream_t stream) {
     const bool needs_rule = rule && (t > 0.0f || act_bits);
     SpmmPlan pl;
-    int rc = make_spmm_plan(hdr, M, needs_rule, &pl);
+    int rc = make_spmm_plan(hdr, M, needs_rule, &pl, 0, !rule);
     if (rc != SPW_OK) return rc;
     if (pl.ws_bytes) {
         if (!d_ws) return SPW_ERR_INVALID_ARG;
@@ -802,7 +1041,7 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
     const cuuint64_t dims[2] = {(cuuint64_t)hdr->K, (cuuint64_t)M};
     const cuuint64_t ld_bytes = (cuuint64_t)((M > 1 ? ldx : ((ldx + 7) / 8 * 8)) * 2);
     const cuuint64_t strides[1] = {ld_bytes};
-    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)(pl.MT / pl.nh)};
+    const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)(pl.MT / pl.nh / (pl.pair ? 2 : 1))};
     const cuuint32_t estr[2] = {1, 1};
     CUresult cr = g_encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (void*)d_X, dims, strides, box,
                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -846,20 +1085,36 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
     prm.off_bar = pl.off_bar;
     prm.wait_limit = wait_limit_cycles();
 
-    static size_t attr_smem[kMaxDevices];
+    static size_t attr_smem[2][kMaxDevices];
     int dev = 0;
     SPW_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= kMaxDevices) return SPW_ERR_CUDA;
-    if (attr_smem[dev] < pl.smem) {
-        SPW_CUDA_TRY(cudaFuncSetAttribute(spmm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)pl.smem));
-        attr_smem[dev] = pl.smem;
+    if (attr_smem[pl.pair][dev] < pl.smem) {
+        SPW_CUDA_TRY(cudaFuncSetAttribute(pl.pair ? spmm_kernel<true> : spmm_kernel<false>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem));
+        attr_smem[pl.pair][dev] = pl.smem;
     }
     const long long tiles = (long long)pl.m_tiles * pl.n_tiles;
-    const long long ctas = pl.n_whole + (tiles - pl.n_whole) * pl.ksplit;
+    const long long slots = pl.n_whole + (tiles - pl.n_whole) * pl.ksplit;  // tiles or parts
+    const long long ctas = slots * (pl.pair ? 2 : 1);
     if (ctas > 0x7fffffffll) return SPW_ERR_UNSUPPORTED;
-    const dim3 grid((unsigned)ctas);
-    spmm_kernel<<<grid, kThreads, pl.smem, stream>>>(tmap, prm);
+    if (pl.pair) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)ctas);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = pl.smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        SPW_CUDA_TRY(cudaLaunchKernelEx(&cfg, spmm_kernel<true>, tmap, prm));
+    } else {
+        spmm_kernel<false><<<dim3((unsigned)ctas), kThreads, pl.smem, stream>>>(tmap, prm);
+    }
     SPW_LAUNCH_CHECK();
     return SPW_OK;
 }
@@ -876,7 +1131,7 @@ int spw_spmm_plan(const spw_format* hdr, int M, int sm_count, spw_spmm_plan_info
     const int rc = check_header(hdr);
     if (rc != SPW_OK) return rc;
     SpmmPlan pl;
-    const int prc = make_spmm_plan(hdr, M, false, &pl, sm_count);
+    const int prc = make_spmm_plan(hdr, M, false, &pl, sm_count, true);
     if (prc != SPW_OK) return prc;
     const long long tiles = (long long)pl.m_tiles * pl.n_tiles;
     out->token_tile = pl.MT;
@@ -884,7 +1139,9 @@ int spw_spmm_plan(const spw_format* hdr, int M, int sm_count, spw_spmm_plan_info
     out->weight_tiles = pl.n_tiles;
     out->k_parts = pl.ksplit;
     out->whole_tiles = pl.n_whole;
-    out->ctas = (int32_t)(pl.n_whole + (tiles - pl.n_whole) * pl.ksplit);
+    out->ctas = (int32_t)((pl.n_whole + (tiles - pl.n_whole) * pl.ksplit) * (pl.pair ? 2 : 1));
+    out->cta_pair = pl.pair ? 1 : 0;
+    out->reserved = 0;
     out->workspace_bytes = pl.ws_bytes;
     return SPW_OK;
 }
@@ -892,7 +1149,7 @@ int spw_spmm_plan(const spw_format* hdr, int M, int sm_count, spw_spmm_plan_info
 uint64_t spw_spmm_workspace_bytes(const spw_format* hdr, int M) {
     if (check_header(hdr) != SPW_OK || M < 1) return 0;
     SpmmPlan pl;
-    if (make_spmm_plan(hdr, M, false, &pl) != SPW_OK) return 0;
+    if (make_spmm_plan(hdr, M, false, &pl, 0, true) != SPW_OK) return 0;
     return pl.ws_bytes;
 }
 

@@ -106,7 +106,7 @@ def test_llama7b_prefill_m2048_sampled(name, s):
     layer = workloads.pruned_layer(name, N, K, s, "cfg3")
     X = workloads.normal_act(M, K, "cfg3", name)
     Y, _ = run(layer.W, layer.mask, X)
-    rows = np.sort(workloads.rng("cfg3-rows", name).choice(M, 48, replace=False)).astype(np.int32)
+    rows = np.sort(workloads.rng("cfg3-rows", name).choice(M, 128, replace=False)).astype(np.int32)
     ref = oracle.spmm(layer.W, layer.mask, X, rows)
     assert oracle.rel_err(Y[rows], ref) <= TOL
     assert np.isfinite(Y).all()
@@ -127,3 +127,34 @@ def test_hybrid_split_second_wave(N, K, M):
     ref = oracle.spmm(W, mask, X, rows)
     assert oracle.rel_err(Y[rows], ref) <= TOL
     assert np.isfinite(Y).all()
+
+
+@pytest.mark.parametrize("N,K,M", [(256, 512, 256), (513, 1000, 600), (4096, 4096, 2048),
+                                   (5120, 5120, 2048)])
+def test_pair_mode_parity(N, K, M, monkeypatch):
+    # SM-pair tiles (SPW_SPMM_PAIR=1): 256 weight rows per cluster of two CTAs, one
+    # tcgen05 cta_group::2 MMA per k-slice; the ragged shape leaves the second CTA of the
+    # last pair past N, and 5120 x 5120 at M = 2048 splits its second-wave tiles along K
+    # (one counter and partial tile per 128-row half)
+    monkeypatch.setenv("SPW_SPMM_PAIR", "1")
+    W = workloads.weight(N, K, "pair")
+    mask = workloads.random_mask(N, K, 0.5, "pair")
+    X = workloads.normal_act(M, K, "pair")
+    lin = spw.SparseLinear(dev(W), dev(mask))
+    assert spw.spw_spmm_plan(lin.hdr, M)["cta_pair"] == 1
+    Y, _ = run(W, mask, X)
+    if M <= 600:
+        assert oracle.rel_err(Y, oracle.spmm(W, mask, X)) <= TOL
+    else:
+        rows = np.sort(np.concatenate([workloads.rng("pair-rows", N, M).choice(M, 62, replace=False),
+                                       [0, M - 1]])).astype(np.int32)
+        assert oracle.rel_err(Y[rows], oracle.spmm(W, mask, X, rows)) <= TOL
+    assert np.isfinite(Y).all()
+
+
+def test_pair_mode_identity_exact(monkeypatch):
+    monkeypatch.setenv("SPW_SPMM_PAIR", "1")
+    K = 384
+    X = workloads.normal_act(300, K, "pair-id")
+    Y, _ = run(np.eye(K, dtype=np.float16), np.eye(K, dtype=np.uint8), X)
+    np.testing.assert_array_equal(Y, X.astype(np.float64))

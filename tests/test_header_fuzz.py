@@ -59,9 +59,11 @@ def test_valid_headers_plan_consistently(N, K, units, M, sms):
     if rc != spw.SPW_OK:
         return
     tiles = info.token_tiles * info.weight_tiles
-    assert info.weight_tiles == -(-N // 128)
+    pair = info.cta_pair
+    assert pair in (0, 1) and info.reserved == 0
+    assert info.weight_tiles == -(-N // (256 if pair else 128))
     assert info.token_tile % 16 == 0 and info.token_tile * info.token_tiles >= M
     assert 1 <= info.k_parts and 0 <= info.whole_tiles <= tiles
-    assert info.ctas == info.whole_tiles + (tiles - info.whole_tiles) * info.k_parts
+    assert info.ctas == (info.whole_tiles + (tiles - info.whole_tiles) * info.k_parts) * (2 if pair else 1)
     if info.k_parts > 1:
         assert info.k_parts <= max(1, h.n_ktiles)

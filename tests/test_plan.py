@@ -4,10 +4,23 @@ spw_spmm_plan reports, for a format, M and an SM count, the token tile, how the 
 tiles are split along K and the workspace.  The kernel indexes its CTAs and partial
 tiles from exactly these numbers, so the invariants below are the ones its indexing
 relies on."""
+import os
+
 import pytest
 import torch
 
 import spmm_tiled_column_b200 as spw
+
+
+@pytest.fixture(params=[0, 1], ids=["one-cta-tiles", "pair-tiles"])
+def pair_env(request, monkeypatch):
+    """Plans with the default one-CTA tiles and with SM-pair tiles (SPW_SPMM_PAIR=1, read
+    by the library at plan time)."""
+    if request.param:
+        monkeypatch.setenv("SPW_SPMM_PAIR", "1")
+    else:
+        monkeypatch.delenv("SPW_SPMM_PAIR", raising=False)
+    return request.param
 
 
 def header(N, K, units=300):
@@ -23,18 +36,48 @@ def header(N, K, units=300):
     return h
 
 
-def test_llama7b_prefill_runs_whole_tiles():
+def test_llama7b_prefill_runs_whole_tiles(monkeypatch):
+    monkeypatch.delenv("SPW_SPMM_PAIR", raising=False)
     p = spw.spw_spmm_plan(header(4096, 4096), 2048, 148)
+    assert p["cta_pair"] == 0
     assert (p["token_tile"], p["token_tiles"], p["weight_tiles"]) == (512, 4, 32)
     assert (p["k_parts"], p["whole_tiles"], p["ctas"], p["workspace_bytes"]) == (1, 128, 128, 0)
 
 
-def test_second_wave_tiles_are_split():
+def test_llama7b_prefill_pair_tiles(monkeypatch):
+    monkeypatch.setenv("SPW_SPMM_PAIR", "1")
+    # 256-row tiles on SM pairs: 16 weight tiles x 4 token tiles = 64 pair tiles, one wave
+    # on the 74 SM pairs of 148 SMs
+    p = spw.spw_spmm_plan(header(4096, 4096), 2048, 148)
+    assert p["cta_pair"] == 1
+    assert (p["token_tile"], p["token_tiles"], p["weight_tiles"]) == (512, 4, 16)
+    assert (p["k_parts"], p["whole_tiles"], p["ctas"], p["workspace_bytes"]) == (1, 64, 128, 0)
+
+
+def test_second_wave_tiles_are_split(monkeypatch):
+    monkeypatch.delenv("SPW_SPMM_PAIR", raising=False)
     # 160 output tiles on 148 SMs: 148 run whole, the 12 left over in K parts
     p = spw.spw_spmm_plan(header(5120, 5120), 2048, 148)
     assert p["whole_tiles"] == 148 and p["k_parts"] > 1
     assert p["ctas"] == 148 + 12 * p["k_parts"]
     assert p["workspace_bytes"] == 256 + 12 * p["k_parts"] * 512 * 128 * 4
+
+
+def test_second_wave_pair_tiles_are_split(monkeypatch):
+    monkeypatch.setenv("SPW_SPMM_PAIR", "1")
+    # 80 pair tiles on 74 SM pairs: 74 run whole, the 6 left over in K parts; each of a
+    # split tile's two 128-row halves has its own counter and partial tiles
+    p = spw.spw_spmm_plan(header(5120, 5120), 2048, 148)
+    assert p["cta_pair"] == 1 and p["weight_tiles"] == 20
+    assert p["whole_tiles"] == 74 and p["k_parts"] > 1
+    assert p["ctas"] == 2 * (74 + 6 * p["k_parts"])
+    assert p["workspace_bytes"] == 256 + 12 * p["k_parts"] * 512 * 128 * 4
+
+
+def test_one_cta_tiles_below_256_tokens(monkeypatch):
+    monkeypatch.setenv("SPW_SPMM_PAIR", "1")
+    p = spw.spw_spmm_plan(header(4096, 4096), 255, 148)
+    assert p["cta_pair"] == 0 and p["weight_tiles"] == 32
 
 
 def test_small_token_counts_split_every_tile():
@@ -48,23 +91,28 @@ def test_small_token_counts_split_every_tile():
 @pytest.mark.parametrize("N,K", [(128, 64), (1000, 512), (4096, 4096), (5120, 5120), (11008, 4096),
                                  (5120, 13824), (300, 100)])
 @pytest.mark.parametrize("M", [1, 16, 100, 512, 2048, 5000])
-def test_plan_invariants(N, K, M, sms):
+def test_plan_invariants(N, K, M, sms, pair_env):
     h = header(N, K)
     p = spw.spw_spmm_plan(h, M, sms)
+    pair = p["cta_pair"]
+    assert pair == (1 if (pair_env and M >= 256 and N > 128) else 0)
     mt, tiles = p["token_tile"], p["token_tiles"] * p["weight_tiles"]
-    assert p["weight_tiles"] == -(-N // 128)
+    assert p["weight_tiles"] == -(-N // (256 if pair else 128))
     assert mt % 16 == 0 and 16 <= mt <= 512 and mt * p["token_tiles"] >= M
+    if pair:
+        assert mt >= 128  # each CTA loads mt / 2 tokens per MMA half: whole 8-row atoms
     assert 1 <= p["k_parts"] <= max(1, h.n_ktiles)
     assert 0 <= p["whole_tiles"] <= tiles
-    assert p["ctas"] == p["whole_tiles"] + (tiles - p["whole_tiles"]) * p["k_parts"]
-    split = tiles - p["whole_tiles"]
+    assert p["ctas"] == (p["whole_tiles"] + (tiles - p["whole_tiles"]) * p["k_parts"]) * (2 if pair else 1)
+    split = (tiles - p["whole_tiles"]) * (2 if pair else 1)  # 128-row halves with partials
     if p["k_parts"] == 1:
         assert split == 0 and p["workspace_bytes"] == 0
     else:
         assert split > 0
         assert p["workspace_bytes"] == -(-4 * split // 256) * 256 + 4 * split * p["k_parts"] * mt * 128
+    slots = sms // 2 if pair else sms
     if 0 < p["whole_tiles"] < tiles:  # the hybrid only for more than one and fewer than two waves
-        assert sms < tiles < 2 * sms
+        assert slots < tiles < 2 * slots
 
 
 def test_plan_errors():
