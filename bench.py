@@ -60,7 +60,8 @@ GROUPS = [["q", "k", "v"], ["o"], ["gate", "up"], ["down"]]
 WORKLOAD = ("Llama-7B decoder-layer decode, batch 1: 7 pruned linears (q,k,v,o 4096x4096; "
             "gate,up 11008x4096; down 4096x11008), fp16 N(0,0.02) weights, 50% per-row "
             "magnitude mask, TCB v1; q/k/v share an N(0,1) input, gate/up share an N(0,1) "
-            "input, o has its own; down input SiLU(g)*u with the smallest 50% zeroed; one "
+            "input, o has its own; down input SiLU(g)*u with the smallest 50% zeroed, decoded "
+            "with its activation threshold (only the kept columns' bytes are read); one "
             "grouped decode launch per shared input ([q,k,v],[o],[gate,up],[down]) with the "
             "threshold selection fused in")
 
@@ -180,8 +181,13 @@ def make_layer():
             lin = workloads.pruned_layer(name, N, K, SPARSITY, "bench")
             if group[0] not in inputs:
                 a = DOWN_ACT_SPARSITY if name == "down" else 0.0
-                inputs[group[0]], _ = workloads.decode_act(name, 1, K, a, "bench", group[0])
-            layer.append((name, lin.W, lin.mask, inputs[group[0]], 0.0))
+                x, tt = workloads.decode_act(name, 1, K, a, "bench", group[0])
+                # the down projection runs with its activation threshold (the smallest kept
+                # |v|): the same active set as the zeroed input, and the signal that selects
+                # the column-fetch decode; the dense-input layers run with threshold 0
+                inputs[group[0]] = (x, float(tt[0]) if a > 0 else 0.0)
+            x, t = inputs[group[0]]
+            layer.append((name, lin.W, lin.mask, x, t))
     return layer
 
 
@@ -340,9 +346,11 @@ def run_ours(args, rank, world, local_rank):
         gdata.append(per)
     torch.cuda.synchronize()
 
+    group_t = [layer[idx[g[0]]][4] for g in GROUPS]  # per-group threshold
+
     def step(r):
-        for _, hdrs, bufs, xd, ys, ws in gdata[r]:
-            spw.spw_spmv_group(hdrs, bufs, [xd] * len(bufs), 0.0, None, ys, ws)
+        for gi, (_, hdrs, bufs, xd, ys, ws) in enumerate(gdata[r]):
+            spw.spw_spmv_group(hdrs, bufs, [xd] * len(bufs), group_t[gi], None, ys, ws)
 
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
@@ -409,7 +417,7 @@ def run_ours(args, rank, world, local_rank):
     for gi, group in enumerate(GROUPS):
         def call(r, gi=gi):
             _, hdrs, bufs, xd, ys, ws = gdata[r][gi]
-            spw.spw_spmv_group(hdrs, bufs, [xd] * len(bufs), 0.0, None, ys, ws)
+            spw.spw_spmv_group(hdrs, bufs, [xd] * len(bufs), group_t[gi], None, ys, ws)
         us = time_graphs(call)
         nb = sum(decode_bytes(*layer[idx[n]][1:]) for n in group)
         per_group["+".join(group)] = {"us": round(us, 3), "GB/s": round(nb / (us * 1e-6) / 1e9, 1),
@@ -421,11 +429,30 @@ def run_ours(args, rank, world, local_rank):
             ws1 = base[j].workspace(1)
             def call(r, gi=gi, pi=pi, j=j, ws1=ws1):
                 _, hdrs, bufs, xd, ys, _ws = gdata[r][gi]
-                spw.spw_spmv(hdrs[pi], bufs[pi], xd, 0.0, None, ys[pi], ws1)
+                spw.spw_spmv(hdrs[pi], bufs[pi], xd, group_t[gi], None, ys[pi], ws1)
             us = time_graphs(call)
             nb = decode_bytes(*layer[j][1:])
             per_linear[name] = {"us": round(us, 3), "GB/s": round(nb / (us * 1e-6) / 1e9, 1),
                                 "bytes": int(nb)}
+
+    # Column fetch (spw_set_column_fetch): the down launch (50 % of its activations below
+    # the threshold) reading only its active columns' bytes, against whole tiles
+    dgi = GROUPS.index(["down"])
+
+    def down_call(r):
+        _, hdrs, bufs, xd, ys, ws = gdata[r][dgi]
+        spw.spw_spmv_group(hdrs, bufs, [xd] * len(bufs), group_t[dgi], None, ys, ws)
+    prev_fetch = spw.spw_set_column_fetch(1)
+    try:
+        fetch_us = time_graphs(down_call)
+    finally:
+        spw.spw_set_column_fetch(prev_fetch)
+    down_bytes = decode_bytes(*layer[idx["down"]][1:])
+    column_fetch = {"down_whole_tiles_us": per_group["down"]["us"], "down_column_fetch_us": round(fetch_us, 3),
+                    "down_column_fetch_GB/s": round(down_bytes / (fetch_us * 1e-6) / 1e9, 1),
+                    "how": "spw_set_column_fetch(1): the decode copies only the 16-byte chunks of "
+                           "active columns (default 0: whole tiles)"}
+    assert spw.spw_last_device_status() == spw.SPW_OK
 
     # Fused FFN activation (spw_spmv_ffn): the gate and up decode plus h = SiLU(g) * u and
     # its column set in one launch, against the same work as separate launches (grouped
@@ -571,7 +598,7 @@ def run_ours(args, rank, world, local_rank):
                 for n in out_n[gi]:
                     yv.append(dy[r][yo:yo + n].view(1, -1))
                     yo += n
-                calls.append((spw.DecodeGroup(hdrs, bufs, 1, ws), [xv] * len(bufs), yv))
+                calls.append((spw.DecodeGroup(hdrs, bufs, 1, ws), [xv] * len(bufs), yv, group_t[gi]))
                 xo += in_k[gi]
             e2e_calls.append(calls)
         h2d = 2 * sum(in_k)
@@ -579,8 +606,8 @@ def run_ours(args, rank, world, local_rank):
 
         def e2e_step(r):
             dx[r].view(torch.int16).copy_(hx, non_blocking=True)
-            for call, xs, ys in e2e_calls[r]:
-                call(xs, ys)
+            for call, xs, ys, tg in e2e_calls[r]:
+                call(xs, ys, threshold=tg)
             hy.copy_(dy[r].view(torch.int16), non_blocking=True)
 
         e2e_steps = max(10, min(args.steps, 100))
@@ -647,6 +674,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e,
         "dense_cublas_decode": dense,
         "ffn_fused": ffn_fused,
+        "column_fetch": column_fetch,
         "dense_cublas_step": dense_step,
         "prefill": prefill,
         "prefill_detail": prefill_detail,

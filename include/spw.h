@@ -115,6 +115,24 @@ int spw_version(void);
  * compressed at load time and left alone).  Returns the previous setting. */
 int spw_set_launch_overlap(int enable);
 
+/* Column fetch for the CUDA-core decode (process-wide; mode 0 by default).  With a column
+ * set or a threshold the decode skips the work of inactive columns ("Reduced Matrix
+ * Multiplication" §4.2: only W[:, I] takes part); whether it also skips their bytes is
+ * this switch:
+ *   0  whole tiles: each tile's bitmaps and packed values are streamed with bulk copies,
+ *      inactive columns included (their work is skipped, their bytes are read);
+ *   1  column fetch when a call carries a column set or a threshold above zero: each
+ *      decode warp reads a tile's bitmaps, applies the rule, and copies only the 16-byte
+ *      chunks that hold an active column's values (about 60-75 % of a tile's bytes at
+ *      50 % random activation sparsity, falling with sparsity);
+ *   2  column fetch for every call (for tests and measurement).
+ * Results are identical in every mode (same work split and summation order).  On B200
+ * the down projection at 50 % activation sparsity ran slower with column fetch (whole
+ * tiles keep the weight stream ahead of the decode; column fetch can only start a tile's
+ * copies once the activations are known), hence the default.  Returns the previous mode,
+ * or -1 for a mode outside 0..2 (the setting is then unchanged). */
+int spw_set_column_fetch(int mode);
+
 /* Limit of the product kernels' bounded pipeline waits, in SM clock cycles (process-wide).
  * The default, about one second (2e9 cycles), is far above any normal wait, which ends
  * within microseconds; a wait that runs out makes the kernel stop, drain the copies and

@@ -63,6 +63,7 @@ SIGNATURES = {
     "spw_version": ([], _I),
     "spw_set_launch_overlap": ([_I], _I),
     "spw_set_wait_limit_cycles": ([_U64], _U64),
+    "spw_set_column_fetch": ([_I], _I),
     "spw_format_query": ([_P, _I, _I, _I, _P, _P, _P], _I),
     "spw_compress": ([_P, _I, _P, _I, _I, _I, _P, _U64, _FP, _P], _I),
     "spw_format_read": ([_P, _U64, _FP, _P], _I),
@@ -181,6 +182,15 @@ def spw_set_launch_overlap(enable: bool) -> bool:
     """Enable/disable programmatic launch overlap of consecutive spw_spmv calls (see
     include/spw.h for the one condition it needs); returns the previous setting."""
     return bool(lib().spw_set_launch_overlap(1 if enable else 0))
+
+
+def spw_set_column_fetch(mode: int) -> int:
+    """Decode column fetch: 0 whole tiles (default), 1 when a call carries a column set or a
+    threshold above zero, 2 always; returns the previous mode (see include/spw.h)."""
+    prev = int(lib().spw_set_column_fetch(int(mode)))
+    if prev < 0:
+        raise ValueError("column fetch mode must be 0, 1 or 2")
+    return prev
 
 
 def spw_set_wait_limit_cycles(cycles: int) -> int:

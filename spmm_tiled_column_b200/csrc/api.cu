@@ -13,6 +13,7 @@ __device__ int g_device_status;
 
 std::atomic<int> g_launch_overlap{0};
 std::atomic<long long> g_wait_limit{0};  // 0: the default, spw::kWaitLimitCycles
+std::atomic<int> g_column_fetch{0};
 int* g_status_ptr[spw::kMaxDevices];
 int g_sm_count[spw::kMaxDevices];
 std::mutex g_mutex;
@@ -47,6 +48,8 @@ int device_sm_count() {
 }
 
 bool launch_overlap() { return g_launch_overlap.load(std::memory_order_relaxed) != 0; }
+
+int column_fetch_mode() { return g_column_fetch.load(std::memory_order_relaxed); }
 
 long long wait_limit_cycles() {
     const long long v = g_wait_limit.load(std::memory_order_relaxed);
@@ -91,6 +94,11 @@ int spw_version(void) { return 100; }
 
 int spw_set_launch_overlap(int enable) {
     return g_launch_overlap.exchange(enable ? 1 : 0) != 0;
+}
+
+int spw_set_column_fetch(int mode) {
+    if (mode < 0 || mode > 2) return -1;
+    return g_column_fetch.exchange(mode);
 }
 
 uint64_t spw_set_wait_limit_cycles(uint64_t cycles) {

@@ -68,6 +68,11 @@ constexpr int kUnitsOff = 64;
 constexpr int kRecLoOff = 128;
 constexpr int kRecHiOff = kRecLoOff + 64 * 8 + 16;
 constexpr int kXtOff = kRecHiOff + 64 * 8;  // 64 columns x xt_stride(B) halves
+// Column-fetch mode: two record sets and two x~ sets (tiles alternate), then two value
+// buffers of sparse_vbuf bytes, each with 16 bytes of slack on both sides of the values.
+constexpr int kSpRecOff = 128;
+constexpr int kSpRecSet = 1056;  // one set: low block, 16-byte gap, high block (rounded)
+constexpr int kSpXtOff = kSpRecOff + 2 * kSpRecSet;
 constexpr int kSmemPerSm = 227 * 1024;
 constexpr uint32_t kStageValsOff = 512;  // stage: 64 bitmap words, then packed values
 
@@ -94,6 +99,10 @@ struct SpmvParams {
     int n_layers;
     int* status;
     long long wait_limit;  // pipeline waits, in SM cycles (drains use the fixed limit)
+    // Column fetch (the caller passed a column set or a threshold above zero): no producer;
+    // each consumer copies only its active columns' values (sparse_vbuf bytes per buffer).
+    int sparse_fetch;
+    uint32_t sparse_vbuf;
     int n_tiles;      // all layers
     int total_warps;  // working consumer warps
     int stages;
@@ -116,6 +125,10 @@ __host__ __device__ constexpr int xt_stride(int B) {
 
 __host__ __device__ constexpr uint32_t warp_header_bytes(int B) {
     return (uint32_t)((kXtOff + 64 * 2 * xt_stride(B) + 127) / 128 * 128);
+}
+
+__host__ __device__ constexpr uint32_t sparse_header_bytes(int B) {
+    return (uint32_t)((kSpXtOff + 2 * 64 * 2 * xt_stride(B) + 127) / 128 * 128);
 }
 
 // Column pairs decoded per group: the loads of a group are issued before its
@@ -285,6 +298,14 @@ __device__ inline void decode_pairs(const uint4* recp, const uint16_t* xt, int j
         fma_rows<B>(bits[c], bit1, v1[c], xv[c], acc1);
     }
 }
+
+// 16-byte global -> shared copy through L2 only (cp.async.cg), and its group fences.
+__device__ inline void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ inline void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ inline void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Position of a cursor in the group's tile space: layer, tile within the layer, its k-tile
 // and strip.
@@ -459,6 +480,91 @@ __device__ void ffn_strip(const SpmvParams& p, int s, int lane) {
     }
 }
 
+// End of tile i of a warp's range: when it closes the warp's piece of strip cur.s (the
+// strip's last k-tile, or the warp's last tile), write the piece's rows directly (a
+// strip held by one warp) or publish the fp32 partials and let the strip's last
+// contributor sum every piece in a fixed order (deterministic), then run the FFN step;
+// the accumulators restart at zero.
+template <int B>
+__device__ inline void finish_piece(const SpmvParams& p, const SpmvLayer& L, const Cursor& cur, int i,
+                                    int ntiles, int gw, int lane, float* acc0, float* acc1) {
+    const int T = p.n_tiles, PW = p.total_warps;
+    const int nk = L.n_ktiles;
+    if (cur.kt != nk - 1 && i + 1 != ntiles) return;
+    const int s = cur.s;
+    const int first = L.tile_begin + s * nk;
+    const int g_first = (int)warp_of_tile(first, PW, T);
+    const int g_last = (int)warp_of_tile((long long)first + nk - 1, PW, T);
+    const int count = g_last - g_first + 1;
+    const int r0 = s * kStripRows + 2 * lane;
+    bool finished = false;  // this warp wrote the strip's final outputs (warp-uniform)
+    if (count == 1) {
+#pragma unroll
+        for (int b = 0; b < B; b++) {
+            if (r0 < L.N) L.y[(size_t)b * L.ldy + r0] = __half_as_ushort(__float2half_rn(acc0[b]));
+            if (r0 + 1 < L.N)
+                L.y[(size_t)b * L.ldy + r0 + 1] = __half_as_ushort(__float2half_rn(acc1[b]));
+        }
+        finished = true;
+    } else {
+        // Publish this piece: store the partials, then one release atomic per warp.
+        const int idx = gw - g_first;
+        float2* mine = (float2*)(L.partials + ((size_t)s * L.maxc + idx) * B * 64);
+#pragma unroll
+        for (int b = 0; b < B; b++) mine[b * 32 + lane] = make_float2(acc0[b], acc1[b]);
+        __syncwarp();
+        uint32_t old = 0;
+        if (lane == 0) old = atom_add_release_gpu(&L.counters[s], 1u);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if ((int)old == count - 1) {
+            // Last contributor: sum every piece in a fixed order (deterministic).  Lanes
+            // l and l+16 read rows 4(l mod 16)..+3 of the even and odd pieces with 16-byte
+            // loads, 32 pieces in flight per round; the two halves then add up.
+            __threadfence();
+            const float* base = L.partials + (size_t)s * L.maxc * B * 64;
+            const int half = lane >> 4, r4 = 4 * (lane & 15);
+#pragma unroll 1
+            for (int b = 0; b < B; b++) {
+                float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll 1
+                for (int j0 = half; j0 < count; j0 += 32) {
+                    float4 v[16];
+#pragma unroll
+                    for (int u = 0; u < 16; u++) {
+                        const int j = j0 + 2 * u;
+                        v[u] = j < count ? __ldcg((const float4*)(base + ((size_t)j * B + b) * 64 + r4))
+                                         : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 16; u++) {
+                        acc.x += v[u].x;
+                        acc.y += v[u].y;
+                        acc.z += v[u].z;
+                        acc.w += v[u].w;
+                    }
+                }
+                acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
+                acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 16);
+                acc.z += __shfl_xor_sync(0xffffffffu, acc.z, 16);
+                acc.w += __shfl_xor_sync(0xffffffffu, acc.w, 16);
+                const int r = s * kStripRows + r4;
+                uint16_t* yb = L.y + (size_t)b * L.ldy;
+                if (half == 0) {
+                    if (r < L.N) yb[r] = __half_as_ushort(__float2half_rn(acc.x));
+                    if (r + 1 < L.N) yb[r + 1] = __half_as_ushort(__float2half_rn(acc.y));
+                    if (r + 2 < L.N) yb[r + 2] = __half_as_ushort(__float2half_rn(acc.z));
+                    if (r + 3 < L.N) yb[r + 3] = __half_as_ushort(__float2half_rn(acc.w));
+                }
+            }
+            if (lane == 0) L.counters[s] = 0u;
+            finished = true;
+        }
+    }
+    if (p.ffn_h && finished) ffn_strip<B>(p, s, lane);
+#pragma unroll
+    for (int b = 0; b < B; b++) acc0[b] = acc1[b] = 0.0f;
+}
+
 // Consumer warp gw: its tile range, decoded from its ring; partial sums flushed per strip.
 template <int B>
 __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lane) {
@@ -617,81 +723,210 @@ __device__ void consume(const SpmvParams& p, unsigned char* reg, int gw, int lan
             phase ^= 1u;
         }
 
-        // End of this warp's piece of strip s: write or combine the partial sums.
-        const int nk = L.n_ktiles;
-        if (cur.kt != nk - 1 && i + 1 != ntiles) continue;
-        const int s = cur.s;
-        const int first = L.tile_begin + s * nk;
-        const int g_first = (int)warp_of_tile(first, PW, T);
-        const int g_last = (int)warp_of_tile((long long)first + nk - 1, PW, T);
-        const int count = g_last - g_first + 1;
-        const int r0 = s * kStripRows + 2 * lane;
-        bool finished = false;  // this warp wrote the strip's final outputs (warp-uniform)
-        if (count == 1) {
+        finish_piece<B>(p, L, cur, i, ntiles, gw, lane, acc0, acc1);
+    }
+}
+
+// ---------------------------------------------------------------- column-fetch consumer
+// Used when the caller passes a column set or a threshold above zero: the bytes of
+// inactive columns are never read ("Reduced Matrix Multiplication" §4.2: only W[:, I]
+// takes part in the product).  There is no producer: each consumer warp loads a tile's
+// bitmap words and tile pointers with plain 16-byte loads two tiles ahead of its decode;
+// one tile ahead it applies the threshold rule and column set, builds the records and
+// copies, with per-lane 16-byte cp.async, only the 16-byte chunks that hold an active
+// column's values; tiles alternate between two record / x~ / value sets.
+template <int B>
+struct SpTile {  // one tile before its preparation
+    Cursor c;
+    uint32_t xw[B], aw;
+    uint4 bw;  // this lane's two columns' bitmap words
+    uint32_t u0, u1;
+};
+
+template <int B>
+__device__ inline void sp_load(const SpmvParams& p, const Cursor& c, int lane, SpTile<B>& d) {
+    d.c = c;
+    load_act<B>(p, c, lane, d.xw, d.aw);
+    const SpmvLayer& L = p.L[c.l];
+    d.bw = __ldg((const uint4*)(L.bitmaps + (size_t)c.t * kTileCols) + lane);
+    d.u0 = __ldg(L.tileptr + c.t);
+    d.u1 = __ldg(L.tileptr + c.t + 1);
+}
+
+// Prepares tile d into set `set` (records, x~, value copies as one cp.async group, which
+// is committed even when empty).  Returns the tile's active column count; *all64 when
+// every column is active and B <= 4 (records then in column order, fully unrolled decode).
+template <int B>
+__device__ inline int sp_prepare(const SpmvParams& p, unsigned char* reg, uint32_t reg_s, int set,
+                                 const SpTile<B>& d, int lane, uint32_t ltmask, bool zero_t,
+                                 bool* all64) {
+    constexpr int XS = xt_stride(B);
+    const SpmvLayer& L = p.L[d.c.l];
+    unsigned char* rset = reg + kSpRecOff + set * kSpRecSet;
+    uint2* rec_lo = (uint2*)rset;
+    uint2* rec_hi = (uint2*)(rset + (kRecHiOff - kRecLoOff));
+    uint16_t* xt = (uint16_t*)(reg + kSpXtOff + set * 128 * XS);
+    const uint32_t vb = reg_s + sparse_header_bytes(B) + (uint32_t)set * p.sparse_vbuf + 16u;
+    const uint4 bw = d.bw;
+    const int cl0 = __popc(bw.x), c0 = cl0 + __popc(bw.y);
+    const int cl1 = __popc(bw.z), c1 = cl1 + __popc(bw.w);
+    const int incl = warp_inclusive_scan(c0 + c1, lane);
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    // The tile's value range inside the section and the buffer, and the bitmaps' count
+    // consistent with it (the checks of the whole-tile path); a tile that fails is decoded
+    // as empty and reported.
+    const bool range_ok = d.u1 >= d.u0 && d.u1 <= L.values_units &&
+                          16ull * (d.u1 - d.u0) + 32ull <= (uint64_t)p.sparse_vbuf;
+    const bool ok = range_ok && (uint32_t)(total + 7) >> 3 == d.u1 - d.u0;  // warp-uniform
+    if (!ok && lane == 0) raise_status(p.status, SPW_ERR_FORMAT);
+    const int col = d.c.kt * kTileCols + 2 * lane;
+    const bool in0 = ok && col < L.K && (d.aw & 1u), in1 = ok && col + 1 < L.K && (d.aw & 2u);
+    uint16_t xa[B], xb[B];
+    bool any0 = false, any1 = false;
+#pragma unroll
+    for (int b = 0; b < B; b++) {
+        uint16_t lo, hi;
+        split_halves(d.xw[b], lo, hi);
+        const bool p0 = in0 && (zero_t ? (lo & 0x7fffu) != 0u : passes_threshold(lo, p.t));
+        const bool p1 = in1 && (zero_t ? (hi & 0x7fffu) != 0u : passes_threshold(hi, p.t));
+        xa[b] = p0 ? lo : (uint16_t)0;
+        xb[b] = p1 ? hi : (uint16_t)0;
+        any0 |= p0;
+        any1 |= p1;
+    }
+    any0 = any0 && (bw.x | bw.y) != 0u;
+    any1 = any1 && (bw.z | bw.w) != 0u;
+    const uint32_t m0 = __ballot_sync(0xffffffffu, any0);
+    const uint32_t m1 = __ballot_sync(0xffffffffu, any1);
+    const int n_act = __popc(m0) + __popc(m1);
+    *all64 = B <= 4 && n_act == 64;
+    __syncwarp();  // the tile that used this set two tiles back is fully decoded
+    if (n_act > 0) {
+        const int st0 = incl - c0 - c1;  // index of column 2l's first value in the tile
+        const uint32_t a0 = vb + 2u * (uint32_t)st0;
+        const uint32_t a1 = a0 + 2u * (uint32_t)c0;
+        const uint2 lo0 = make_uint2(bw.x, a0 + 2u * (uint32_t)cl0);
+        const uint2 hi0 = make_uint2(bw.y, a0 + 2u * (uint32_t)c0);
+        const uint2 lo1 = make_uint2(bw.z, a1 + 2u * (uint32_t)cl1);
+        const uint2 hi1 = make_uint2(bw.w, a1 + 2u * (uint32_t)c1);
+        if (*all64) {
+            *(uint4*)(rec_lo + 2 * lane) = make_uint4(lo0.x, lo0.y, lo1.x, lo1.y);
+            *(uint4*)(rec_hi + 2 * lane) = make_uint4(hi0.x, hi0.y, hi1.x, hi1.y);
 #pragma unroll
             for (int b = 0; b < B; b++) {
-                if (r0 < L.N) L.y[(size_t)b * L.ldy + r0] = __half_as_ushort(__float2half_rn(acc0[b]));
-                if (r0 + 1 < L.N)
-                    L.y[(size_t)b * L.ldy + r0 + 1] = __half_as_ushort(__float2half_rn(acc1[b]));
+                xt[(2 * lane) * XS + b] = xa[b];
+                xt[(2 * lane + 1) * XS + b] = xb[b];
             }
-            finished = true;
         } else {
-            // Publish this piece: store the partials, then one release atomic per warp.
-            const int idx = gw - g_first;
-            float2* mine = (float2*)(L.partials + ((size_t)s * L.maxc + idx) * B * 64);
+            const int pos0 = __popc(m0 & ltmask) + __popc(m1 & ltmask);
+            const int pos1 = pos0 + (any0 ? 1 : 0);
+            if (any0) {
+                rec_lo[pos0] = lo0;
+                rec_hi[pos0] = hi0;
 #pragma unroll
-            for (int b = 0; b < B; b++) mine[b * 32 + lane] = make_float2(acc0[b], acc1[b]);
-            __syncwarp();
-            uint32_t old = 0;
-            if (lane == 0) old = atom_add_release_gpu(&L.counters[s], 1u);
-            old = __shfl_sync(0xffffffffu, old, 0);
-            if ((int)old == count - 1) {
-                // Last contributor: sum every piece in a fixed order (deterministic).  Lanes
-                // l and l+16 read rows 4(l mod 16)..+3 of the even and odd pieces with 16-byte
-                // loads, 32 pieces in flight per round; the two halves then add up.
-                __threadfence();
-                const float* base = L.partials + (size_t)s * L.maxc * B * 64;
-                const int half = lane >> 4, r4 = 4 * (lane & 15);
-#pragma unroll 1
-                for (int b = 0; b < B; b++) {
-                    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll 1
-                    for (int j0 = half; j0 < count; j0 += 32) {
-                        float4 v[16];
+                for (int b = 0; b < B; b++) xt[pos0 * XS + b] = xa[b];
+            }
+            if (any1) {
+                rec_lo[pos1] = lo1;
+                rec_hi[pos1] = hi1;
 #pragma unroll
-                        for (int u = 0; u < 16; u++) {
-                            const int j = j0 + 2 * u;
-                            v[u] = j < count ? __ldcg((const float4*)(base + ((size_t)j * B + b) * 64 + r4))
-                                             : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                        }
-#pragma unroll
-                        for (int u = 0; u < 16; u++) {
-                            acc.x += v[u].x;
-                            acc.y += v[u].y;
-                            acc.z += v[u].z;
-                            acc.w += v[u].w;
-                        }
-                    }
-                    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
-                    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 16);
-                    acc.z += __shfl_xor_sync(0xffffffffu, acc.z, 16);
-                    acc.w += __shfl_xor_sync(0xffffffffu, acc.w, 16);
-                    const int r = s * kStripRows + r4;
-                    uint16_t* yb = L.y + (size_t)b * L.ldy;
-                    if (half == 0) {
-                        if (r < L.N) yb[r] = __half_as_ushort(__float2half_rn(acc.x));
-                        if (r + 1 < L.N) yb[r + 1] = __half_as_ushort(__float2half_rn(acc.y));
-                        if (r + 2 < L.N) yb[r + 2] = __half_as_ushort(__float2half_rn(acc.z));
-                        if (r + 3 < L.N) yb[r + 3] = __half_as_ushort(__float2half_rn(acc.w));
-                    }
-                }
-                if (lane == 0) L.counters[s] = 0u;
-                finished = true;
+                for (int b = 0; b < B; b++) xt[pos1 * XS + b] = xb[b];
+            }
+            if ((n_act & 1) && lane == 0) {
+                rec_lo[n_act] = make_uint2(0u, vb);
+                rec_hi[n_act] = make_uint2(0u, vb);
             }
         }
-        if (p.ffn_h && finished) ffn_strip<B>(p, s, lane);
+        // The 16-byte chunks that hold this lane's active columns' values (the two
+        // columns' values are adjacent, so one range covers both when both are active).
+        int lo = 0, hi = -1;
+        if (any0) {
+            lo = st0 >> 3;
+            hi = (st0 + c0 - 1) >> 3;
+        }
+        if (any1) {
+            if (!any0) lo = (st0 + c0) >> 3;
+            hi = (st0 + c0 + c1 - 1) >> 3;
+        }
+        const uint16_t* src = L.values + (size_t)d.u0 * 8;
+        for (int ch = lo; ch <= hi; ch++) cp_async16(vb + 16u * (uint32_t)ch, src + 8 * ch);
+    }
+    cp_async_commit();
+    return n_act;
+}
+
+template <int B>
+__device__ void consume_sparse(const SpmvParams& p, unsigned char* reg, int gw, int lane) {
+    constexpr int XS = xt_stride(B);
+    constexpr int PG = pair_group(B);
+    const int T = p.n_tiles, PW = p.total_warps;
+    if (gw >= PW) return;
+    const int t_begin = (int)((long long)gw * T / PW);
+    const int ntiles = (int)((long long)(gw + 1) * T / PW) - t_begin;
+    const uint32_t reg_s = smem_u32(reg);
+    const uint32_t ltmask = lanemask_lt();
+    const int q = 2 * (lane & 15);
+    const int sh = q + 1;
+    const uint32_t bit0 = 1u << q, bit1 = 2u << q;
+    const int neg2 = p.neg2;
+    const bool zero_t = p.t == 0.0f;
+
+    pdl_wait();
+    pdl_launch_dependents();
+
+    float acc0[B], acc1[B];
 #pragma unroll
-        for (int b = 0; b < B; b++) acc0[b] = acc1[b] = 0.0f;
+    for (int b = 0; b < B; b++) acc0[b] = acc1[b] = 0.0f;
+    Cursor cc = cursor_at(p, t_begin);
+    SpTile<B> d0, d1;
+    sp_load<B>(p, cc, lane, d0);
+    cursor_next(p, cc);
+    if (ntiles > 1) sp_load<B>(p, cc, lane, d1);
+    bool all_cur = false;
+    int n_cur = sp_prepare<B>(p, reg, reg_s, 0, d0, lane, ltmask, zero_t, &all_cur);
+    Cursor cur = d0.c;
+    for (int i = 0; i < ntiles; i++) {
+        bool all_next = false;
+        int n_next = 0;
+        SpTile<B> d2;
+        if (i + 1 < ntiles) {
+            cursor_next(p, cc);  // tile i + 2
+            if (i + 2 < ntiles) sp_load<B>(p, cc, lane, d2);
+            n_next = sp_prepare<B>(p, reg, reg_s, (i + 1) & 1, d1, lane, ltmask, zero_t, &all_next);
+            cp_async_wait<1>();  // tile i's copies (the older group) have landed
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncwarp();  // and every lane's copies are visible to the whole warp
+        if (n_cur > 0) {
+            unsigned char* rset = reg + kSpRecOff + (i & 1) * kSpRecSet;
+            const uint4* recp = (const uint4*)(rset + (lane < 16 ? 0 : (kRecHiOff - kRecLoOff)));
+            const uint16_t* xt = (const uint16_t*)(reg + kSpXtOff + (i & 1) * 128 * XS);
+            if constexpr (B <= 4) {
+                if (all_cur) {
+#pragma unroll
+                    for (int j = 0; j < 64; j += 2 * PG)
+                        decode_pairs<B, PG>(recp, xt, j, sh, neg2, bit0, bit1, acc0, acc1);
+                }
+            }
+            if (!all_cur) {
+                const int n_cols = (n_cur + 1) & ~1;
+                int j = 0;
+                for (; j + 2 * PG <= n_cols; j += 2 * PG)
+                    decode_pairs<B, PG>(recp, xt, j, sh, neg2, bit0, bit1, acc0, acc1);
+                if constexpr (PG > 1) {
+                    for (; j < n_cols; j += 2)
+                        decode_pairs<B, 1>(recp, xt, j, sh, neg2, bit0, bit1, acc0, acc1);
+                }
+            }
+        }
+        pin_acc<B>(acc0, acc1);
+        __syncwarp();
+        finish_piece<B>(p, p.L[cur.l], cur, i, ntiles, gw, lane, acc0, acc1);
+        cur = d1.c;
+        n_cur = n_next;
+        all_cur = all_next;
+        d1 = d2;
     }
 }
 
@@ -714,14 +949,19 @@ spmv_kernel(const __grid_constant__ SpmvParams p) {
     }
     __syncthreads();
     if (warp == W) {
-        produce<B>(p, regions, W, lane);
+        if (!p.sparse_fetch) produce<B>(p, regions, W, lane);
         pdl_launch_dependents();
         return;
     }
-    consume<B>(p, regions + (size_t)warp * p.warp_smem, blockIdx.x * W + warp, lane);
+    if (p.sparse_fetch)
+        consume_sparse<B>(p, regions + (size_t)warp * p.warp_smem, blockIdx.x * W + warp, lane);
+    else
+        consume<B>(p, regions + (size_t)warp * p.warp_smem, blockIdx.x * W + warp, lane);
 }
 
 struct Plan {
+    bool sparse;            // column fetch (consume_sparse)
+    uint32_t sparse_vbuf;   // its value buffer bytes
     int grid, warps, ctas_per_sm, stages;  // warps = consumer warps per CTA
     uint32_t stage_bytes, warp_smem;
     size_t smem;
@@ -743,7 +983,9 @@ int env_int(const char* name, int dflt, int lo, int hi) {
 }
 
 // Launch plan for a group of n layers decoded in one launch (n = 1 for spw_spmv).
-int make_plan(int n, const spw_format* h, int B, Plan* pl) {
+// want_sparse: fetch only active columns when their buffers fit the same launch shape
+// (the work partition, and so the workspace and the results, do not depend on the mode).
+int make_plan(int n, const spw_format* h, int B, Plan* pl, bool want_sparse = false) {
     const int sms = device_sm_count();
     if (sms <= 0) return SPW_ERR_CUDA;
     long long T = 0;
@@ -780,6 +1022,19 @@ int make_plan(int n, const spw_format* h, int B, Plan* pl) {
     pl->stages = stages;
     pl->warp_smem = warp_header_bytes(B) + (uint32_t)stages * pl->stage_bytes;
     pl->smem = kCtaHeader + (size_t)pl->warps * pl->warp_smem;
+    pl->sparse = false;
+    pl->sparse_vbuf = 0;
+    if (want_sparse) {
+        const uint32_t vbuf = (uint32_t)round_up_u64(16ull * max_units + 32, 128);
+        const uint32_t sp_warp = sparse_header_bytes(B) + 2u * vbuf;
+        const long long budget = kSmemPerSm / pl->ctas_per_sm - 1024 - kCtaHeader;
+        if ((long long)pl->warps * sp_warp <= budget) {
+            pl->sparse = true;
+            pl->sparse_vbuf = vbuf;
+            pl->warp_smem = sp_warp;
+            pl->smem = kCtaHeader + (size_t)pl->warps * sp_warp;
+        }
+    }
     // Per layer: the most warps that share one strip under this partition, and the
     // layer's workspace section (arrival counters, then fp32 partial sums).
     uint64_t off = 0;
@@ -859,8 +1114,17 @@ int decode_group_launch(int n, const spw_format* hdrs, const void* const* bufs,
         if (rc != SPW_OK) return rc;
     }
     if (!aligned16(d_ws)) return SPW_ERR_ALIGNMENT;
+    // Column fetch (spw_set_column_fetch): never, when the caller signals activation
+    // sparsity (a column set or a threshold above zero), or always.  The mode changes
+    // which bytes are read, never the result.
+    const int fetch = column_fetch_mode();
+    bool want_sparse = fetch == 2;
+    if (fetch == 1) {
+        want_sparse = threshold > 0.0f;
+        for (int l = 0; l < n; l++) want_sparse = want_sparse || (act_bits && act_bits[l]);
+    }
     Plan pl;
-    int rc = make_plan(n, hdrs, B, &pl);
+    int rc = make_plan(n, hdrs, B, &pl, want_sparse && !ffn);
     if (rc != SPW_OK) return rc;
     if (ws_bytes < pl.ws_bytes) return SPW_ERR_BUFFER_TOO_SMALL;
     int* status = device_status_ptr();
@@ -901,6 +1165,8 @@ int decode_group_launch(int n, const spw_format* hdrs, const void* const* bufs,
     prm.t = threshold;
     prm.neg2 = -2;
     prm.wait_limit = wait_limit_cycles();
+    prm.sparse_fetch = pl.sparse ? 1 : 0;
+    prm.sparse_vbuf = pl.sparse_vbuf;
     if (ffn) {
         prm.ffn_h = ffn->h;
         prm.ffn_ldh = ffn->ldh;

@@ -278,6 +278,9 @@ bool launch_overlap();
 // Limit of the kernels' pipeline waits, in SM cycles (spw_set_wait_limit_cycles).
 long long wait_limit_cycles();
 
+// Decode column-fetch mode set by spw_set_column_fetch (0, 1 or 2).
+int column_fetch_mode();
+
 }  // namespace spw
 
 #define SPW_CUDA_TRY(expr)                         \

@@ -63,6 +63,14 @@ def test_wait_limit_setting(spw):
     assert L.spw_set_wait_limit_cycles(0) == 2_000_000_000
 
 
+def test_column_fetch_setting(spw):
+    L = spw.lib()
+    assert L.spw_set_column_fetch(2) == 0
+    assert L.spw_set_column_fetch(1) == 2
+    assert L.spw_set_column_fetch(3) == -1 and L.spw_set_column_fetch(-1) == -1
+    assert L.spw_set_column_fetch(0) == 1
+
+
 def valid_header(spw, N=128, K=128):
     h = spw.spw_format()
     h.magic, h.version, h.N, h.K, h.TN, h.TK = 0x31424354, 1, N, K, 64, 64

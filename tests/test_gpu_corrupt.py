@@ -57,9 +57,17 @@ def status():
     return spw.spw_last_device_status()
 
 
+@pytest.fixture
+def fetch_mode(request):
+    prev = spw.spw_set_column_fetch(request.param)
+    yield request.param
+    spw.spw_set_column_fetch(prev)
+
+
+@pytest.mark.parametrize("fetch_mode", [0, 2], ids=["whole-tiles", "column-fetch"], indirect=True)
 @pytest.mark.parametrize("what", ["bitmaps", "overclaim", "tileptr"])
 @pytest.mark.parametrize("B", [1, 8])
-def test_decode_reports_format_and_recovers(what, B):
+def test_decode_reports_format_and_recovers(what, B, fetch_mode):
     W, mask, lin = layer()
     assert status() == spw.SPW_OK
     x = workloads.normal_act(B, K, "corrupt", B)

@@ -173,3 +173,31 @@ def test_llama13b_full_size_b1(shape, s):
     y, _ = run(layer.W, layer.mask, raw, float(np.float32(t[0])))
     ref = oracle.spmv(layer.W, layer.mask, raw, float(np.float32(t[0])))
     assert oracle.rel_err(y, ref) <= TOL
+
+
+@pytest.mark.parametrize("N,K,B,a,t,use_bits", [
+    (4096, 11008, 1, 0.5, 0.0, False), (4096, 11008, 1, 0.5, 0.3, False),
+    (1000, 3000, 4, 0.3, 0.2, False), (300, 200, 16, 0.7, 0.1, False),
+    (4096, 4096, 1, 0.0, 0.0, False), (513, 1000, 2, 0.5, 0.0, True),
+    (11008, 4096, 8, 0.5, 0.25, True)])
+def test_column_fetch_equals_whole_tiles(N, K, B, a, t, use_bits, monkeypatch):
+    # Column fetch (only the active columns' bytes are copied) and whole-tile copies share
+    # the work split and the summation order, so they give the same bits; both match the
+    # oracle.  spw_set_column_fetch(2) forces column fetch, 0 whole tiles.
+    W = workloads.weight(N, K, "fetch")
+    mask = workloads.random_mask(N, K, 0.5, "fetch")
+    x = workloads.zero_random(workloads.normal_act(B, K, "fetch", B), a, "fetch")
+    bits = None
+    if use_bits:
+        bits, _ = oracle.select_topk(x, K // 2)
+    ys = []
+    try:
+        for mode in (0, 2):
+            spw.spw_set_column_fetch(mode)
+            y, _ = run(W, mask, x, t, bits)
+            ys.append(y)
+    finally:
+        spw.spw_set_column_fetch(0)
+    np.testing.assert_array_equal(ys[0], ys[1])
+    ref = oracle.spmv(W, mask, x, t, bits)
+    assert oracle.rel_err(ys[1], ref) <= TOL
