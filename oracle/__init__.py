@@ -75,9 +75,12 @@ def _load():
         lib.orc_double_to_half.restype = ctypes.c_uint16
         lib.orc_round_to_half.argtypes = [P, ctypes.c_int64, P]
         lib.orc_silu_mul.argtypes = [P, P, i, i, i, P]
+        lib.orc_spmm_tokens.argtypes = [P, i, P, i, i, i, P, i, i, f, P, i, P]
+        lib.orc_token_groups.argtypes = [P, i, i, i, f, i, P, P]
         for name in ("orc_tcb_query", "orc_tcb_encode", "orc_tcb_decode",
                      "orc_select_threshold", "orc_select_topk", "orc_spmv", "orc_spmm",
-                     "orc_round_to_half", "orc_silu_mul"):
+                     "orc_round_to_half", "orc_silu_mul", "orc_spmm_tokens",
+                     "orc_token_groups"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -200,6 +203,44 @@ def spmm(W: np.ndarray, mask: np.ndarray, X: np.ndarray,
     _check(_load().orc_spmm(_ptr(Wb), K, _ptr(mask), K, N, K, _ptr(Xb), M, K, _ptr(rows),
                             n_rows, _ptr(Y)), "orc_spmm")
     return Y
+
+
+def spmm_tokens(W: np.ndarray, mask: np.ndarray, X: np.ndarray, t: float,
+                rows: np.ndarray | None = None) -> np.ndarray:
+    """fp64 prefill result with a per-token index set: Y = X~ . W_masked^T, where x~[m,k]
+    keeps X[m,k] only when the threshold rule keeps it (only the listed rows if given)."""
+    Wb = _half_bits(W)
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    Xb = _half_bits(np.atleast_2d(X))
+    N, K = Wb.shape
+    M = Xb.shape[0]
+    assert Xb.shape[1] == K and mask.shape == (N, K)
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, dtype=np.int32)
+        n_rows = rows.size
+    else:
+        n_rows = M
+    Y = np.zeros((n_rows, N), dtype=np.float64)
+    _check(_load().orc_spmm_tokens(_ptr(Wb), K, _ptr(mask), K, N, K, _ptr(Xb), M, K,
+                                   ctypes.c_float(t), _ptr(rows), n_rows, _ptr(Y)),
+           "orc_spmm_tokens")
+    return Y
+
+
+def token_groups(X: np.ndarray, t: float, token_tile: int) -> tuple[np.ndarray, np.ndarray]:
+    """Token grouping: (perm uint32[M], tile_sig uint64[ceil(M/T), words]).
+
+    perm lists the tokens sorted by k-tile signature (ties by index); tile_sig[j] is the
+    OR of the signatures of positions j*T .. (j+1)*T-1."""
+    Xb = _half_bits(np.atleast_2d(X))
+    M, K = Xb.shape
+    words = (-(-K // 64) + 63) // 64
+    tiles = -(-M // token_tile)
+    perm = np.zeros(M, dtype=np.uint32)
+    tile_sig = np.zeros((tiles, words), dtype=np.uint64)
+    _check(_load().orc_token_groups(_ptr(Xb), M, K, K, ctypes.c_float(t), int(token_tile),
+                                    _ptr(perm), _ptr(tile_sig)), "orc_token_groups")
+    return perm, tile_sig
 
 
 def round_to_half(v: np.ndarray) -> np.ndarray:

@@ -40,6 +40,8 @@
  *   orc_double_to_half   IEEE-754 binary16 encoding, round to nearest, ties to even
  *   orc_round_to_half    (and its element-wise form).
  *   orc_silu_mul         h = fp16(SiLU(g) * u) for the gated FFN    [RMM] §4.2, §3.2.
+ *   orc_spmm_tokens      Y = X~ . W_masked^T, each token its own index set [RMM] §4.2, §6.1.
+ *   orc_token_groups     token order and token-tile k-tile sets      [RMM] §6.1.
  *
  * Pins: tests/test_oracle_*.py check every function against things fixed outside this
  * file: numpy's binary16 decoder over all 65536 bit patterns, hand-derived TCB buffers
@@ -471,5 +473,92 @@ int orc_silu_mul(const uint16_t* g, const uint16_t* u, int B, int N, int ld, uin
             double silu = gv / (1.0 + exp(-gv));
             h[(size_t)b * ld + r] = orc_double_to_half(silu * uv);
         }
+    return ORC_OK;
+}
+
+/* Prefill with a per-token index set ([RMM] §4.2: the reduced product over the columns a
+ * token keeps; §6.1: every token of a batch has its own index set):
+ *   Y[m,n] = sum over k of x~[m,k] * W[n,k] * mask[n,k],
+ *   x~[m,k] = X[m,k] if the threshold rule keeps it (X[m,k] != 0 and not |X[m,k]| < t),
+ *             else 0,
+ * i.e. row m is the decode result of token m alone (orc_spmv with B = 1).  When rows is
+ * not NULL only the listed rows are computed, in the listed order. */
+int orc_spmm_tokens(const uint16_t* W, int ldw, const uint8_t* mask, int ld_mask, int N, int K,
+                    const uint16_t* X, int M, int ldx, float t, const int* rows, int n_rows,
+                    double* Y) {
+    if (!W || !mask || !X || !Y || check_dims(N, K, ldw, ld_mask) || M < 0 || ldx < K ||
+        !valid_threshold(t))
+        return ORC_ERR_ARG;
+    int count = rows ? n_rows : M;
+    for (int i = 0; i < count; i++) {
+        int m = rows ? rows[i] : i;
+        if (m < 0 || m >= M) return ORC_ERR_ARG;
+        for (int n = 0; n < N; n++) {
+            double acc = 0.0;
+            for (int k = 0; k < K; k++) {
+                if (mask[(size_t)n * ld_mask + k] == 0) continue;
+                double xv = orc_half_to_double(X[(size_t)m * ldx + k]);
+                if (!passes_threshold(xv, (double)t)) continue; /* k is not in token m's set */
+                acc += xv * orc_half_to_double(W[(size_t)n * ldw + k]);
+            }
+            Y[(size_t)i * N + n] = acc;
+        }
+    }
+    return ORC_OK;
+}
+
+/* Token grouping ([RMM] §6.1: tokens whose index sets are the same or alike go into one
+ * group, and each group runs its own dense product over the columns it uses).  The
+ * pages leave the similarity measure open; this is the plainest reading at the
+ * granularity of the stored tiles (64 columns):
+ *   - signature of token m: bit kt (bit kt % 64 of word kt / 64, words = ceil(K / 4096))
+ *     is set iff the threshold rule keeps some X[m,k] with 64 kt <= k < 64 kt + 64;
+ *   - order: tokens sorted by signature, the words compared one after another from word
+ *     0 as unsigned 64-bit integers, equal signatures by lower token index; perm[r] is the
+ *     token at position r (identical signatures end up next to each other);
+ *   - token tiles: positions [j T, min((j + 1) T, M)) form tile j; its signature
+ *     tile_sig[j * words + w] is the OR of its tokens' signatures -- the k-tiles that
+ *     tile's product has to visit.
+ * K <= 16384 (at most 4 words). */
+typedef struct {
+    uint64_t sig[4];
+    int words;
+    int token;
+} token_key;
+
+static int cmp_token_key(const void* a, const void* b) {
+    const token_key* x = (const token_key*)a;
+    const token_key* y = (const token_key*)b;
+    for (int w = 0; w < x->words; w++)
+        if (x->sig[w] != y->sig[w]) return x->sig[w] < y->sig[w] ? -1 : 1;
+    return (x->token > y->token) - (x->token < y->token);
+}
+
+int orc_token_groups(const uint16_t* X, int M, int K, int ldx, float t, int T, uint32_t* perm,
+                     uint64_t* tile_sig) {
+    if (!X || !perm || !tile_sig || M < 1 || K < 1 || K > 16384 || ldx < K || T < 1 ||
+        !valid_threshold(t))
+        return ORC_ERR_ARG;
+    int n_ktiles = (K + 63) / 64;
+    int words = (n_ktiles + 63) / 64;
+    token_key* keys = (token_key*)calloc((size_t)M, sizeof(token_key));
+    if (!keys) return ORC_ERR_ARG;
+    for (int m = 0; m < M; m++) {
+        keys[m].words = words;
+        keys[m].token = m;
+        for (int k = 0; k < K; k++)
+            if (passes_threshold(orc_half_to_double(X[(size_t)m * ldx + k]), (double)t)) {
+                int kt = k / 64;
+                keys[m].sig[kt / 64] |= (uint64_t)1 << (kt % 64);
+            }
+    }
+    qsort(keys, (size_t)M, sizeof(token_key), cmp_token_key);
+    int tiles = (M + T - 1) / T;
+    for (int j = 0; j < tiles * words; j++) tile_sig[j] = 0;
+    for (int r = 0; r < M; r++) {
+        perm[r] = (uint32_t)keys[r].token;
+        for (int w = 0; w < words; w++) tile_sig[(size_t)(r / T) * words + w] |= keys[r].sig[w];
+    }
+    free(keys);
     return ORC_OK;
 }

@@ -25,6 +25,7 @@ SELECT_PINS = "select"
 PRODUCT_PINS = "products"
 HALF_PINS = "half"
 FFN_PINS = "ffn"
+TOKEN_PINS = "tokens"
 
 CHILD = {
     "half": "import test_oracle_half as H; H.test_all_half_patterns_match_numpy()",
@@ -47,6 +48,14 @@ CHILD = {
             "Q.test_round_to_half_matches_numpy(); Q.test_round_to_half_round_trip_and_ties()\n"
             "Q.test_silu_mul_worked_value(); Q.test_silu_odd_part_identity()\n"
             "Q.test_silu_limits_and_zeros()"),
+    "tokens": ("import test_oracle_tokens as G\n"
+               "[G.test_spmm_tokens_exact_rational(s) for s in range(20)]\n"
+               "[G.test_each_row_is_that_tokens_decode(t) for t in (0.0, 0.4, 1.2)]\n"
+               "G.test_threshold_zero_is_the_plain_product(); G.test_rule_boundary_and_rows()\n"
+               "G.test_groups_reverse_order_closed_form()\n"
+               "G.test_groups_equal_signatures_keep_index_order()\n"
+               "G.test_groups_word_zero_decides_first_and_threshold_counts()\n"
+               "[G.test_groups_match_vectorised_restatement(s) for s in range(12)]"),
 }
 
 MUTANTS = [
@@ -83,6 +92,19 @@ MUTANTS = [
     ("half_ties_away", "if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;",
      "if (frac >= 0.5) r += 1.0;", [FFN_PINS]),
     ("half_no_carry", "    if (r == 2048.0) {", "    if (r == 4096.0) {", [FFN_PINS]),
+    ("tokens_rule_ignored",
+     "if (!passes_threshold(xv, (double)t)) continue; /* k is not in token m's set */", "",
+     [TOKEN_PINS]),
+    ("tokens_other_token", "double xv = orc_half_to_double(X[(size_t)m * ldx + k]);",
+     "double xv = orc_half_to_double(X[(size_t)(M - 1 - m) * ldx + k]);", [TOKEN_PINS]),
+    ("token_order_reversed",
+     "if (x->sig[w] != y->sig[w]) return x->sig[w] < y->sig[w] ? -1 : 1;",
+     "if (x->sig[w] != y->sig[w]) return x->sig[w] < y->sig[w] ? 1 : -1;", [TOKEN_PINS]),
+    ("token_ties_high_first", "return (x->token > y->token) - (x->token < y->token);",
+     "return (x->token < y->token) - (x->token > y->token);", [TOKEN_PINS]),
+    ("token_ktile_width", "int kt = k / 64;", "int kt = k / 32;", [TOKEN_PINS]),
+    ("token_tile_shifted", "tile_sig[(size_t)(r / T) * words + w] |= keys[r].sig[w];",
+     "tile_sig[(size_t)(((r + 1) % M) / T) * words + w] |= keys[r].sig[w];", [TOKEN_PINS]),
 ]
 
 
