@@ -637,6 +637,10 @@ def run_ours(args, rank, world, local_rank):
         prefill, prefill_detail = run_prefill(args, dev, stream, tc_peak, peak_src)
     except Exception as exc:  # the prefill leg must not hide the decode number
         prefill = {"unavailable": f"{type(exc).__name__}: {exc}"[:300]}
+    try:
+        prefill_tokens = run_prefill_tokens(dev, stream)
+    except Exception as exc:
+        prefill_tokens = {"unavailable": f"{type(exc).__name__}: {exc}"[:300]}
 
     # Decode time against a plain copy of the same bytes (the launch's compressed
     # weights), per grouped launch: the three-layer-format page's comparison of global
@@ -678,6 +682,7 @@ def run_ours(args, rank, world, local_rank):
         "dense_cublas_step": dense_step,
         "prefill": prefill,
         "prefill_detail": prefill_detail,
+        "prefill_tokens": prefill_tokens,
         "decode_vs_plain_copy": decode_vs_read,
         "storage_bytes_per_weight": storage,
     }
@@ -760,6 +765,65 @@ def run_prefill(args, dev, stream, tc_peak, peak_src):
                              "with fp16 reduced-precision reductions disabled"}
     flat["peak_tflops"] = tc_peak
     return flat, detail
+
+
+def run_prefill_tokens(dev, stream):
+    """spw_spmm_tokens (per-token index sets, token grouping; "Reduced Matrix
+    Multiplication" §6.1-§6.2) at M = 2048 on the down shape: tokens from D domains that
+    each use a random half of the 64-column channel blocks, SiLU(g) * u values, threshold
+    0.3.  Against spw_spmm and cuBLAS on the same thresholded input (no skipping); graph
+    replays over 3 rotated operand sets."""
+    import torch
+    import spmm_tiled_column_b200 as spw
+    M, R, t, name = 2048, 3, 0.3, "down"
+    N, K = workloads.LLAMA7B_LAYERS[name]
+    lin = workloads.pruned_layer(name, N, K, SPARSITY, "bench-tokens")
+    W = torch.from_numpy(lin.W.view(np.int16)).to(dev).view(torch.float16)
+    mask = torch.from_numpy(lin.mask).to(dev)
+    sl = spw.SparseLinear(W, mask)
+    bufs = [sl.buf] + [sl.buf.clone() for _ in range(R - 1)]
+    Wd0 = W * mask.to(torch.float16)
+    Wds = [Wd0] + [Wd0.clone() for _ in range(R - 1)]
+    plan = spw.spw_spmm_tokens_plan(sl.hdr, M)
+    out = {"layer": f"{name} {N}x{K}", "M": M, "threshold": t, "token_tile": plan["token_tile"]}
+    for D in (1, 4):
+        Xs, Xts = [], []
+        for r in range(R):
+            X, _ = workloads.domain_tokens(M, K, D, 0.5, "bench-tokens", r, silu=True)
+            Xd = _dev(X)
+            Xs.append(Xd)
+            keep = (Xd != 0) & ~(Xd.abs() < t)
+            Xts.append(torch.where(keep, Xd, torch.zeros_like(Xd)))
+        Ys = [torch.empty((M, N), device=dev, dtype=torch.float16) for _ in range(R)]
+        wss = [torch.zeros(plan["workspace_bytes"], dtype=torch.uint8, device=dev) for _ in range(R)]
+        us = graph_us([(lambda r=r: spw.spw_spmm_tokens(sl.hdr, bufs[r], Xs[r], t, Ys[r], wss[r]))
+                       for r in range(R)], stream)
+        gws = [torch.empty(spw.spw_group_tokens_workspace_bytes(M, K), dtype=torch.uint8, device=dev)
+               for _ in range(R)]
+        gus = graph_us([(lambda r=r: spw.spw_group_tokens(Xs[r], t, plan["token_tile"], gws[r]))
+                        for r in range(R)], stream)
+        _, _, tsig = spw.spw_group_tokens(Xs[0], t, plan["token_tile"], gws[0])
+        ts = tsig.cpu().numpy().view(np.uint64)
+        visited = [sum(bin(int(v)).count("1") for v in row) for row in ts]
+        swss = [torch.zeros(max(spw.spw_spmm_workspace_bytes(sl.hdr, M), 16), dtype=torch.uint8,
+                            device=dev) for _ in range(R)]
+        sus = graph_us([(lambda r=r: spw.spw_spmm(sl.hdr, bufs[r], Xts[r], Ys[r], swss[r]))
+                        for r in range(R)], stream)
+        dus = graph_us([(lambda r=r: torch.matmul(Xts[r], Wds[r].t(), out=Ys[r])) for r in range(R)],
+                       stream)
+        assert spw.spw_last_device_status() == spw.SPW_OK
+        nk = -(-K // 64)
+        out[f"domains_{D}"] = {
+            "us": round(us, 2), "grouping_us": round(gus, 2),
+            "k_tiles_visited_per_token_tile": visited, "k_tiles": nk,
+            "spw_spmm_same_input_us": round(sus, 2), "dense_cublas_same_input_us": round(dus, 2),
+            "speedup_vs_spw_spmm": round(sus / us, 3), "speedup_vs_dense": round(dus / us, 3)}
+        del Xs, Xts, Ys, wss, gws, swss
+    out["how"] = ("spw_spmm_tokens = grouping (signature, rank, gather of x~) + the product over "
+                  "each token tile's k-tiles; the kernel time follows the longest k-tile list")
+    del bufs, Wds, Wd0, sl
+    torch.cuda.empty_cache()
+    return out
 
 
 def storage_bytes_per_weight(dev):

@@ -328,6 +328,59 @@ int spw_spmm_plan(const spw_format* hdr, int M, int sm_count, spw_spmm_plan_info
 int spw_spmm(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int M, int ldx,
              uint16_t* d_Y, int ldy, void* d_ws, uint64_t ws_bytes, void* stream);
 
+/* Token grouping ("Reduced Matrix Multiplication" §6.1: tokens whose channel sets are the
+ * same or alike are grouped, each group running its own dense product; the pages leave
+ * the similarity open, and this is the plainest reading at the stored tile width):
+ *   signature of token m: bit kt (bit kt % 64 of word kt / 64, words = ceil(ceil(K/64)
+ *     / 64)) is set iff the threshold rule keeps some X[m,k], 64 kt <= k < 64 kt + 64;
+ *   order: tokens sorted by signature (words compared from word 0 as unsigned 64-bit
+ *     integers), equal signatures by lower token index;
+ *   outputs: d_perm[r] = the token at position r (M words); row r of d_Xg (M rows at
+ *     ldxg >= K, a multiple of 8) = x~ of that token (entries the rule drops written as
+ *     +0, columns K..ldxg-1 as 0); d_tile_sig[j * words + w] = OR of the signatures of
+ *     positions j T .. min((j+1) T, M) - 1 (T = token_tile), i.e. the k-tiles token tile
+ *     j has to visit.
+ * 1 <= M <= 16384, 1 <= K <= 16384, token_tile >= 1, t finite and >= 0.  d_ws: scratch of
+ * spw_group_tokens_workspace_bytes(M, K) bytes (no state kept between calls).
+ * Deterministic.  Asynchronous.  Errors: INVALID_ARG, ALIGNMENT (any pointer not 16-byte
+ * aligned), UNSUPPORTED (M or K too large), BUFFER_TOO_SMALL, CUDA. */
+uint64_t spw_group_tokens_workspace_bytes(int M, int K);
+int spw_group_tokens(const uint16_t* d_X, int M, int K, int ldx, float t, int token_tile,
+                     uint16_t* d_Xg, int ldxg, uint32_t* d_perm, uint64_t* d_tile_sig, void* d_ws,
+                     uint64_t ws_bytes, void* stream);
+
+/* Workspace bytes of spw_spmm_tokens for M tokens (0 for an invalid header, M < 1, or
+ * M or K above 16384). */
+uint64_t spw_spmm_tokens_workspace_bytes(const spw_format* hdr, int M);
+
+/* The launch plan of spw_spmm_tokens, as spw_spmm_plan reports it for spw_spmm (never
+ * SM-pair tiles); workspace_bytes is spw_spmm_tokens_workspace_bytes.  token_tile is the
+ * T of its token grouping.  Errors: as spw_spmm_plan, plus UNSUPPORTED (M or K too
+ * large). */
+int spw_spmm_tokens_plan(const spw_format* hdr, int M, int sm_count, spw_spmm_plan_info* out);
+
+/* Prefill with a per-token index set ("Reduced Matrix Multiplication" §4.2, each token
+ * keeping its own channels; §6.1-§6.2, token grouping):
+ *   Y[m,n] = sum_k x~[m,k] W[n,k] mask[n,k],
+ *   x~[m,k] = X[m,k] if X[m,k] != 0 and not |X[m,k]| < threshold, else 0,
+ * i.e. row m is what spw_spmv computes for token m alone.  The call groups the tokens
+ * as spw_group_tokens does, with T = the token tile of spw_spmm_tokens_plan, into the
+ * workspace, then runs the prefill product (as spw_spmm) on the grouped rows, where
+ * every token tile visits only the k-tiles of its tile signature (a skipped k-tile holds
+ * no kept entry of the tile's tokens) and its rows are written back to their tokens' rows
+ * of Y.  Without a shared zero pattern among the tokens of a tile nothing is skipped
+ * and the call costs spw_spmm plus the grouping (a read of X, a write of x~).
+ * Non-finite kept entries reach every output row, as in spw_spmm.  M >= 0 (M == 0 does
+ * nothing), M and K <= 16384, threshold finite and >= 0.  d_ws: at least
+ * spw_spmm_tokens_workspace_bytes(hdr, M) bytes; its first bytes are the split-K
+ * counters of spw_spmm (zero before the first call, left zero by each call that
+ * completes), then the grouped input, perm, tile signatures and grouping scratch.
+ * Deterministic.  Asynchronous.  Errors: as spw_spmm, plus UNSUPPORTED (M or K too
+ * large) and INVALID_ARG for a bad threshold or a NULL workspace. */
+int spw_spmm_tokens(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int M, int ldx,
+                    float threshold, uint16_t* d_Y, int ldy, void* d_ws, uint64_t ws_bytes,
+                    void* stream);
+
 /* Workspace bytes spw_spmv_tc needs (the rules of spw_spmm_workspace_bytes with M = B);
  * 0 for B outside 1..16. */
 uint64_t spw_spmv_tc_workspace_bytes(const spw_format* hdr, int B);

@@ -84,6 +84,11 @@ SIGNATURES = {
     "spw_spmv_ffn_workspace_bytes": ([_FP, _FP, _I], _U64),
     "spw_spmm_plan": ([_FP, _I, _I, ctypes.POINTER(spw_spmm_plan_info)], _I),
     "spw_spmv_ffn": ([_FP, _P, _FP, _P, _P, _I, _I, _F, _P, _I, _P, _P, _U64, _P], _I),
+    "spw_group_tokens_workspace_bytes": ([_I, _I], _U64),
+    "spw_group_tokens": ([_P, _I, _I, _I, _F, _I, _P, _I, _P, _P, _P, _U64, _P], _I),
+    "spw_spmm_tokens_workspace_bytes": ([_FP, _I], _U64),
+    "spw_spmm_tokens_plan": ([_FP, _I, _I, ctypes.POINTER(spw_spmm_plan_info)], _I),
+    "spw_spmm_tokens": ([_FP, _P, _P, _I, _I, _F, _P, _I, _P, _U64, _P], _I),
 }
 
 
@@ -418,6 +423,67 @@ def spw_spmm_plan(hdr, M: int, sm_count: int = 0) -> dict:
     return {name: getattr(info, name) for name, _ in info._fields_}
 
 
+def spw_group_tokens_workspace_bytes(M: int, K: int) -> int:
+    return int(lib().spw_group_tokens_workspace_bytes(int(M), int(K)))
+
+
+def spw_group_tokens(X: torch.Tensor, t: float, token_tile: int, ws: torch.Tensor | None = None,
+                     stream=None) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Token grouping of X (M x K fp16): (Xg M x ceil8(K) fp16, perm int32[M], tile_sig
+    int64[ceil(M / token_tile), words]); see spw_group_tokens in include/spw.h."""
+    X2, ldx = _rows(_half(X, "X"), "X")
+    M, K = X2.shape[0], X2.shape[1]
+    words = ((K + 63) // 64 + 63) // 64
+    ldg = (K + 7) // 8 * 8
+    Xg = torch.empty((M, ldg), dtype=torch.float16, device=X.device)
+    perm = torch.empty(M, dtype=torch.int32, device=X.device)
+    tsig = torch.empty((-(-M // int(token_tile)), words), dtype=torch.int64, device=X.device)
+    need = spw_group_tokens_workspace_bytes(M, K)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
+    _check("spw_group_tokens", lib().spw_group_tokens(
+        _ptr(X2), M, K, ldx, ctypes.c_float(t), int(token_tile), _ptr(Xg), ldg, _ptr(perm),
+        _ptr(tsig), _ptr(ws), ws.numel(), _stream(stream)))
+    return Xg, perm, tsig
+
+
+def spw_spmm_tokens_workspace_bytes(hdr, M: int) -> int:
+    return int(lib().spw_spmm_tokens_workspace_bytes(ctypes.byref(_hdr(hdr)), int(M)))
+
+
+def spw_spmm_tokens_plan(hdr, M: int, sm_count: int = 0) -> dict:
+    """The launch plan of spw_spmm_tokens (its token tile is the grouping's T)."""
+    info = spw_spmm_plan_info()
+    _check("spw_spmm_tokens_plan", lib().spw_spmm_tokens_plan(
+        ctypes.byref(_hdr(hdr)), int(M), int(sm_count), ctypes.byref(info)))
+    return {name: getattr(info, name) for name, _ in info._fields_}
+
+
+def spw_spmm_tokens(hdr, buf: torch.Tensor, X: torch.Tensor, threshold: float,
+                    Y: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """Prefill with per-token index sets: Y = X~ . W_masked^T, tokens grouped by the
+    k-tiles they use (see spw_spmm_tokens in include/spw.h).  ws: a uint8 workspace of
+    spw_spmm_tokens_workspace_bytes(hdr, M) bytes whose first (split-K counter) bytes are
+    zero; allocated zeroed here when omitted."""
+    h = _hdr(hdr)
+    X2, ldx = _rows(_half(X, "X"), "X")
+    M = X2.shape[0]
+    if Y is None:
+        Y = torch.empty((M, h.N), dtype=torch.float16, device=X.device)
+    Y2, ldy = _rows(_half(Y, "Y"), "Y")
+    _need_buf(buf, h)
+    _need(X2, M, h.K, "X")
+    _need(Y2, M, h.N, "Y")
+    if ws is None:
+        ws = torch.zeros(max(spw_spmm_tokens_workspace_bytes(h, M), 16), dtype=torch.uint8,
+                         device=X.device)
+    _check("spw_spmm_tokens", lib().spw_spmm_tokens(
+        ctypes.byref(h), _ptr(buf), _ptr(X2), M, ldx, ctypes.c_float(threshold), _ptr(Y2), ldy,
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return Y
+
+
 def spw_spmv_tc_workspace_bytes(hdr, B: int) -> int:
     h = _hdr(hdr)
     return int(lib().spw_spmv_tc_workspace_bytes(ctypes.byref(h), int(B)))
@@ -570,6 +636,9 @@ class SparseLinear:
 
     def spmm(self, X, Y=None, stream=None):
         return spw_spmm(self.hdr, self.buf, X, Y, stream=stream)
+
+    def spmm_tokens(self, X, threshold=0.0, Y=None, ws=None, stream=None):
+        return spw_spmm_tokens(self.hdr, self.buf, X, threshold, Y, ws, stream=stream)
 
     def decompress(self, out=None, stream=None):
         return spw_decompress(self.hdr, self.buf, out, stream)

@@ -95,6 +95,13 @@ struct SpmmParams {
     uint32_t tmem_cols;
     uint32_t off_w, off_raw, off_rec, off_tptr, off_bar;  // dynamic smem offsets
     long long wait_limit;       // pipeline waits, in SM cycles (drains use the fixed limit)
+    // Token grouping (spw_spmm_tokens): X rows are in grouped order; token tile mt visits
+    // only the k-tiles set in tile_sig[mt * sig_words ..] and its row r is row perm[r] of
+    // Y.  Null tile_sig: every k-tile, rows in place.
+    const uint64_t* tile_sig;
+    const uint32_t* perm;
+    int sig_words;
+    uint32_t off_klist;         // dynamic smem: the visited k-tile count, then the list
 };
 
 // ------------------------------------------------------------------ tcgen05 helpers
@@ -329,14 +336,6 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     const int n0 = ntile * (PAIR ? 2 * kTileRows : kTileRows) + kTileRows * (int)rank;
     const int s0 = n0 / kStripRows;
     const int nk = p.n_ktiles;
-    const int k_begin = (int)((long long)kz * nk / parts);
-    const int k_end = (int)((long long)(kz + 1) * nk / parts);
-    // Every role walks the CTA's k-steps from a start rotated by the weight-row tile: the
-    // CTAs that share an X tile then read different k-columns of it at any moment instead
-    // of all hitting the same L2 lines together.
-    const int n_kc = k_end - k_begin;
-    const int k_rot = n_kc > 0 ? ntile % n_kc : 0;
-    auto kstep = [&](int i) { return k_begin + (i + k_rot < n_kc ? i + k_rot : i + k_rot - n_kc); };
     const int SX = p.sx, SR = p.sr;
 
     uint64_t* bars = (uint64_t*)(smem + p.off_bar);
@@ -354,6 +353,8 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     volatile uint32_t* last_flag = (volatile uint32_t*)(tmem_slot + 2);
     uint32_t* tptr = (uint32_t*)(smem + p.off_tptr);
+    volatile int* klist_n = (volatile int*)(smem + p.off_klist);
+    uint16_t* klist = (uint16_t*)(smem + p.off_klist + 16);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < SX; i++) {
@@ -381,6 +382,19 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         const int s = s0 + j;
         tptr[i] = (s < p.n_strips) ? __ldg(p.tileptr + (size_t)s * nk + kt) : 0u;
     }
+    if (p.tile_sig && warp == 2) {
+        // Token grouping: the k-tiles of this token tile's signature, ascending.
+        const uint64_t* ts = p.tile_sig + (size_t)mt * p.sig_words;
+        int count = 0;
+        for (int base = 0; base < nk; base += 32) {
+            const int kt = base + lane;
+            const bool on = kt < nk && ((__ldg(ts + (kt >> 6)) >> (kt & 63)) & 1ull);
+            const uint32_t b = __ballot_sync(0xffffffffu, on);
+            if (on) klist[count + __popc(b & lanemask_lt())] = (uint16_t)kt;
+            count += __popc(b);
+        }
+        if (lane == 0) *klist_n = count;
+    }
     if (warp == 1) {  // TMEM allocation (whole warp; in pair mode warp 1 of both CTAs)
         if constexpr (PAIR) {
             asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -407,6 +421,19 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         if constexpr (PAIR) asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer_abort), "r"(1) : "memory");
     };
     const uint32_t tmem = *tmem_slot;
+    // The k-tiles this CTA visits: its part of 0 .. nk-1, or of the token tile's list.
+    // Every role walks them from a start rotated by the weight-row tile: the CTAs that
+    // share an X tile then read different k-columns of it at any moment instead of all
+    // hitting the same L2 lines together.
+    const int n_list = p.tile_sig ? *klist_n : nk;
+    const int k_begin = (int)((long long)kz * n_list / parts);
+    const int k_end = (int)((long long)(kz + 1) * n_list / parts);
+    const int n_kc = k_end - k_begin;
+    const int k_rot = n_kc > 0 ? ntile % n_kc : 0;
+    auto kstep = [&](int i) {
+        const int j = k_begin + (i + k_rot < n_kc ? i + k_rot : i + k_rot - n_kc);
+        return p.tile_sig ? (int)klist[j] : j;
+    };
 
     int x_issued = 0, r_issued = 0;  // lane 0 of warp 0 (X) and of the TCB warp: stages armed
     if (warp == 0 || warp == kTcbWarp) {
@@ -685,7 +712,12 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             const int n_used = min(p.n_acc, (k_end - k_begin) * (kBK / 16));
             for (int j = part_of; j < (p.MT + 31) / 32; j += 4) {
                 uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + 32u * j, r);
+                if (n_kc > 0) {
+                    tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + 32u * j, r);
+                } else {  // no k-step (a token tile with an empty list): no MMA wrote TMEM
+#pragma unroll
+                    for (int c = 0; c < 32; c++) r[c] = 0u;
+                }
                 for (int a = 1; a < n_used; a++) {  // narrow tiles: add the other chains
                     uint32_t r2[32];
                     tmem_ld32(tmem + ((uint32_t)(32 * quarter) << 16) + 32u * (uint32_t)a, r2);
@@ -701,8 +733,10 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 #pragma unroll
                     for (int c = 0; c < 32; c++) {
                         const int m = m0 + 32 * j + c;
-                        if (c < lim && m < p.M)
-                            p.Y[(size_t)m * p.ldy + n] = __half_as_ushort(__float2half_rn(__uint_as_float(r[c])));
+                        if (c < lim && m < p.M) {
+                            const int ym = p.perm ? (int)__ldg(p.perm + m) : m;
+                            p.Y[(size_t)ym * p.ldy + n] = __half_as_ushort(__float2half_rn(__uint_as_float(r[c])));
+                        }
                     }
                 }
             }
@@ -766,11 +800,12 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     const int tok = (4 * i) / kTileRows, row = (4 * i) % kTileRows;
                     const int m = m0 + tok;
                     if (m >= p.M) continue;
+                    const int ym = p.perm ? (int)__ldg(p.perm + m) : m;
                     const float v[4] = {acc[u].x, acc[u].y, acc[u].z, acc[u].w};
 #pragma unroll
                     for (int e = 0; e < 4; e++)
                         if (n0 + row + e < p.N)
-                            p.Y[(size_t)m * p.ldy + n0 + row + e] = __half_as_ushort(__float2half_rn(v[e]));
+                            p.Y[(size_t)ym * p.ldy + n0 + row + e] = __half_as_ushort(__float2half_rn(v[e]));
                 }
             }
         }
@@ -831,7 +866,7 @@ struct SpmmPlan {
     bool pair;  // 256-row tiles on SM pairs (tcgen05 cta_group::2)
     int MT, nh, n_acc, m_tiles, n_tiles, ksplit, n_whole, sx, sr, sw, ctas_per_sm;
     uint32_t x_stage_bytes, val_slot, raw_stage_bytes, tmem_cols;
-    uint32_t off_w, off_raw, off_rec, off_tptr, off_bar;
+    uint32_t off_w, off_raw, off_rec, off_tptr, off_klist, off_bar;
     size_t smem;
     uint64_t ws_counters, ws_bytes;
     uint64_t ws_xt;  // decode with a rule: offset of x~ (B rows of K rounded up to 8)
@@ -880,11 +915,11 @@ int device_pair_slots() {
 // bound by shared-memory bandwidth (decoder traffic, X writes, MMA operand reads) rather
 // than by the L2 traffic of X that it halves.
 int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_count = 0,
-                   bool allow_pair = false) {
+                   bool allow_pair = false, bool tokens = false) {
     const int sms = sm_count > 0 ? sm_count : device_sm_count();
     if (sms <= 0) return SPW_ERR_CUDA;
     pl->pair = false;
-    if (allow_pair && !rule && M >= 256 && h->N > (uint32_t)kTileRows) {
+    if (allow_pair && !rule && !tokens && M >= 256 && h->N > (uint32_t)kTileRows) {
         const char* e = getenv("SPW_SPMM_PAIR");
         const bool env_on = e && e[0] == '1';
         const int pairs = env_on ? (sm_count > 0 ? sm_count / 2 : device_pair_slots()) : 0;
@@ -964,6 +999,8 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
     pl->val_slot = (uint32_t)round_up_u64(16ull * h->max_tile_units + 16, 16);
     pl->raw_stage_bytes = 1024u + (uint32_t)kTileStrips * pl->val_slot;
     const uint32_t tptr_bytes = (uint32_t)round_up_u64(4ull * kTileStrips * (h->n_ktiles + 1), 16);
+    // token grouping: the visited k-tile count (16 bytes) and list (2 bytes each)
+    const uint32_t klist_bytes = tokens ? 16u + (uint32_t)round_up_u64(2ull * h->n_ktiles, 16) : 0u;
     // {X, TCB, decoded-weight} stages, deepest first
     const int options[][3] = {{4, 4, 4}, {3, 4, 4}, {2, 4, 4}, {2, 4, 3}, {2, 3, 3},
                               {2, 3, 2}, {2, 2, 2}};
@@ -974,7 +1011,8 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
         const uint32_t off_raw = off_w + (uint32_t)sw * kWStageBytes;
         const uint32_t off_rec = off_raw + (uint32_t)sr * pl->raw_stage_bytes;
         const uint32_t off_tptr = off_rec + kRecBytesPerWarp * kDecoderWarps;
-        const uint32_t off_bar = (uint32_t)round_up_u64(off_tptr + tptr_bytes, 8);
+        const uint32_t off_klist = off_tptr + tptr_bytes;
+        const uint32_t off_bar = (uint32_t)round_up_u64(off_klist + klist_bytes, 8);
         const uint32_t bar_bytes = 8u * (2 * sx + 2 * sr + 2 * sw + 2 + kPeerSlots) + 16u;
         const size_t total = (size_t)off_bar + bar_bytes + 1024;  // + base alignment slack
         if (total <= (size_t)kSmemLimit) {
@@ -985,6 +1023,7 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
             pl->off_raw = off_raw;
             pl->off_rec = off_rec;
             pl->off_tptr = off_tptr;
+            pl->off_klist = off_klist;
             pl->off_bar = off_bar;
             pl->smem = total;
             found = true;
@@ -1010,12 +1049,16 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
 }
 
 // Shared by spw_spmm and spw_spmv_tc: checks, tensor map, launch.
+// Token grouping (tile_sig not null): X is the grouped input, perm and tile_sig as
+// group_tokens_launch wrote them for the plan's token tile.
 int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int M, int ldx,
                uint16_t* d_Y, int ldy, int rule, float t, const uint32_t* act_bits, void* d_ws,
-               uint64_t ws_bytes, cudaStream_t stream) {
+               uint64_t ws_bytes, cudaStream_t stream, const uint32_t* perm = nullptr,
+               const uint64_t* tile_sig = nullptr, int sig_words = 0) {
     const bool needs_rule = rule && (t > 0.0f || act_bits);
+    const bool tokens = tile_sig != nullptr;
     SpmmPlan pl;
-    int rc = make_spmm_plan(hdr, M, needs_rule, &pl, 0, !rule);
+    int rc = make_spmm_plan(hdr, M, needs_rule, &pl, 0, !rule && !tokens, tokens);
     if (rc != SPW_OK) return rc;
     if (pl.ws_bytes) {
         if (!d_ws) return SPW_ERR_INVALID_ARG;
@@ -1082,7 +1125,11 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
     prm.off_raw = pl.off_raw;
     prm.off_rec = pl.off_rec;
     prm.off_tptr = pl.off_tptr;
+    prm.off_klist = pl.off_klist;
     prm.off_bar = pl.off_bar;
+    prm.tile_sig = tile_sig;
+    prm.perm = perm;
+    prm.sig_words = sig_words;
     prm.wait_limit = wait_limit_cycles();
 
     static size_t attr_smem[2][kMaxDevices];
@@ -1164,6 +1211,86 @@ int spw_spmm(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int 
     if (!aligned16(d_buf) || !aligned16(d_X) || !aligned16(d_Y)) return SPW_ERR_ALIGNMENT;
     return tc_product(hdr, d_buf, d_X, M, ldx, d_Y, ldy, 0, 0.0f, nullptr, d_ws, ws_bytes,
                       (cudaStream_t)stream);
+}
+
+// Token grouping: workspace sections after the product's own (split-K) bytes.
+struct TokensLayout {
+    SpmmPlan pl;
+    int ldg, words;
+    uint64_t off_xg, off_perm, off_tsig, off_scratch, total;
+};
+
+static int tokens_layout(const spw_format* hdr, int M, int sm_count, TokensLayout* L) {
+    const int rc = make_spmm_plan(hdr, M, false, &L->pl, sm_count, false, true);
+    if (rc != SPW_OK) return rc;
+    const int K = (int)hdr->K;
+    L->ldg = (int)round_up_u64((uint64_t)K, 8);
+    L->words = token_sig_words(K);
+    L->off_xg = round_up_u64(L->pl.ws_bytes, 256);
+    L->off_perm = L->off_xg + round_up_u64(2ull * (uint64_t)M * L->ldg, 256);
+    L->off_tsig = L->off_perm + round_up_u64(4ull * (uint64_t)M, 256);
+    L->off_scratch = L->off_tsig + round_up_u64(8ull * (uint64_t)L->pl.m_tiles * L->words, 256);
+    L->total = L->off_scratch + token_groups_scratch_bytes(M, K);
+    return SPW_OK;
+}
+
+uint64_t spw_spmm_tokens_workspace_bytes(const spw_format* hdr, int M) {
+    if (check_header(hdr) != SPW_OK || M < 1 || M > kMaxGroupTokens || hdr->K > (uint32_t)kMaxTokenK)
+        return 0;
+    TokensLayout L;
+    if (tokens_layout(hdr, M, 0, &L) != SPW_OK) return 0;
+    return L.total;
+}
+
+int spw_spmm_tokens_plan(const spw_format* hdr, int M, int sm_count, spw_spmm_plan_info* out) {
+    if (!out || M < 1) return SPW_ERR_INVALID_ARG;
+    const int rc = check_header(hdr);
+    if (rc != SPW_OK) return rc;
+    if (M > kMaxGroupTokens || hdr->K > (uint32_t)kMaxTokenK) return SPW_ERR_UNSUPPORTED;
+    TokensLayout L;
+    const int prc = tokens_layout(hdr, M, sm_count, &L);
+    if (prc != SPW_OK) return prc;
+    const SpmmPlan& pl = L.pl;
+    const long long tiles = (long long)pl.m_tiles * pl.n_tiles;
+    out->token_tile = pl.MT;
+    out->token_tiles = pl.m_tiles;
+    out->weight_tiles = pl.n_tiles;
+    out->k_parts = pl.ksplit;
+    out->whole_tiles = pl.n_whole;
+    out->ctas = (int32_t)(pl.n_whole + (tiles - pl.n_whole) * pl.ksplit);
+    out->cta_pair = 0;
+    out->reserved = 0;
+    out->workspace_bytes = L.total;
+    return SPW_OK;
+}
+
+int spw_spmm_tokens(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int M, int ldx,
+                    float threshold, uint16_t* d_Y, int ldy, void* d_ws, uint64_t ws_bytes,
+                    void* stream) {
+    int rc = check_header(hdr);
+    if (rc != SPW_OK) return rc;
+    if (M < 0) return SPW_ERR_INVALID_ARG;
+    if (M == 0) return SPW_OK;
+    if (!d_buf || !d_X || !d_Y || !d_ws) return SPW_ERR_INVALID_ARG;
+    if (!(threshold >= 0.0f) || isinf(threshold)) return SPW_ERR_INVALID_ARG;
+    if (!ld_ok(ldx, (int)hdr->K, M) || ldy < (int)hdr->N) return SPW_ERR_INVALID_ARG;
+    if (!aligned16(d_buf) || !aligned16(d_X) || !aligned16(d_Y) || !aligned16(d_ws))
+        return SPW_ERR_ALIGNMENT;
+    if (M > kMaxGroupTokens || hdr->K > (uint32_t)kMaxTokenK) return SPW_ERR_UNSUPPORTED;
+    TokensLayout L;
+    rc = tokens_layout(hdr, M, 0, &L);
+    if (rc != SPW_OK) return rc;
+    if (ws_bytes < L.total) return SPW_ERR_BUFFER_TOO_SMALL;
+    uint8_t* ws = (uint8_t*)d_ws;
+    uint16_t* xg = (uint16_t*)(ws + L.off_xg);
+    uint32_t* perm = (uint32_t*)(ws + L.off_perm);
+    uint64_t* tsig = (uint64_t*)(ws + L.off_tsig);
+    cudaStream_t st = (cudaStream_t)stream;
+    rc = group_tokens_launch(d_X, M, (int)hdr->K, ldx, threshold, L.pl.MT, xg, L.ldg, perm, tsig,
+                             ws + L.off_scratch, st);
+    if (rc != SPW_OK) return rc;
+    return tc_product(hdr, d_buf, xg, M, L.ldg, d_Y, ldy, 0, 0.0f, nullptr, d_ws, L.pl.ws_bytes, st,
+                      perm, tsig, L.words);
 }
 
 uint64_t spw_spmv_tc_workspace_bytes(const spw_format* hdr, int B) {

@@ -281,6 +281,20 @@ long long wait_limit_cycles();
 // Decode column-fetch mode set by spw_set_column_fetch (0, 1 or 2).
 int column_fetch_mode();
 
+// Token grouping for prefill (tokens.cu): signatures of up to 4 words of k-tile bits.
+constexpr int kMaxTokenWords = 4;
+constexpr int kMaxTokenK = 64 * 64 * kMaxTokenWords;  // 16384 columns
+constexpr int kMaxGroupTokens = 16384;
+inline int token_sig_words(int K) { return ((K + 63) / 64 + 63) / 64; }
+// Scratch bytes (per-token signatures and rank counters) of group_tokens_launch.
+uint64_t token_groups_scratch_bytes(int M, int K);
+// Launches the three grouping kernels on stream: X (M x K at ldx) -> Xg (M x ldg, the
+// rule applied, rows in grouped order), perm[M] (row r of Xg is token perm[r]) and
+// tile_sig[ceil(M / T) * words] (k-tiles each token tile of T rows visits).
+int group_tokens_launch(const uint16_t* X, int M, int K, int ldx, float t, int T, uint16_t* Xg,
+                        int ldg, uint32_t* perm, uint64_t* tile_sig, void* scratch,
+                        cudaStream_t stream);
+
 }  // namespace spw
 
 #define SPW_CUDA_TRY(expr)                         \

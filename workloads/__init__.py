@@ -145,3 +145,30 @@ def decode_act(layer_name: str, B: int, K: int, act_sparsity: float, *seed_parts
         x = normal_act(B, K, layer_name, *seed_parts)
     zx, t = zero_smallest(x, act_sparsity)
     return zx, t
+
+
+def domain_tokens(M: int, K: int, n_domains: int, block_density: float, *seed_parts,
+                  silu: bool = False) -> tuple[np.ndarray, np.ndarray]:
+    """Prefill tokens drawn from n_domains "domains" whose channel use differs.
+
+    Each domain keeps a seeded random subset of the 64-column channel blocks (each block
+    with probability block_density, at least one block); every token belongs to one
+    domain (drawn uniformly, tokens interleaved in random order), takes N(0, 1) values --
+    SiLU(g) * u with g, u ~ N(0, 1) when silu is set -- and is zero in every block its
+    domain does not use.  Returns (fp16 M x K tokens, domain id per token)."""
+    r = rng("domains", M, K, n_domains, block_density, *seed_parts)
+    nk = -(-K // 64)
+    blocks = r.random((n_domains, nk)) < block_density
+    for d in range(n_domains):
+        if not blocks[d].any():
+            blocks[d, r.integers(nk)] = True
+    dom = r.integers(0, n_domains, size=M)
+    if silu:
+        g = r.standard_normal((M, K))
+        u = r.standard_normal((M, K))
+        x = g / (1.0 + np.exp(-g)) * u
+    else:
+        x = r.standard_normal((M, K))
+    cols = np.repeat(blocks, 64, axis=1)[:, :K]
+    x[~cols[dom]] = 0.0
+    return x.astype(np.float16), dom
