@@ -77,10 +77,11 @@ def _load():
         lib.orc_silu_mul.argtypes = [P, P, i, i, i, P]
         lib.orc_spmm_tokens.argtypes = [P, i, P, i, i, i, P, i, i, f, P, i, P]
         lib.orc_token_groups.argtypes = [P, i, i, i, f, i, P, P]
+        lib.orc_split24.argtypes = [P, i, i, i, P, P]
         for name in ("orc_tcb_query", "orc_tcb_encode", "orc_tcb_decode",
                      "orc_select_threshold", "orc_select_topk", "orc_spmv", "orc_spmm",
                      "orc_round_to_half", "orc_silu_mul", "orc_spmm_tokens",
-                     "orc_token_groups"):
+                     "orc_token_groups", "orc_split24"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -241,6 +242,18 @@ def token_groups(X: np.ndarray, t: float, token_tile: int) -> tuple[np.ndarray, 
     _check(_load().orc_token_groups(_ptr(Xb), M, K, K, ctypes.c_float(t), int(token_tile),
                                     _ptr(perm), _ptr(tile_sig)), "orc_token_groups")
     return perm, tile_sig
+
+
+def split24(mask: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """2:4 + residual split of a mask: (mask_s, mask_r), uint8 N x K each; in every
+    group of four columns of a row the first two kept weights go to mask_s, the rest to
+    mask_r."""
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    N, K = mask.shape
+    ms = np.zeros((N, K), np.uint8)
+    mr = np.zeros((N, K), np.uint8)
+    _check(_load().orc_split24(_ptr(mask), K, N, K, _ptr(ms), _ptr(mr)), "orc_split24")
+    return ms, mr
 
 
 def round_to_half(v: np.ndarray) -> np.ndarray:

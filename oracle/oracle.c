@@ -42,6 +42,7 @@
  *   orc_silu_mul         h = fp16(SiLU(g) * u) for the gated FFN    [RMM] §4.2, §3.2.
  *   orc_spmm_tokens      Y = X~ . W_masked^T, each token its own index set [RMM] §4.2, §6.1.
  *   orc_token_groups     token order and token-tile k-tile sets      [RMM] §6.1.
+ *   orc_split24          2:4 part and residual of a mask             [3LF] abstract, §1.
  *
  * Pins: tests/test_oracle_*.py check every function against things fixed outside this
  * file: numpy's binary16 decoder over all 65536 bit patterns, hand-derived TCB buffers
@@ -560,5 +561,37 @@ int orc_token_groups(const uint16_t* X, int M, int K, int ldx, float t, int T, u
         for (int w = 0; w < words; w++) tile_sig[(size_t)(r / T) * words + w] |= keys[r].sig[w];
     }
     free(keys);
+    return ORC_OK;
+}
+
+/* 2:4 + residual split ("Accelerating LLM GPU inference with moderately unstructured
+ * sparse weight matrices": abstract and §1, layers (i) and (iii) of its three-layer
+ * format -- a structured part for the sparse tensor cores and a residual that keeps the
+ * product exact; the related-work paragraph on SparTA describes the same two-way split).
+ * The pages do not say which kept weights of a group go to the structured part; this
+ * reading takes the first two in column order:
+ *   for every row n and every group of four columns 4g .. 4g+3 (the last group of a
+ *   ragged K is shorter), the kept weights (mask != 0) at the two lowest columns go to
+ *   the 2:4 part (mask_s), every further kept weight of the group to the residual
+ *   (mask_r).  mask_s and mask_r are disjoint and their union is mask. */
+int orc_split24(const uint8_t* mask, int ld_mask, int N, int K, uint8_t* mask_s,
+                uint8_t* mask_r) {
+    if (!mask || !mask_s || !mask_r || N < 0 || K < 0 || ld_mask < K) return ORC_ERR_ARG;
+    for (int n = 0; n < N; n++)
+        for (int g = 0; g < K; g += 4) {
+            int taken = 0;
+            for (int k = g; k < g + 4 && k < K; k++) {
+                size_t i = (size_t)n * K + k;
+                mask_s[i] = 0;
+                mask_r[i] = 0;
+                if (!mask[(size_t)n * ld_mask + k]) continue;
+                if (taken < 2) {
+                    mask_s[i] = 1;
+                    taken++;
+                } else {
+                    mask_r[i] = 1;
+                }
+            }
+        }
     return ORC_OK;
 }

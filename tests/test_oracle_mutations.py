@@ -26,6 +26,7 @@ PRODUCT_PINS = "products"
 HALF_PINS = "half"
 FFN_PINS = "ffn"
 TOKEN_PINS = "tokens"
+SPLIT_PINS = "split24"
 
 CHILD = {
     "half": "import test_oracle_half as H; H.test_all_half_patterns_match_numpy()",
@@ -56,6 +57,10 @@ CHILD = {
                "G.test_groups_equal_signatures_keep_index_order()\n"
                "G.test_groups_word_zero_decides_first_and_threshold_counts()\n"
                "[G.test_groups_match_vectorised_restatement(s) for s in range(12)]"),
+    "split24": ("import test_oracle_split24 as S\n"
+                "S.test_hand_example(); S.test_structured_mask_has_empty_residual()\n"
+                "S.test_partition_and_counts(33, 130, 0.5); S.test_partition_and_counts(64, 257, 0.7)\n"
+                "S.test_parts_sum_to_the_product()"),
 }
 
 MUTANTS = [
@@ -105,6 +110,11 @@ MUTANTS = [
     ("token_ktile_width", "int kt = k / 64;", "int kt = k / 32;", [TOKEN_PINS]),
     ("token_tile_shifted", "tile_sig[(size_t)(r / T) * words + w] |= keys[r].sig[w];",
      "tile_sig[(size_t)(((r + 1) % M) / T) * words + w] |= keys[r].sig[w];", [TOKEN_PINS]),
+    ("split_three_structured", "if (taken < 2) {", "if (taken < 3) {", [SPLIT_PINS]),
+    ("split_groups_of_two", "for (int k = g; k < g + 4 && k < K; k++) {",
+     "for (int k = g; k < g + 4 && k < K; k++) { if (k == g + 2) taken = 0;", [SPLIT_PINS]),
+    ("split_last_two_structured", "if (taken < 2) {",
+     "if (taken < 2 && !(k == g && mask[(size_t)n * ld_mask + k + (k + 1 < K)])) {", [SPLIT_PINS]),
 ]
 
 
