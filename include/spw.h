@@ -381,6 +381,49 @@ int spw_spmm_tokens(const spw_format* hdr, const void* d_buf, const uint16_t* d_
                     float threshold, uint16_t* d_Y, int ldy, void* d_ws, uint64_t ws_bytes,
                     void* stream);
 
+/* 2:4 + residual split ("Accelerating LLM GPU inference with moderately unstructured
+ * sparse weight matrices", abstract and §1: a 2:4 layer for the sparse tensor cores and a
+ * residual layer that keeps the SpMM exact; the pages' slot-filling middle layer is not
+ * built).  In every group of four columns 4g .. 4g+3 of a row, the first two kept
+ * weights (mask != 0, column order) form the 2:4 part; every further kept weight of the
+ * group is set in the residual mask d_mask_r (N x K u8 at ld_mask_r, written: 1 for a
+ * residual weight, 0 elsewhere), which the caller compresses into an ordinary TCB v1
+ * buffer (spw_format_query / spw_compress with the same W) for spw_spmm24.
+ * d_s24 (spw_s24_bytes(N, K) bytes, written) holds the 2:4 part per 64 x 64 tile t =
+ * strip * n_ktiles + k-tile:
+ *   values at t * 4096: row r's 32 halves -- for each group of four columns, the values
+ *     at its two selected positions, lower position first -- fill bytes 64 r .. 64 r +
+ *     63, the 16-byte chunk c (groups 4c .. 4c+3) at position c ^ ((r >> 1) & 3);
+ *   metadata at n_tiles * 4096 + t * 512: for each half j of the tile's columns, 64
+ *     32-bit words; word L holds row 16 (L/16) + L%8 in bits 0-15 and that row + 8 in
+ *     bits 16-31, for columns 32 j + 16 ((L/8) % 2) .. +15 as four 4-bit groups (group g
+ *     at bits 4g of the half: the first selected position in bits 0-1, the second in
+ *     bits 2-3, first < second).
+ * A group with fewer than two kept weights selects the lowest free positions with value
+ * 0; rows past N and columns past K keep nothing.  W: N x K fp16 at ldw; mask: N x K u8
+ * at ld_mask.  Asynchronous.  Errors: INVALID_ARG, ALIGNMENT (d_s24), BUFFER_TOO_SMALL,
+ * UNSUPPORTED (too many tiles), CUDA. */
+uint64_t spw_s24_bytes(int N, int K);
+int spw_split24(const uint16_t* d_W, int ldw, const uint8_t* d_mask, int ld_mask, int N, int K,
+                void* d_s24, uint64_t s24_bytes, uint8_t* d_mask_r, int ld_mask_r, void* stream);
+
+/* Workspace bytes and launch plan of spw_spmm24 (as spw_spmm's, with at most 256 tokens
+ * per tile and no SM-pair tiles); hdr_r is the residual's TCB header. */
+uint64_t spw_spmm24_workspace_bytes(const spw_format* hdr_r, int M);
+int spw_spmm24_plan(const spw_format* hdr_r, int M, int sm_count, spw_spmm_plan_info* out);
+
+/* Prefill on the 2:4 + residual split ([3LF] layers (i) and (iii)):
+ *   Y[m,n] = sum_k X[m,k] (S[n,k] + R[n,k]),  S + R = W masked (spw_split24),
+ * where S (d_s24) runs on the sparse tensor cores (tcgen05.mma.sp, K = 32 per
+ * instruction, metadata in tensor memory) and R (hdr_r / d_buf_r, a TCB v1 buffer of the
+ * residual) is decoded in shared memory and runs as dense MMA into the same fp32
+ * accumulator; a k-tile whose residual tiles are empty costs no decode and no dense MMA.
+ * X, Y, M, ldx, ldy, workspace, determinism and errors as spw_spmm; d_s24 must hold
+ * spw_s24_bytes(N, K) bytes (BUFFER_TOO_SMALL otherwise) and be 16-byte aligned. */
+int spw_spmm24(const spw_format* hdr_r, const void* d_buf_r, const void* d_s24, uint64_t s24_bytes,
+               const uint16_t* d_X, int M, int ldx, uint16_t* d_Y, int ldy, void* d_ws,
+               uint64_t ws_bytes, void* stream);
+
 /* Workspace bytes spw_spmv_tc needs (the rules of spw_spmm_workspace_bytes with M = B);
  * 0 for B outside 1..16. */
 uint64_t spw_spmv_tc_workspace_bytes(const spw_format* hdr, int B);

@@ -89,6 +89,11 @@ SIGNATURES = {
     "spw_spmm_tokens_workspace_bytes": ([_FP, _I], _U64),
     "spw_spmm_tokens_plan": ([_FP, _I, _I, ctypes.POINTER(spw_spmm_plan_info)], _I),
     "spw_spmm_tokens": ([_FP, _P, _P, _I, _I, _F, _P, _I, _P, _U64, _P], _I),
+    "spw_s24_bytes": ([_I, _I], _U64),
+    "spw_split24": ([_P, _I, _P, _I, _I, _I, _P, _U64, _P, _I, _P], _I),
+    "spw_spmm24_workspace_bytes": ([_FP, _I], _U64),
+    "spw_spmm24_plan": ([_FP, _I, _I, ctypes.POINTER(spw_spmm_plan_info)], _I),
+    "spw_spmm24": ([_FP, _P, _P, _U64, _P, _I, _I, _P, _I, _P, _U64, _P], _I),
 }
 
 
@@ -612,6 +617,70 @@ class DecodeGroup:
             self.n, self._harr, self._pbufs, self._px, self._ldx, ab, self._py, self._ldy,
             self.B, float(threshold), _ptr(self.ws), self.ws.numel(), _stream(stream)))
         return ys
+
+
+def spw_s24_bytes(N: int, K: int) -> int:
+    return int(lib().spw_s24_bytes(int(N), int(K)))
+
+
+def spw_split24(W: torch.Tensor, mask: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """2:4 + residual split: (s24 uint8 buffer of the 2:4 part, residual mask uint8 N x K);
+    see spw_split24 in include/spw.h."""
+    W2, ldw = _rows(_half(W, "W"), "W")
+    m2, ldm = _rows(mask, "mask")
+    if m2.dtype != torch.uint8:
+        raise ValueError("mask must be uint8")
+    N, K = W2.shape
+    s24 = torch.empty(spw_s24_bytes(N, K), dtype=torch.uint8, device=W.device)
+    mask_r = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    _check("spw_split24", lib().spw_split24(_ptr(W2), ldw, _ptr(m2), ldm, N, K, _ptr(s24), s24.numel(),
+                                            _ptr(mask_r), K, _stream(stream)))
+    return s24, mask_r
+
+
+def spw_spmm24_workspace_bytes(hdr_r, M: int) -> int:
+    return int(lib().spw_spmm24_workspace_bytes(ctypes.byref(_hdr(hdr_r)), int(M)))
+
+
+def spw_spmm24_plan(hdr_r, M: int, sm_count: int = 0) -> dict:
+    info = spw_spmm_plan_info()
+    _check("spw_spmm24_plan", lib().spw_spmm24_plan(ctypes.byref(_hdr(hdr_r)), int(M), int(sm_count),
+                                                    ctypes.byref(info)))
+    return {name: getattr(info, name) for name, _ in info._fields_}
+
+
+def spw_spmm24(hdr_r, buf_r: torch.Tensor, s24: torch.Tensor, X: torch.Tensor,
+               Y: torch.Tensor | None = None, ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Prefill on the 2:4 + residual split: Y = X . (S + R)^T, S on sparse tensor cores."""
+    h = _hdr(hdr_r)
+    X2, ldx = _rows(_half(X, "X"), "X")
+    M = X2.shape[0]
+    if Y is None:
+        Y = torch.empty((M, h.N), dtype=torch.float16, device=X.device)
+    Y2, ldy = _rows(_half(Y, "Y"), "Y")
+    _need_buf(buf_r, h, "buf_r")
+    _need(X2, M, h.K, "X")
+    _need(Y2, M, h.N, "Y")
+    need = spw_spmm24_workspace_bytes(h, M)
+    if ws is None and need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=X.device)
+    _check("spw_spmm24", lib().spw_spmm24(
+        ctypes.byref(h), _ptr(buf_r), _ptr(s24), s24.numel(), _ptr(X2), M, ldx, _ptr(Y2), ldy,
+        _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return Y
+
+
+class SparseLinear24:
+    """A weight held as its 2:4 part (sparse tensor cores) plus a TCB residual: a holder
+    for spw_split24, spw_compress and spw_spmm24 (it adds no arithmetic)."""
+
+    def __init__(self, W: torch.Tensor, mask: torch.Tensor, stream=None):
+        self.N, self.K = W.shape
+        self.s24, self.mask_r = spw_split24(W, mask, stream)
+        self.buf_r, self.hdr_r = spw_compress(W, self.mask_r, stream=stream)
+
+    def spmm(self, X, Y=None, ws=None, stream=None):
+        return spw_spmm24(self.hdr_r, self.buf_r, self.s24, X, Y, ws, stream)
 
 
 class SparseLinear:

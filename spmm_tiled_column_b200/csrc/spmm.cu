@@ -71,6 +71,12 @@ constexpr int kTcbWarp = 2 + kDecoderWarps;             // the TCB producer's wa
 constexpr int kThreads = 32 * (3 + kDecoderWarps);      // X producer, MMA, decoders, TCB producer
 constexpr uint32_t kWStageBytes = kTileRows * kBK * 2;  // 16 KB
 constexpr int kSmemLimit = 227 * 1024;
+// 2:4 mode (spw_spmm24): per k-step S stage = the 2:4 values of both strips (2 x 4 KB, the
+// 64-byte-swizzled K-major layout of split24.cu) and their metadata (2 x 512 bytes).
+constexpr uint32_t kS24ValBytes = 4096;
+constexpr uint32_t kS24MetaBytes = 512;
+constexpr uint32_t kSStageBytes = kTileStrips * (kS24ValBytes + kS24MetaBytes);  // 9 KB
+constexpr int kMaxTokens24 = 256;  // accumulators <= 256 columns: the metadata slots fit
 
 struct SpmmParams {
     const uint64_t* bitmaps;
@@ -102,6 +108,13 @@ struct SpmmParams {
     const uint32_t* perm;
     int sig_words;
     uint32_t off_klist;         // dynamic smem: the visited k-tile count, then the list
+    // 2:4 + residual (spw_spmm24): the structured part (split24.cu layout); the TCB
+    // sections above then describe the residual.  ss S stages at off_s; the metadata of
+    // W stage w sits in tensor-memory columns e_col + 2 w and e_col + 2 w + 1.
+    const uint8_t* s24_vals;
+    const uint8_t* s24_meta;
+    int ss;
+    uint32_t off_s, e_col;
 };
 
 // ------------------------------------------------------------------ tcgen05 helpers
@@ -118,6 +131,37 @@ __device__ inline uint64_t umma_desc_sw128(uint32_t saddr) {
 }
 
 // kind::f16 instruction descriptor: fp32 accumulator, fp16 A and B, both K-major.
+// K-major, 64-byte swizzle: 8-row atoms of 512 bytes (the 2:4 values, 64 bytes per row).
+__device__ inline uint64_t umma_desc_sw64(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)(16 >> 4) << 16;
+    d |= (uint64_t)(512 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)4 << 61;
+    return d;
+}
+
+// Sparse MMA (2:4 A): A holds two of every four K positions (16 halves per row for K =
+// 32), the metadata selecting them sits in tensor memory at e_tmem (an even column;
+// idesc bits 0-1 pick the column pair's half), idesc bit 2 marks the MMA sparse.
+__device__ inline void umma_f16_sp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                   uint32_t e_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%5], %3, {%6, %6, %6, %6}, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(e_tmem), "r"(0u)
+        : "memory");
+}
+
+// Two 32-bit columns of this warp's 32 tensor-memory lanes (one value per thread each).
+__device__ inline void tmem_st2(uint32_t taddr, uint32_t v0, uint32_t v1) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(v0), "r"(v1)
+                 : "memory");
+}
+__device__ inline void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
     return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
@@ -313,7 +357,7 @@ __global__ void __launch_bounds__(256) rule_kernel(const uint16_t* __restrict__ 
 // CTA's MMA warp relays "my X and W stages are ready" to rank 0 with a cluster-scope
 // arrive; rank 0's commits release the stages in both CTAs.  Per output element the X
 // tile crosses L2 half as often as with one CTA per 128-row tile.
-template <bool PAIR>
+template <bool PAIR, bool SP24 = false>
 __global__ void __launch_bounds__(kThreads, 1)
 spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ SpmmParams p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -349,7 +393,10 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     uint64_t* acc_full = w_empty + SW;
     uint64_t* drain = acc_full + 1;
     uint64_t* peer_ready = drain + 1;  // PAIR, on rank 0: the other CTA's stages are ready
-    uint32_t* tmem_slot = (uint32_t*)(peer_ready + kPeerSlots);
+    const int SS = SP24 ? p.ss : 0;
+    uint64_t* s_full = peer_ready + kPeerSlots;  // 2:4 mode: the S ring
+    uint64_t* s_empty = s_full + SS;
+    uint32_t* tmem_slot = (uint32_t*)(s_empty + SS);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     volatile uint32_t* last_flag = (volatile uint32_t*)(tmem_slot + 2);
     uint32_t* tptr = (uint32_t*)(smem + p.off_tptr);
@@ -372,6 +419,10 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         mbar_init(smem_u32(acc_full), 1);
         mbar_init(smem_u32(drain), 1);
         for (int i = 0; i < kPeerSlots; i++) mbar_init(smem_u32(&peer_ready[i]), 1);
+        for (int i = 0; i < SS; i++) {
+            mbar_init(smem_u32(&s_full[i]), 1);
+            mbar_init(smem_u32(&s_empty[i]), 1);
+        }
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
@@ -434,8 +485,16 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         const int j = k_begin + (i + k_rot < n_kc ? i + k_rot : i + k_rot - n_kc);
         return p.tile_sig ? (int)klist[j] : j;
     };
+    // 2:4 mode: k-tile kt holds no residual weight in either strip (no decode, no dense MMA)
+    auto residual_empty = [&](int kt) {
+        bool e = true;
+#pragma unroll
+        for (int q = 0; q < kTileStrips; q++)
+            if (s0 + q < p.n_strips && tptr[q * (nk + 1) + kt + 1] != tptr[q * (nk + 1) + kt]) e = false;
+        return e;
+    };
 
-    int x_issued = 0, r_issued = 0;  // lane 0 of warp 0 (X) and of the TCB warp: stages armed
+    int x_issued = 0, r_issued = 0, s_issued = 0;  // producers' lane 0: stages armed
     if (warp == 0 || warp == kTcbWarp) {
         // ------------------------------------------------------------ producer
         if (warp == 0 && lane == 0) {  // X ring
@@ -497,6 +556,28 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 }
                 r_issued++;
                 if (++rs == SR) { rs = 0; rph ^= 1u; }
+                if constexpr (SP24) {  // the 2:4 values and metadata of both strips
+                    const int ss_ = i % SS;
+                    if (i >= SS && !wait_or_abort(smem_u32(&s_empty[ss_]), (uint32_t)(((i / SS) - 1) & 1),
+                                                  abort_flag, p.wait_limit)) {
+                        abort_both();
+                        break;
+                    }
+                    const uint32_t sbar = smem_u32(&s_full[ss_]);
+                    const uint32_t sst = sbase + p.off_s + (uint32_t)ss_ * kSStageBytes;
+                    uint32_t sbytes = 0;
+                    for (int j = 0; j < kTileStrips; j++)
+                        if (s0 + j < p.n_strips) sbytes += kS24ValBytes + kS24MetaBytes;
+                    mbar_arrive_expect_tx(sbar, sbytes);
+                    for (int j = 0; j < kTileStrips; j++) {
+                        if (s0 + j >= p.n_strips) continue;
+                        const size_t t = (size_t)(s0 + j) * nk + kt;
+                        bulk_g2s(sst + kS24ValBytes * j, p.s24_vals + t * kS24ValBytes, kS24ValBytes, sbar);
+                        bulk_g2s(sst + kTileStrips * kS24ValBytes + kS24MetaBytes * j,
+                                 p.s24_meta + t * kS24MetaBytes, kS24MetaBytes, sbar);
+                    }
+                    s_issued++;
+                }
             }
         }
     } else if (warp == 1 && (!PAIR || rank == 0)) {
@@ -516,6 +597,10 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                                       wait_or_abort_cluster(smem_u32(&peer_ready[i % kPeerSlots]),
                                                             (uint32_t)((i / kPeerSlots) & 1), abort_flag,
                                                             p.wait_limit));
+            if constexpr (SP24)
+                ok = ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&s_full[i % SS]),
+                                                                 (uint32_t)((i / SS) & 1), abort_flag,
+                                                                 p.wait_limit));
             if (!ok) {
                 if (lane == 0) abort_both();
                 break;
@@ -524,12 +609,30 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 tc_fence_after();
                 const uint32_t xa = sbase + (uint32_t)xs * p.x_stage_bytes;
                 const uint32_t wa = sbase + p.off_w + (uint32_t)ws * kWStageBytes;
+                bool dense = true;  // the decoded W stage takes part (always, except 2:4 mode)
+                if constexpr (SP24) {
+                    // Two sparse MMAs (K = 32 each: 16 stored halves = 32 bytes of the S
+                    // stage's rows, 64 bytes of X's), then the residual's dense MMAs when
+                    // the k-tile holds any residual weight.
+                    const uint32_t sa = sbase + p.off_s + (uint32_t)(i % SS) * kSStageBytes;
+                    const uint32_t idesc_sp = idesc | (1u << 2);
+#pragma unroll
+                    for (int j = 0; j < 2; j++) {
+                        const uint64_t adesc = umma_desc_sw64(sa + 32u * j);
+                        const uint64_t bdesc = umma_desc_sw128(xa + 64u * j);
+                        umma_f16_sp(tmem, adesc, bdesc, idesc_sp | (uint32_t)j, tmem + p.e_col + 2u * ws,
+                                    (i > 0 || j > 0) ? 1u : 0u);
+                    }
+                    dense = !residual_empty(kstep(i));
+                }
 #pragma unroll
                 for (int j = 0; j < kBK / 16; j++) {
+                    if (!dense) break;
                     const uint64_t adesc = umma_desc_sw128(wa + 32u * j);
                     const int slice = i * (kBK / 16) + j;
                     const uint32_t acc = p.n_acc > 1 ? 32u * (uint32_t)(slice % p.n_acc) : 0u;
-                    const uint32_t first = p.n_acc > 1 ? (uint32_t)(slice < p.n_acc) : (uint32_t)(slice == 0);
+                    const uint32_t first = SP24 ? 0u
+                                                : p.n_acc > 1 ? (uint32_t)(slice < p.n_acc) : (uint32_t)(slice == 0);
                     for (int h = 0; h < p.nh; h++) {
                         const uint64_t bdesc = umma_desc_sw128(xa + brows * 128u * h + 32u * j);
                         if constexpr (PAIR)
@@ -544,6 +647,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 } else {
                     umma_commit(smem_u32(&x_empty[xs]));
                     umma_commit(smem_u32(&w_empty[ws]));
+                    if constexpr (SP24) umma_commit(smem_u32(&s_empty[i % SS]));
                 }
             }
             __syncwarp();
@@ -661,7 +765,33 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 break;
             }
             unsigned char* wst = smem + p.off_w + (uint32_t)ws * kWStageBytes;
-            {  // 8 columns -> one 16-byte chunk per row
+            // 2:4 mode: a k-tile without residual weights needs no dense W stage (the MMA
+            // warp skips its dense MMAs); decoder warps 0-3 (one per tensor-memory lane
+            // quarter) move the k-step's metadata into the W stage's two metadata columns.
+            const bool skip = SP24 && residual_empty(kstep(i));
+            if constexpr (SP24) {
+                if (d < 4) {
+                    if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&s_full[i % SS]), (uint32_t)((i / SS) & 1),
+                                                               abort_flag, p.wait_limit))) {
+                        abort_both();
+                        break;
+                    }
+                    const int quarter = warp & 3;
+                    const int gl = 32 * quarter + lane;  // tensor-memory lane = row block lane
+                    const int sq = gl >> 6, L = gl & 63;
+                    uint32_t m0 = 0x44444444u, m1 = 0x44444444u;  // rows past N: {0, 1} groups
+                    if (s0 + sq < p.n_strips) {
+                        const uint32_t* mw = (const uint32_t*)(smem + p.off_s + (size_t)(i % SS) * kSStageBytes +
+                                                               kTileStrips * kS24ValBytes + kS24MetaBytes * sq);
+                        m0 = mw[L];
+                        m1 = mw[64 + L];
+                    }
+                    tmem_st2(tmem + ((uint32_t)(32 * quarter) << 16) + p.e_col + 2u * (uint32_t)ws, m0, m1);
+                    tmem_st_wait();
+                    tc_fence_before();
+                }
+            }
+            if (!skip) {  // 8 columns -> one 16-byte chunk per row
                 uint32_t o0[4] = {0u, 0u, 0u, 0u}, o1[4] = {0u, 0u, 0u, 0u};
                 if (dec) {
 #pragma unroll
@@ -822,6 +952,11 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             const int last = i + ((r_issued - 1 - i) / SR) * SR;
             (void)mbar_drain(smem_u32(&r_full[i]), (uint32_t)((last / SR) & 1));
         }
+        if constexpr (SP24)
+            for (int i = 0; warp == kTcbWarp && lane == 0 && i < SS && i < s_issued; i++) {
+                const int last = i + ((s_issued - 1 - i) / SS) * SS;
+                (void)mbar_drain(smem_u32(&s_full[i]), (uint32_t)((last / SS) & 1));
+            }
     }
     __syncthreads();
     // Pair mode: rank 0's MMAs read both CTAs' shared memory and write both tensor
@@ -864,6 +999,9 @@ int get_encoder() {
 
 struct SpmmPlan {
     bool pair;  // 256-row tiles on SM pairs (tcgen05 cta_group::2)
+    bool sp24;  // 2:4 + residual: S stages, metadata columns, at most 256 tokens per tile
+    int ss;
+    uint32_t off_s, e_col;
     int MT, nh, n_acc, m_tiles, n_tiles, ksplit, n_whole, sx, sr, sw, ctas_per_sm;
     uint32_t x_stage_bytes, val_slot, raw_stage_bytes, tmem_cols;
     uint32_t off_w, off_raw, off_rec, off_tptr, off_klist, off_bar;
@@ -915,11 +1053,15 @@ int device_pair_slots() {
 // bound by shared-memory bandwidth (decoder traffic, X writes, MMA operand reads) rather
 // than by the L2 traffic of X that it halves.
 int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_count = 0,
-                   bool allow_pair = false, bool tokens = false) {
+                   bool allow_pair = false, bool tokens = false, bool sp24 = false) {
     const int sms = sm_count > 0 ? sm_count : device_sm_count();
     if (sms <= 0) return SPW_ERR_CUDA;
     pl->pair = false;
-    if (allow_pair && !rule && !tokens && M >= 256 && h->N > (uint32_t)kTileRows) {
+    pl->sp24 = sp24;
+    pl->ss = 0;
+    pl->off_s = 0;
+    pl->e_col = 0;
+    if (allow_pair && !rule && !tokens && !sp24 && M >= 256 && h->N > (uint32_t)kTileRows) {
         const char* e = getenv("SPW_SPMM_PAIR");
         const bool env_on = e && e[0] == '1';
         const int pairs = env_on ? (sm_count > 0 ? sm_count / 2 : device_pair_slots()) : 0;
@@ -938,9 +1080,10 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
     const long long nk_all = h->n_ktiles;
     const long long kcap = nk_all / 2 > 0 ? (nk_all / 2 < 16 ? nk_all / 2 : 16) : 1;
     double best = 1e300;
-    int best_mt_max = kMaxTokens, best_ks = 1;
+    const int tok_cap = sp24 ? kMaxTokens24 : kMaxTokens;
+    int best_mt_max = tok_cap, best_ks = 1;
     long long best_whole = -1;  // -1: every tile in best_ks parts (or whole when best_ks == 1)
-    for (int tok_max = kMaxTokens; tok_max >= 128; tok_max /= 2) {
+    for (int tok_max = tok_cap; tok_max >= 128; tok_max /= 2) {
         const int mt = (M + tok_max - 1) / tok_max;
         const int per_t = (M + mt - 1) / mt;
         const int nh_t = per_t > 256 ? 2 : 1;
@@ -992,33 +1135,44 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
     pl->nh = per > 256 ? 2 : 1;
     pl->MT = (int)round_up_u64((uint64_t)per, 16u * pl->nh);  // each MMA's N a multiple of 16
     pl->x_stage_bytes = (uint32_t)pl->MT * (pl->pair ? 64u : 128u);  // this CTA's share of X
-    pl->n_acc = pl->MT <= 32 ? 4 : 1;
+    pl->n_acc = (pl->MT <= 32 && !sp24) ? 4 : 1;
     uint32_t cols = 32;
     while (cols < (uint32_t)(pl->n_acc > 1 ? 32 * pl->n_acc : pl->MT)) cols <<= 1;
     pl->tmem_cols = cols;
+    if (sp24) {  // accumulators in columns 0 .. MT-1 (MT <= 256), metadata from column 256
+        pl->tmem_cols = 512;
+        pl->e_col = 256;
+    }
     pl->val_slot = (uint32_t)round_up_u64(16ull * h->max_tile_units + 16, 16);
     pl->raw_stage_bytes = 1024u + (uint32_t)kTileStrips * pl->val_slot;
     const uint32_t tptr_bytes = (uint32_t)round_up_u64(4ull * kTileStrips * (h->n_ktiles + 1), 16);
     // token grouping: the visited k-tile count (16 bytes) and list (2 bytes each)
     const uint32_t klist_bytes = tokens ? 16u + (uint32_t)round_up_u64(2ull * h->n_ktiles, 16) : 0u;
-    // {X, TCB, decoded-weight} stages, deepest first
-    const int options[][3] = {{4, 4, 4}, {3, 4, 4}, {2, 4, 4}, {2, 4, 3}, {2, 3, 3},
-                              {2, 3, 2}, {2, 2, 2}};
+    // {X, TCB, decoded-weight, 2:4} stages, deepest first
+    const int options[][4] = {{4, 4, 4, 0}, {3, 4, 4, 0}, {2, 4, 4, 0}, {2, 4, 3, 0}, {2, 3, 3, 0},
+                              {2, 3, 2, 0}, {2, 2, 2, 0}};
+    const int options24[][4] = {{4, 3, 3, 3}, {3, 3, 3, 3}, {3, 2, 3, 3}, {2, 3, 3, 3}, {2, 2, 2, 2}};
     bool found = false;
-    for (const auto& o : options) {
-        const int sx = o[0], sr = o[1], sw = o[2];
+    const int n_opt = sp24 ? (int)(sizeof(options24) / sizeof(options24[0]))
+                           : (int)(sizeof(options) / sizeof(options[0]));
+    for (int oi = 0; oi < n_opt; oi++) {
+        const int* o = sp24 ? options24[oi] : options[oi];
+        const int sx = o[0], sr = o[1], sw = o[2], ss = o[3];
         const uint32_t off_w = (uint32_t)sx * pl->x_stage_bytes;
-        const uint32_t off_raw = off_w + (uint32_t)sw * kWStageBytes;
+        const uint32_t off_s = off_w + (uint32_t)sw * kWStageBytes;  // 1024-byte aligned
+        const uint32_t off_raw = off_s + (uint32_t)ss * kSStageBytes;
         const uint32_t off_rec = off_raw + (uint32_t)sr * pl->raw_stage_bytes;
         const uint32_t off_tptr = off_rec + kRecBytesPerWarp * kDecoderWarps;
         const uint32_t off_klist = off_tptr + tptr_bytes;
         const uint32_t off_bar = (uint32_t)round_up_u64(off_klist + klist_bytes, 8);
-        const uint32_t bar_bytes = 8u * (2 * sx + 2 * sr + 2 * sw + 2 + kPeerSlots) + 16u;
+        const uint32_t bar_bytes = 8u * (2 * sx + 2 * sr + 2 * sw + 2 + kPeerSlots + 2 * ss) + 16u;
         const size_t total = (size_t)off_bar + bar_bytes + 1024;  // + base alignment slack
         if (total <= (size_t)kSmemLimit) {
             pl->sx = sx;
             pl->sr = sr;
             pl->sw = sw;
+            pl->ss = ss;
+            pl->off_s = off_s;
             pl->off_w = off_w;
             pl->off_raw = off_raw;
             pl->off_rec = off_rec;
@@ -1054,11 +1208,12 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
 int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, int M, int ldx,
                uint16_t* d_Y, int ldy, int rule, float t, const uint32_t* act_bits, void* d_ws,
                uint64_t ws_bytes, cudaStream_t stream, const uint32_t* perm = nullptr,
-               const uint64_t* tile_sig = nullptr, int sig_words = 0) {
+               const uint64_t* tile_sig = nullptr, int sig_words = 0, const uint8_t* s24 = nullptr) {
     const bool needs_rule = rule && (t > 0.0f || act_bits);
     const bool tokens = tile_sig != nullptr;
+    const bool sp24 = s24 != nullptr;
     SpmmPlan pl;
-    int rc = make_spmm_plan(hdr, M, needs_rule, &pl, 0, !rule && !tokens, tokens);
+    int rc = make_spmm_plan(hdr, M, needs_rule, &pl, 0, !rule && !tokens && !sp24, tokens, sp24);
     if (rc != SPW_OK) return rc;
     if (pl.ws_bytes) {
         if (!d_ws) return SPW_ERR_INVALID_ARG;
@@ -1130,16 +1285,26 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
     prm.tile_sig = tile_sig;
     prm.perm = perm;
     prm.sig_words = sig_words;
+    if (sp24) {
+        const uint64_t n_tiles = (uint64_t)hdr->n_strips * hdr->n_ktiles;
+        prm.s24_vals = s24;
+        prm.s24_meta = s24 + n_tiles * kS24ValBytes;
+        prm.ss = pl.ss;
+        prm.off_s = pl.off_s;
+        prm.e_col = pl.e_col;
+    }
     prm.wait_limit = wait_limit_cycles();
 
-    static size_t attr_smem[2][kMaxDevices];
+    static size_t attr_smem[3][kMaxDevices];
     int dev = 0;
     SPW_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= kMaxDevices) return SPW_ERR_CUDA;
-    if (attr_smem[pl.pair][dev] < pl.smem) {
-        SPW_CUDA_TRY(cudaFuncSetAttribute(pl.pair ? spmm_kernel<true> : spmm_kernel<false>,
+    const int variant = pl.pair ? 1 : sp24 ? 2 : 0;
+    if (attr_smem[variant][dev] < pl.smem) {
+        SPW_CUDA_TRY(cudaFuncSetAttribute(pl.pair ? spmm_kernel<true>
+                                                  : sp24 ? spmm_kernel<false, true> : spmm_kernel<false>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem));
-        attr_smem[pl.pair][dev] = pl.smem;
+        attr_smem[variant][dev] = pl.smem;
     }
     const long long tiles = (long long)pl.m_tiles * pl.n_tiles;
     const long long slots = pl.n_whole + (tiles - pl.n_whole) * pl.ksplit;  // tiles or parts
@@ -1159,6 +1324,8 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         SPW_CUDA_TRY(cudaLaunchKernelEx(&cfg, spmm_kernel<true>, tmap, prm));
+    } else if (sp24) {
+        spmm_kernel<false, true><<<dim3((unsigned)ctas), kThreads, pl.smem, stream>>>(tmap, prm);
     } else {
         spmm_kernel<false><<<dim3((unsigned)ctas), kThreads, pl.smem, stream>>>(tmap, prm);
     }
@@ -1291,6 +1458,50 @@ int spw_spmm_tokens(const spw_format* hdr, const void* d_buf, const uint16_t* d_
     if (rc != SPW_OK) return rc;
     return tc_product(hdr, d_buf, xg, M, L.ldg, d_Y, ldy, 0, 0.0f, nullptr, d_ws, L.pl.ws_bytes, st,
                       perm, tsig, L.words);
+}
+
+uint64_t spw_spmm24_workspace_bytes(const spw_format* hdr_r, int M) {
+    if (check_header(hdr_r) != SPW_OK || M < 1) return 0;
+    SpmmPlan pl;
+    if (make_spmm_plan(hdr_r, M, false, &pl, 0, false, false, true) != SPW_OK) return 0;
+    return pl.ws_bytes;
+}
+
+int spw_spmm24_plan(const spw_format* hdr_r, int M, int sm_count, spw_spmm_plan_info* out) {
+    if (!out || M < 1) return SPW_ERR_INVALID_ARG;
+    const int rc = check_header(hdr_r);
+    if (rc != SPW_OK) return rc;
+    SpmmPlan pl;
+    const int prc = make_spmm_plan(hdr_r, M, false, &pl, sm_count, false, false, true);
+    if (prc != SPW_OK) return prc;
+    const long long tiles = (long long)pl.m_tiles * pl.n_tiles;
+    out->token_tile = pl.MT;
+    out->token_tiles = pl.m_tiles;
+    out->weight_tiles = pl.n_tiles;
+    out->k_parts = pl.ksplit;
+    out->whole_tiles = pl.n_whole;
+    out->ctas = (int32_t)(pl.n_whole + (tiles - pl.n_whole) * pl.ksplit);
+    out->cta_pair = 0;
+    out->reserved = 0;
+    out->workspace_bytes = pl.ws_bytes;
+    return SPW_OK;
+}
+
+int spw_spmm24(const spw_format* hdr_r, const void* d_buf_r, const void* d_s24, uint64_t s24_bytes,
+               const uint16_t* d_X, int M, int ldx, uint16_t* d_Y, int ldy, void* d_ws,
+               uint64_t ws_bytes, void* stream) {
+    int rc = check_header(hdr_r);
+    if (rc != SPW_OK) return rc;
+    if (M < 0) return SPW_ERR_INVALID_ARG;
+    if (M == 0) return SPW_OK;
+    if (!d_buf_r || !d_s24 || !d_X || !d_Y) return SPW_ERR_INVALID_ARG;
+    if (!ld_ok(ldx, (int)hdr_r->K, M) || ldy < (int)hdr_r->N) return SPW_ERR_INVALID_ARG;
+    if (!aligned16(d_buf_r) || !aligned16(d_s24) || !aligned16(d_X) || !aligned16(d_Y))
+        return SPW_ERR_ALIGNMENT;
+    const uint64_t need = (uint64_t)hdr_r->n_strips * hdr_r->n_ktiles * (kS24ValBytes + kS24MetaBytes);
+    if (s24_bytes < need) return SPW_ERR_BUFFER_TOO_SMALL;
+    return tc_product(hdr_r, d_buf_r, d_X, M, ldx, d_Y, ldy, 0, 0.0f, nullptr, d_ws, ws_bytes,
+                      (cudaStream_t)stream, nullptr, nullptr, 0, (const uint8_t*)d_s24);
 }
 
 uint64_t spw_spmv_tc_workspace_bytes(const spw_format* hdr, int B) {

@@ -172,3 +172,18 @@ def domain_tokens(M: int, K: int, n_domains: int, block_density: float, *seed_pa
     cols = np.repeat(blocks, 64, axis=1)[:, :K]
     x[~cols[dom]] = 0.0
     return x.astype(np.float16), dom
+
+
+def structured24_mask(N: int, K: int, *seed_parts, extra: float = 0.0) -> np.ndarray:
+    """A 2:4-structured mask: in every group of four columns of a row, 0, 1 or 2 kept
+    positions (uniform count, seeded random positions); with extra > 0, each dropped
+    position is then kept with that probability as well (weights outside the 2:4
+    pattern, the residual of a 2:4 + residual split)."""
+    r = rng("mask24", N, K, extra, *seed_parts)
+    G = -(-K // 4)
+    cnt = r.integers(0, 3, size=(N, G, 1))
+    rank = np.argsort(np.argsort(r.random((N, G, 4)), axis=2), axis=2)
+    keep = (rank < cnt).reshape(N, 4 * G)[:, :K]
+    if extra > 0:
+        keep |= r.random((N, K)) < extra
+    return keep.astype(np.uint8)
