@@ -71,8 +71,9 @@ constexpr int kTcbWarp = 2 + kDecoderWarps;             // the TCB producer's wa
 constexpr int kThreads = 32 * (3 + kDecoderWarps);      // X producer, MMA, decoders, TCB producer
 constexpr uint32_t kWStageBytes = kTileRows * kBK * 2;  // 16 KB
 constexpr int kSmemLimit = 227 * 1024;
-// 2:4 mode (spw_spmm24): per k-step S stage = the 2:4 values of both strips (2 x 4 KB, the
-// 64-byte-swizzled K-major layout of split24.cu) and their metadata (2 x 512 bytes).
+// 2:4 mode (spw_spmm24): per k-step S area = the 2:4 values of both strips (2 x 4 KB, the
+// 64-byte-swizzled K-major layout of split24.cu) and their metadata (2 x 512 bytes), held
+// in the X stage right after the token tile.
 constexpr uint32_t kS24ValBytes = 4096;
 constexpr uint32_t kS24MetaBytes = 512;
 constexpr uint32_t kSStageBytes = kTileStrips * (kS24ValBytes + kS24MetaBytes);  // 9 KB
@@ -95,7 +96,7 @@ struct SpmmParams {
     int n_whole;                // tiles 0 .. n_whole-1 run whole; the rest are split
     int m_tiles;                // token tiles (tile t: token tile t % m_tiles, weight rows t / m_tiles)
     int sx, sr, sw;             // X, raw-tile and decoded-weight stage counts
-    uint32_t x_stage_bytes;     // MT * 128
+    uint32_t x_stage_bytes;     // MT * 128 (2:4 mode: + the S area)
     uint32_t raw_stage_bytes;   // 1024 + 2 * val_slot
     uint32_t val_slot;          // bytes per strip's values slot (incl. 16 bytes of slack)
     uint32_t tmem_cols;
@@ -109,11 +110,11 @@ struct SpmmParams {
     int sig_words;
     uint32_t off_klist;         // dynamic smem: the visited k-tile count, then the list
     // 2:4 + residual (spw_spmm24): the structured part (split24.cu layout); the TCB
-    // sections above then describe the residual.  ss S stages at off_s; the metadata of
-    // W stage w sits in tensor-memory columns e_col + 2 w and e_col + 2 w + 1.
+    // sections above then describe the residual.  Each X stage holds the k-step's S area
+    // at byte off_s; the metadata of X stage s sits in tensor-memory columns e_col + 2 s
+    // and e_col + 2 s + 1.
     const uint8_t* s24_vals;
     const uint8_t* s24_meta;
-    int ss;
     uint32_t off_s, e_col;
 };
 
@@ -393,10 +394,9 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     uint64_t* acc_full = w_empty + SW;
     uint64_t* drain = acc_full + 1;
     uint64_t* peer_ready = drain + 1;  // PAIR, on rank 0: the other CTA's stages are ready
-    const int SS = SP24 ? p.ss : 0;
-    uint64_t* s_full = peer_ready + kPeerSlots;  // 2:4 mode: the S ring
-    uint64_t* s_empty = s_full + SS;
-    uint32_t* tmem_slot = (uint32_t*)(s_empty + SS);
+    const int SMF = SP24 ? SX : 0;
+    uint64_t* m_full = peer_ready + kPeerSlots;  // 2:4 mode: an X stage's metadata is in tensor memory
+    uint32_t* tmem_slot = (uint32_t*)(m_full + SMF);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     volatile uint32_t* last_flag = (volatile uint32_t*)(tmem_slot + 2);
     uint32_t* tptr = (uint32_t*)(smem + p.off_tptr);
@@ -419,10 +419,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         mbar_init(smem_u32(acc_full), 1);
         mbar_init(smem_u32(drain), 1);
         for (int i = 0; i < kPeerSlots; i++) mbar_init(smem_u32(&peer_ready[i]), 1);
-        for (int i = 0; i < SS; i++) {
-            mbar_init(smem_u32(&s_full[i]), 1);
-            mbar_init(smem_u32(&s_empty[i]), 1);
-        }
+        for (int i = 0; i < SMF; i++) mbar_init(smem_u32(&m_full[i]), 4);  // the four metadata warps
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
@@ -494,7 +491,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         return e;
     };
 
-    int x_issued = 0, r_issued = 0, s_issued = 0;  // producers' lane 0: stages armed
+    int x_issued = 0, r_issued = 0;  // lane 0 of warp 0 (X) and of the TCB warp: stages armed
     if (warp == 0 || warp == kTcbWarp) {
         // ------------------------------------------------------------ producer
         if (warp == 0 && lane == 0) {  // X ring
@@ -513,10 +510,27 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     break;
                 }
                 const uint32_t xbar = smem_u32(&x_full[xs]);
-                mbar_arrive_expect_tx(xbar, p.x_stage_bytes);
+                const uint32_t xst = sbase + (uint32_t)xs * p.x_stage_bytes;
+                uint32_t xbytes = p.x_stage_bytes;
+                if constexpr (SP24) {  // the token tile, then the 2:4 values and metadata
+                    xbytes = p.off_s;
+                    for (int j = 0; j < kTileStrips; j++)
+                        if (s0 + j < p.n_strips) xbytes += kS24ValBytes + kS24MetaBytes;
+                }
+                mbar_arrive_expect_tx(xbar, xbytes);
                 for (int h = 0; h < p.nh; h++)
-                    tma_load_2d(sbase + (uint32_t)xs * p.x_stage_bytes + (uint32_t)(h * crows * 128),
-                                &tmap_x, kt * kBK, m0 + h * rows + (int)rank * crows, xbar);
+                    tma_load_2d(xst + (uint32_t)(h * crows * 128), &tmap_x, kt * kBK,
+                                m0 + h * rows + (int)rank * crows, xbar);
+                if constexpr (SP24) {
+                    for (int j = 0; j < kTileStrips; j++) {
+                        if (s0 + j >= p.n_strips) continue;
+                        const size_t t = (size_t)(s0 + j) * nk + kt;
+                        bulk_g2s(xst + p.off_s + kS24ValBytes * j, p.s24_vals + t * kS24ValBytes,
+                                 kS24ValBytes, xbar);
+                        bulk_g2s(xst + p.off_s + kTileStrips * kS24ValBytes + kS24MetaBytes * j,
+                                 p.s24_meta + t * kS24MetaBytes, kS24MetaBytes, xbar);
+                    }
+                }
                 x_issued++;
                 if (++xs == SX) { xs = 0; xph ^= 1u; }
             }
@@ -556,28 +570,6 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 }
                 r_issued++;
                 if (++rs == SR) { rs = 0; rph ^= 1u; }
-                if constexpr (SP24) {  // the 2:4 values and metadata of both strips
-                    const int ss_ = i % SS;
-                    if (i >= SS && !wait_or_abort(smem_u32(&s_empty[ss_]), (uint32_t)(((i / SS) - 1) & 1),
-                                                  abort_flag, p.wait_limit)) {
-                        abort_both();
-                        break;
-                    }
-                    const uint32_t sbar = smem_u32(&s_full[ss_]);
-                    const uint32_t sst = sbase + p.off_s + (uint32_t)ss_ * kSStageBytes;
-                    uint32_t sbytes = 0;
-                    for (int j = 0; j < kTileStrips; j++)
-                        if (s0 + j < p.n_strips) sbytes += kS24ValBytes + kS24MetaBytes;
-                    mbar_arrive_expect_tx(sbar, sbytes);
-                    for (int j = 0; j < kTileStrips; j++) {
-                        if (s0 + j >= p.n_strips) continue;
-                        const size_t t = (size_t)(s0 + j) * nk + kt;
-                        bulk_g2s(sst + kS24ValBytes * j, p.s24_vals + t * kS24ValBytes, kS24ValBytes, sbar);
-                        bulk_g2s(sst + kTileStrips * kS24ValBytes + kS24MetaBytes * j,
-                                 p.s24_meta + t * kS24MetaBytes, kS24MetaBytes, sbar);
-                    }
-                    s_issued++;
-                }
             }
         }
     } else if (warp == 1 && (!PAIR || rank == 0)) {
@@ -590,16 +582,18 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         uint32_t xph = 0, wph = 0;
         bool ok = true;
         for (int i = 0; i < n_kc && ok; i++) {
+            // 2:4 mode: the W ring advances only on k-steps with residual weights
+            const bool dense = !SP24 || !residual_empty(kstep(i));
             ok = __all_sync(0xffffffffu, wait_or_abort(smem_u32(&x_full[xs]), xph, abort_flag, p.wait_limit));
-            ok = ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_full[ws]), wph, abort_flag, p.wait_limit));
+            if (dense)
+                ok = ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_full[ws]), wph, abort_flag, p.wait_limit));
             if constexpr (PAIR)
                 ok = ok && __all_sync(0xffffffffu,
                                       wait_or_abort_cluster(smem_u32(&peer_ready[i % kPeerSlots]),
                                                             (uint32_t)((i / kPeerSlots) & 1), abort_flag,
                                                             p.wait_limit));
             if constexpr (SP24)
-                ok = ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&s_full[i % SS]),
-                                                                 (uint32_t)((i / SS) & 1), abort_flag,
+                ok = ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&m_full[xs]), xph, abort_flag,
                                                                  p.wait_limit));
             if (!ok) {
                 if (lane == 0) abort_both();
@@ -609,21 +603,19 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 tc_fence_after();
                 const uint32_t xa = sbase + (uint32_t)xs * p.x_stage_bytes;
                 const uint32_t wa = sbase + p.off_w + (uint32_t)ws * kWStageBytes;
-                bool dense = true;  // the decoded W stage takes part (always, except 2:4 mode)
                 if constexpr (SP24) {
                     // Two sparse MMAs (K = 32 each: 16 stored halves = 32 bytes of the S
                     // stage's rows, 64 bytes of X's), then the residual's dense MMAs when
                     // the k-tile holds any residual weight.
-                    const uint32_t sa = sbase + p.off_s + (uint32_t)(i % SS) * kSStageBytes;
+                    const uint32_t sa = xa + p.off_s;
                     const uint32_t idesc_sp = idesc | (1u << 2);
 #pragma unroll
                     for (int j = 0; j < 2; j++) {
                         const uint64_t adesc = umma_desc_sw64(sa + 32u * j);
                         const uint64_t bdesc = umma_desc_sw128(xa + 64u * j);
-                        umma_f16_sp(tmem, adesc, bdesc, idesc_sp | (uint32_t)j, tmem + p.e_col + 2u * ws,
-                                    (i > 0 || j > 0) ? 1u : 0u);
+                        umma_f16_sp(tmem, adesc, bdesc, idesc_sp | (uint32_t)j,
+                                    tmem + p.e_col + 2u * (uint32_t)xs, (i > 0 || j > 0) ? 1u : 0u);
                     }
-                    dense = !residual_empty(kstep(i));
                 }
 #pragma unroll
                 for (int j = 0; j < kBK / 16; j++) {
@@ -646,13 +638,12 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                     umma_commit_pair_both(smem_u32(&w_empty[ws]));
                 } else {
                     umma_commit(smem_u32(&x_empty[xs]));
-                    umma_commit(smem_u32(&w_empty[ws]));
-                    if constexpr (SP24) umma_commit(smem_u32(&s_empty[i % SS]));
+                    if (dense) umma_commit(smem_u32(&w_empty[ws]));
                 }
             }
             __syncwarp();
             if (++xs == SX) { xs = 0; xph ^= 1u; }
-            if (++ws == SW) { ws = 0; wph ^= 1u; }
+            if (dense && ++ws == SW) { ws = 0; wph ^= 1u; }
         }
         if (lane == 0) {
             if constexpr (PAIR) {
@@ -706,7 +697,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         // the 8 lanes of each quarter-warp write 8 distinct swizzled chunk positions.
         const uint32_t swap = ((uint32_t)lane >> 2) & 1u;
         const uint32_t rowA = nl0 + swap, rowB = nl0 + 1u - swap;
-        int rs = 0, ws = 0;
+        int rs = 0, ws = 0, wi = 0;  // wi: W stages filled so far
         uint32_t rph = 0, wph = 0;
         for (int i = 0; i < n_kc; i++) {
             // every lane waits; __all_sync keeps the outcome warp-uniform
@@ -759,38 +750,16 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 }
             }
             __syncwarp();
-            if (i >= SW &&
+            // 2:4 mode: a k-tile without residual weights needs no dense W stage (the MMA
+            // warp skips its dense MMAs), so the W ring (w_full / w_empty, the stage index)
+            // advances only on k-steps with residual weights, on both sides alike.
+            const bool skip = SP24 && residual_empty(kstep(i));
+            if (!skip && wi >= SW &&
                 !__all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_empty[ws]), wph ^ 1u, abort_flag, p.wait_limit))) {
                 abort_both();
                 break;
             }
             unsigned char* wst = smem + p.off_w + (uint32_t)ws * kWStageBytes;
-            // 2:4 mode: a k-tile without residual weights needs no dense W stage (the MMA
-            // warp skips its dense MMAs); decoder warps 0-3 (one per tensor-memory lane
-            // quarter) move the k-step's metadata into the W stage's two metadata columns.
-            const bool skip = SP24 && residual_empty(kstep(i));
-            if constexpr (SP24) {
-                if (d < 4) {
-                    if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&s_full[i % SS]), (uint32_t)((i / SS) & 1),
-                                                               abort_flag, p.wait_limit))) {
-                        abort_both();
-                        break;
-                    }
-                    const int quarter = warp & 3;
-                    const int gl = 32 * quarter + lane;  // tensor-memory lane = row block lane
-                    const int sq = gl >> 6, L = gl & 63;
-                    uint32_t m0 = 0x44444444u, m1 = 0x44444444u;  // rows past N: {0, 1} groups
-                    if (s0 + sq < p.n_strips) {
-                        const uint32_t* mw = (const uint32_t*)(smem + p.off_s + (size_t)(i % SS) * kSStageBytes +
-                                                               kTileStrips * kS24ValBytes + kS24MetaBytes * sq);
-                        m0 = mw[L];
-                        m1 = mw[64 + L];
-                    }
-                    tmem_st2(tmem + ((uint32_t)(32 * quarter) << 16) + p.e_col + 2u * (uint32_t)ws, m0, m1);
-                    tmem_st_wait();
-                    tc_fence_before();
-                }
-            }
             if (!skip) {  // 8 columns -> one 16-byte chunk per row
                 uint32_t o0[4] = {0u, 0u, 0u, 0u}, o1[4] = {0u, 0u, 0u, 0u};
                 if (dec) {
@@ -818,11 +787,45 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             fence_proxy_async_smem();  // generic-proxy stores -> tensor-core reads
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(smem_u32(&w_full[ws]));
+                if (!skip) mbar_arrive(smem_u32(&w_full[ws]));
                 mbar_arrive(smem_u32(&r_empty[rs]));
             }
             if (++rs == SR) { rs = 0; rph ^= 1u; }
-            if (++ws == SW) { ws = 0; wph ^= 1u; }
+            if (!skip) {
+                wi++;
+                if (++ws == SW) { ws = 0; wph ^= 1u; }
+            }
+            // 2:4 mode: decoder warps 0-3 (one per tensor-memory lane quarter) move the
+            // k-step's metadata from its X stage into that stage's two metadata columns and
+            // arrive on the stage's m_full -- after releasing the raw stage, so that the
+            // TCB ring never waits for the X stage.  The columns are free: the copy waited
+            // for here was issued only after the MMAs of the stage's previous k-step had
+            // completed.
+            if constexpr (SP24) {
+                if (d < 4) {
+                    const int xs_ = i % SX;
+                    if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&x_full[xs_]), (uint32_t)((i / SX) & 1),
+                                                               abort_flag, p.wait_limit))) {
+                        abort_both();
+                        break;
+                    }
+                    const int quarter = warp & 3;
+                    const int gl = 32 * quarter + lane;  // tensor-memory lane = row block lane
+                    const int sq = gl >> 6, L = gl & 63;
+                    uint32_t m0 = 0x44444444u, m1 = 0x44444444u;  // rows past N: {0, 1} groups
+                    if (s0 + sq < p.n_strips) {
+                        const uint32_t* mw = (const uint32_t*)(smem + (size_t)xs_ * p.x_stage_bytes + p.off_s +
+                                                               kTileStrips * kS24ValBytes + kS24MetaBytes * sq);
+                        m0 = mw[L];
+                        m1 = mw[64 + L];
+                    }
+                    tmem_st2(tmem + ((uint32_t)(32 * quarter) << 16) + p.e_col + 2u * (uint32_t)xs_, m0, m1);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&m_full[xs_]));
+                }
+            }
         }
 
         // ------------------------------------------------------------ epilogue
@@ -952,11 +955,6 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             const int last = i + ((r_issued - 1 - i) / SR) * SR;
             (void)mbar_drain(smem_u32(&r_full[i]), (uint32_t)((last / SR) & 1));
         }
-        if constexpr (SP24)
-            for (int i = 0; warp == kTcbWarp && lane == 0 && i < SS && i < s_issued; i++) {
-                const int last = i + ((s_issued - 1 - i) / SS) * SS;
-                (void)mbar_drain(smem_u32(&s_full[i]), (uint32_t)((last / SS) & 1));
-            }
     }
     __syncthreads();
     // Pair mode: rank 0's MMAs read both CTAs' shared memory and write both tensor
@@ -999,8 +997,7 @@ int get_encoder() {
 
 struct SpmmPlan {
     bool pair;  // 256-row tiles on SM pairs (tcgen05 cta_group::2)
-    bool sp24;  // 2:4 + residual: S stages, metadata columns, at most 256 tokens per tile
-    int ss;
+    bool sp24;  // 2:4 + residual: S areas in the X stages, metadata columns, <= 256 tokens
     uint32_t off_s, e_col;
     int MT, nh, n_acc, m_tiles, n_tiles, ksplit, n_whole, sx, sr, sw, ctas_per_sm;
     uint32_t x_stage_bytes, val_slot, raw_stage_bytes, tmem_cols;
@@ -1058,7 +1055,6 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
     if (sms <= 0) return SPW_ERR_CUDA;
     pl->pair = false;
     pl->sp24 = sp24;
-    pl->ss = 0;
     pl->off_s = 0;
     pl->e_col = 0;
     if (allow_pair && !rule && !tokens && !sp24 && M >= 256 && h->N > (uint32_t)kTileRows) {
@@ -1135,6 +1131,10 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
     pl->nh = per > 256 ? 2 : 1;
     pl->MT = (int)round_up_u64((uint64_t)per, 16u * pl->nh);  // each MMA's N a multiple of 16
     pl->x_stage_bytes = (uint32_t)pl->MT * (pl->pair ? 64u : 128u);  // this CTA's share of X
+    if (sp24) {  // the k-step's 2:4 values and metadata follow the token tile
+        pl->off_s = pl->x_stage_bytes;
+        pl->x_stage_bytes += kSStageBytes;
+    }
     pl->n_acc = (pl->MT <= 32 && !sp24) ? 4 : 1;
     uint32_t cols = 32;
     while (cols < (uint32_t)(pl->n_acc > 1 ? 32 * pl->n_acc : pl->MT)) cols <<= 1;
@@ -1151,7 +1151,7 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
     // {X, TCB, decoded-weight, 2:4} stages, deepest first
     const int options[][4] = {{4, 4, 4, 0}, {3, 4, 4, 0}, {2, 4, 4, 0}, {2, 4, 3, 0}, {2, 3, 3, 0},
                               {2, 3, 2, 0}, {2, 2, 2, 0}};
-    const int options24[][4] = {{4, 3, 3, 3}, {3, 3, 3, 3}, {3, 2, 3, 3}, {2, 3, 3, 3}, {2, 2, 2, 2}};
+    const int options24[][4] = {{4, 3, 2, 0}, {3, 3, 2, 0}, {3, 2, 2, 0}, {2, 2, 2, 0}};
     bool found = false;
     const int n_opt = sp24 ? (int)(sizeof(options24) / sizeof(options24[0]))
                            : (int)(sizeof(options) / sizeof(options[0]));
@@ -1159,20 +1159,18 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
         const int* o = sp24 ? options24[oi] : options[oi];
         const int sx = o[0], sr = o[1], sw = o[2], ss = o[3];
         const uint32_t off_w = (uint32_t)sx * pl->x_stage_bytes;
-        const uint32_t off_s = off_w + (uint32_t)sw * kWStageBytes;  // 1024-byte aligned
-        const uint32_t off_raw = off_s + (uint32_t)ss * kSStageBytes;
+        const uint32_t off_raw = off_w + (uint32_t)sw * kWStageBytes;
+        (void)ss;
         const uint32_t off_rec = off_raw + (uint32_t)sr * pl->raw_stage_bytes;
         const uint32_t off_tptr = off_rec + kRecBytesPerWarp * kDecoderWarps;
         const uint32_t off_klist = off_tptr + tptr_bytes;
         const uint32_t off_bar = (uint32_t)round_up_u64(off_klist + klist_bytes, 8);
-        const uint32_t bar_bytes = 8u * (2 * sx + 2 * sr + 2 * sw + 2 + kPeerSlots + 2 * ss) + 16u;
+        const uint32_t bar_bytes = 8u * (2 * sx + 2 * sr + 2 * sw + 2 + kPeerSlots + (sp24 ? sx : 0)) + 16u;
         const size_t total = (size_t)off_bar + bar_bytes + 1024;  // + base alignment slack
         if (total <= (size_t)kSmemLimit) {
             pl->sx = sx;
             pl->sr = sr;
             pl->sw = sw;
-            pl->ss = ss;
-            pl->off_s = off_s;
             pl->off_w = off_w;
             pl->off_raw = off_raw;
             pl->off_rec = off_rec;
@@ -1289,7 +1287,6 @@ int tc_product(const spw_format* hdr, const void* d_buf, const uint16_t* d_X, in
         const uint64_t n_tiles = (uint64_t)hdr->n_strips * hdr->n_ktiles;
         prm.s24_vals = s24;
         prm.s24_meta = s24 + n_tiles * kS24ValBytes;
-        prm.ss = pl.ss;
         prm.off_s = pl.off_s;
         prm.e_col = pl.e_col;
     }
