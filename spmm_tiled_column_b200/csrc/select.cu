@@ -117,8 +117,9 @@ __device__ inline uint32_t block_exclusive_scan(uint32_t v, uint32_t* s_warp, ui
 // it starts at the highest bit any key has set (the keys' top bits are mostly zero), takes
 // 11 bits per pass (2048 bins, a CTA-wide scan from the top bin down), and stops as soon
 // as the kk-th key's bin is selected whole.  The selected set is {key >= threshold}.
-// (Measured on B200 at K = 11008: 16.7 us; per-warp-pair 256-bin histograms and warp-
-// aggregated histogram updates were both slower.)
+// Used for B > 1 (about 40 us at K = 11008 on B200, graph-timed; per-warp-pair 256-bin
+// histograms and warp-aggregated histogram updates were both slower); one row takes
+// topk1_kernel below.
 constexpr int kDigitBits = 11;
 constexpr int kBins = 1 << kDigitBits;
 static_assert(kBins == 2 * kSelThreads, "the scan gives each thread two bins");
@@ -234,6 +235,138 @@ topk_kernel(const uint16_t* __restrict__ x, int B, int K, int ldx, int kk,
     }
 }
 
+// Writes act_bits and, when idx is not NULL, the ascending index list from the selected
+// words s_selw[n_words] (s_wofs: n_words words of scratch).  Whole CTA.
+__device__ inline void emit_selection(const uint32_t* s_selw, uint32_t* s_wofs, uint32_t* s_warp,
+                                      int K, uint32_t* act_bits, uint32_t* idx) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int n_words = (K + 31) / 32;
+    uint32_t carry = 0;
+    for (int w0 = 0; w0 < n_words; w0 += kSelThreads) {
+        const int w = w0 + tid;
+        const uint32_t word = w < n_words ? s_selw[w] : 0u;
+        if (w < n_words) act_bits[w] = word;
+        uint32_t total;
+        const uint32_t ex = block_exclusive_scan((uint32_t)__popc(word), s_warp, &total);
+        if (w < n_words) s_wofs[w] = carry + ex;
+        carry += total;
+    }
+    if (!idx) return;
+    __syncthreads();
+    for (int w0 = 0; w0 < n_words; w0 += kSelThreads / 32) {
+        const int w = w0 + (tid >> 5);
+        if (w >= n_words) continue;
+        const uint32_t word = s_selw[w];
+        if ((word >> lane) & 1u) idx[s_wofs[w] + __popc(word & lanemask_lt())] = (uint32_t)(32 * w + lane);
+    }
+}
+
+// In warp 0: bins hist[nb-1] .. hist[0] from the top, nb / 32 per lane; finds the bin
+// holding the kk-th largest element (1 <= kk <= the histogram's total) and how many
+// elements lie in higher bins, returned to every lane.
+__device__ inline void find_bin_from_top(const uint32_t* hist, int nb, uint32_t kk, int lane,
+                                         uint32_t* bin, uint32_t* above) {
+    const int per = nb / 32;
+    uint32_t sum = 0;
+    for (int j = 0; j < per; j++) sum += hist[nb - 1 - per * lane - j];
+    const uint32_t incl = (uint32_t)warp_inclusive_scan((int)sum, lane);
+    const uint32_t excl = incl - sum;
+    uint32_t b = 0, a = 0;
+    bool found = false;
+    if (excl < kk && kk <= incl) {
+        uint32_t run = excl;
+        for (int j = 0; j < per; j++) {
+            const uint32_t c = hist[nb - 1 - per * lane - j];
+            if (run + c >= kk) {
+                b = (uint32_t)(nb - 1 - per * lane - j);
+                a = run;
+                found = true;
+                break;
+            }
+            run += c;
+        }
+    }
+    const uint32_t m = __ballot_sync(0xffffffffu, found);
+    const int src = m ? __ffs(m) - 1 : 0;
+    *bin = __shfl_sync(0xffffffffu, b, src);
+    *above = __shfl_sync(0xffffffffu, a, src);
+}
+
+// Top-k of one row (B = 1).  The score is |x| itself, so the fp16 magnitude bits (15
+// bits; Inf and NaN clamped to 0x7C00, tying above every finite value) order the columns
+// exactly.  Two histogram passes -- the top 7 bits, then the low 8 bits within the chosen
+// top bin -- give the threshold magnitude T and how many columns of magnitude T to keep;
+// those are the lowest-index ones (ties to the lower index), found with one CTA-wide scan
+// over the columns in index order (thread t owns a contiguous run of columns).
+constexpr int kT1Hi = 128, kT1Lo = 256;
+
+__global__ void __launch_bounds__(kSelThreads)
+topk1_kernel(const uint16_t* __restrict__ x, int K, int kk, uint32_t* __restrict__ act_bits,
+             uint32_t* __restrict__ idx) {
+    extern __shared__ uint32_t s_dyn[];  // K magnitudes (u16), selected words, word offsets
+    const int n_words = (K + 31) / 32;
+    uint16_t* s_mag = (uint16_t*)s_dyn;
+    uint32_t* s_selw = s_dyn + (K + 1) / 2;
+    uint32_t* s_wofs = s_selw + n_words;
+    __shared__ uint32_t s_hist[kT1Lo];
+    __shared__ uint32_t s_warp[kSelThreads / 32 + 1];
+    __shared__ uint32_t s_bin, s_rem;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int k = tid; k < K; k += kSelThreads) {
+        const uint32_t m = (uint32_t)__ldg(x + k) & 0x7fffu;
+        s_mag[k] = (uint16_t)(m > 0x7c00u ? 0x7c00u : m);
+    }
+    for (int w = tid; w < n_words; w += kSelThreads) s_selw[w] = 0u;
+    if (tid < kT1Lo) s_hist[tid] = 0u;
+    __syncthreads();
+    if (kk > 0) {
+        for (int k = tid; k < K; k += kSelThreads) atomicAdd(&s_hist[s_mag[k] >> 8], 1u);
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t b, a;
+            find_bin_from_top(s_hist, kT1Hi, (uint32_t)kk, lane, &b, &a);
+            if (lane == 0) {
+                s_bin = b;
+                s_rem = (uint32_t)kk - a;
+            }
+        }
+        __syncthreads();
+        const uint32_t hb = s_bin, rem = s_rem;
+        __syncthreads();  // every thread has read s_bin and s_rem
+        if (tid < kT1Lo) s_hist[tid] = 0u;
+        __syncthreads();
+        for (int k = tid; k < K; k += kSelThreads) {
+            const uint32_t m = s_mag[k];
+            if ((m >> 8) == hb) atomicAdd(&s_hist[m & 0xffu], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t b, a;
+            find_bin_from_top(s_hist, kT1Lo, rem, lane, &b, &a);
+            if (lane == 0) {
+                s_bin = (hb << 8) | b;
+                s_rem = rem - a;  // columns of magnitude T to keep, the lowest indices first
+            }
+        }
+        __syncthreads();
+        const uint32_t T = s_bin, take = s_rem;
+        const int c = (K + kSelThreads - 1) / kSelThreads;
+        const int k0 = tid * c, k1 = min(k0 + c, K);
+        uint32_t ties = 0;
+        for (int k = k0; k < k1; k++) ties += s_mag[k] == T ? 1u : 0u;
+        uint32_t total;
+        uint32_t rank = block_exclusive_scan(ties, s_warp, &total);
+        for (int k = k0; k < k1; k++) {
+            const uint32_t m = s_mag[k];
+            bool sel = m > T;
+            if (m == T) sel = rank++ < take;
+            if (sel) atomicOr(&s_selw[k >> 5], 1u << (k & 31));
+        }
+    }
+    __syncthreads();
+    emit_selection(s_selw, s_wofs, s_warp, K, act_bits, kk > 0 ? idx : nullptr);
+}
+
 int check_x(const uint16_t* d_x, int B, int K, int ldx) {
     if (!d_x || B < 1 || B > 16 || K < 1 || ldx < K) return SPW_ERR_INVALID_ARG;
     if (!aligned16(d_x)) return SPW_ERR_ALIGNMENT;
@@ -266,6 +399,21 @@ int spw_select_topk(const uint16_t* d_x, int B, int K, int ldx, int k, uint32_t*
     if (!d_act_bits || k < 0 || k > K) return SPW_ERR_INVALID_ARG;
     if (!aligned16(d_act_bits) || ((uintptr_t)d_idx & 3u)) return SPW_ERR_ALIGNMENT;
     if (K > kTopkMaxK) return SPW_ERR_UNSUPPORTED;
+    if (B == 1) {
+        // magnitudes (u16, rounded up to whole words), selected words, word offsets
+        const size_t smem1 = 4 * (size_t)((K + 1) / 2) + 8 * (size_t)((K + 31) / 32);
+        static bool attr1_set[kMaxDevices];
+        int dev1 = 0;
+        SPW_CUDA_TRY(cudaGetDevice(&dev1));
+        if (dev1 >= 0 && dev1 < kMaxDevices && !attr1_set[dev1]) {
+            SPW_CUDA_TRY(cudaFuncSetAttribute(topk1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              4 * ((kTopkMaxK + 1) / 2) + 8 * (kTopkMaxK / 32)));
+            attr1_set[dev1] = true;
+        }
+        topk1_kernel<<<1, kSelThreads, smem1, (cudaStream_t)stream>>>(d_x, K, k, d_act_bits, d_idx);
+        SPW_LAUNCH_CHECK();
+        return SPW_OK;
+    }
     // keys, then one word offset per 32 columns
     const size_t smem = (size_t)K * sizeof(unsigned long long) + 4 * (size_t)((K + 31) / 32);
     static bool attr_set[kMaxDevices];

@@ -64,6 +64,23 @@ def test_topk_ties_and_specials():
         np.testing.assert_array_equal(host(idx), ref_idx)
 
 
+@pytest.mark.parametrize("K", [1, 33, 1000, 11008, 24576])
+def test_topk_one_row_ties_and_specials(K):
+    # one row: few distinct magnitudes (many ties, both signs), and Inf / NaN, which tie
+    # above every finite value; every k from none to all
+    r = np.random.default_rng(K)
+    vals = np.array([0, -0.0, 0.5, -0.5, 1, -1, 2, 65504, -65504, 6e-8, np.inf, -np.inf, np.nan],
+                    np.float16)
+    x = r.choice(vals, size=(1, K), p=[.2, .1, .15, .15, .1, .1, .1, .02, .02, .02, .01, .01, .02])
+    for k in sorted({0, 1, K // 3, K // 2, K - 1, K} - {-1}):
+        if k < 0:
+            continue
+        bits, idx = spw.spw_select_topk(dev(x), k)
+        ref_bits, ref_idx = oracle.select_topk(x, k)
+        np.testing.assert_array_equal(host(bits)[:words(K)], ref_bits)
+        np.testing.assert_array_equal(host(idx)[:k], ref_idx)
+
+
 def test_topk_too_large_k_is_unsupported():
     x = dev(np.ones((1, 30000), np.float16))
     with pytest.raises(spw.SpwError) as e:
