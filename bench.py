@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --sweep decode|prefill|taxonomy [--quick] [--out FILE]
-    python bench.py --case spmv|spmm|tc|ffn [--layer L] [--batch B] [--act A] [--m M] ...
+    python bench.py --case spmv|spmm|tc|ffn|spmm24|tokens [--layer L] [--batch B] [--act A] [--m M] ...
 
 A step is one decode pass over the seven pruned linear layers of one Llama-7B decoder
 layer (q, k, v, o: 4096 x 4096; gate, up: 11008 x 4096; down: 4096 x 11008), fp16
@@ -20,8 +20,10 @@ value = algorithmic bytes / time (GB/s): per linear, the values and bitmap words
 active columns plus the activations read and the outputs written.  Prefill (spw_spmm at
 M = 2048, graph-replayed over rotated operands), the dense cuBLAS comparisons (fp32
 accumulation, no fp16 reduced-precision reductions), the decode time against a plain
-copy of the same bytes (the three-layer-format page's Fig. 5) and the bytes per weight
-of dense / CSR / TCB storage (its Fig. 3) are extra keys of the same JSON line.
+copy of the same bytes (the three-layer-format page's Fig. 5), the bytes per weight
+of dense / CSR / TCB storage (its Fig. 3), prefill with per-token index sets and token
+grouping (spw_spmm_tokens) and the 2:4 + residual prefill on sparse tensor cores
+(spw_spmm24) are extra keys of the same JSON line.
 
 --impl reference times the fp64 CPU oracle (this path's reference implementation) on
 one pinned host core: each step is a bounded sample of the same workload (the decode of
@@ -641,6 +643,10 @@ def run_ours(args, rank, world, local_rank):
         prefill_tokens = run_prefill_tokens(dev, stream)
     except Exception as exc:
         prefill_tokens = {"unavailable": f"{type(exc).__name__}: {exc}"[:300]}
+    try:
+        prefill24 = run_prefill24(dev, stream, tc_peak)
+    except Exception as exc:
+        prefill24 = {"unavailable": f"{type(exc).__name__}: {exc}"[:300]}
 
     # Decode time against a plain copy of the same bytes (the launch's compressed
     # weights), per grouped launch: the three-layer-format page's comparison of global
@@ -683,6 +689,7 @@ def run_ours(args, rank, world, local_rank):
         "prefill": prefill,
         "prefill_detail": prefill_detail,
         "prefill_tokens": prefill_tokens,
+        "prefill_2of4_residual": prefill24,
         "decode_vs_plain_copy": decode_vs_read,
         "storage_bytes_per_weight": storage,
     }
@@ -823,6 +830,68 @@ def run_prefill_tokens(dev, stream):
                   "each token tile's k-tiles; the kernel time follows the longest k-tile list")
     del bufs, Wds, Wd0, sl
     torch.cuda.empty_cache()
+    return out
+
+
+def run_prefill24(dev, stream, tc_peak):
+    """spw_spmm24 (2:4 part on tcgen05.mma.sp + TCB residual; the three-layer-format
+    page's layers (i) and (iii)) at M = 2048 on the q shape for three masks: the 50 %
+    magnitude mask (residual = every kept weight beyond two per group of four), an exact
+    2:4 mask (no residual) and 2:4 plus 0.5 % of the input channels kept whole (residual
+    in those columns).  Against spw_spmm on the same mask and cuBLAS on the dense masked
+    weight; graph replays over 3 rotated operand sets."""
+    import torch
+    import spmm_tiled_column_b200 as spw
+    M, R, name = 2048, 3, "q"
+    N, K = workloads.LLAMA7B_LAYERS[name]
+    layer = workloads.pruned_layer(name, N, K, SPARSITY, "bench-24")
+    masks = {"magnitude_50": layer.mask,
+             "exact_2of4": workloads.structured24_mask(N, K, "bench-24", count=2),
+             "2of4_plus_dense_channels_0.5pct": workloads.structured24_mask(
+                 N, K, "bench-24", count=2, dense_channels=0.005)}
+    W = _dev(layer.W)
+    g = torch.Generator(device=dev).manual_seed(24)
+    Xs = [torch.randn((M, K), device=dev, dtype=torch.float16, generator=g) for _ in range(R)]
+    Ys = [torch.empty((M, N), device=dev, dtype=torch.float16) for _ in range(R)]
+    out = {"layer": f"{name} {N}x{K}", "M": M}
+    for key, mask in masks.items():
+        md = _dev(mask)
+        l24 = spw.SparseLinear24(W, md)
+        sl = spw.SparseLinear(W, md)
+        s24s = [l24.s24] + [l24.s24.clone() for _ in range(R - 1)]
+        brs = [l24.buf_r] + [l24.buf_r.clone() for _ in range(R - 1)]
+        need = spw.spw_spmm24_workspace_bytes(l24.hdr_r, M)
+        wss = [torch.zeros(max(need, 16), dtype=torch.uint8, device=dev) for _ in range(R)]
+        us24 = graph_us([(lambda r=r: spw.spw_spmm24(l24.hdr_r, brs[r], s24s[r], Xs[r], Ys[r], wss[r]))
+                         for r in range(R)], stream)
+        bufs = [sl.buf] + [sl.buf.clone() for _ in range(R - 1)]
+        sneed = spw.spw_spmm_workspace_bytes(sl.hdr, M)
+        swss = [torch.zeros(max(sneed, 16), dtype=torch.uint8, device=dev) for _ in range(R)]
+        us = graph_us([(lambda r=r: spw.spw_spmm(sl.hdr, bufs[r], Xs[r], Ys[r], swss[r]))
+                       for r in range(R)], stream)
+        Wd0 = W * md.to(torch.float16)
+        Wds = [Wd0] + [Wd0.clone() for _ in range(R - 1)]
+        dus = graph_us([(lambda r=r: torch.matmul(Xs[r], Wds[r].t(), out=Ys[r])) for r in range(R)],
+                       stream)
+        assert spw.spw_last_device_status() == spw.SPW_OK
+        nnz = int(mask.sum())
+        nnz_r = int(l24.hdr_r.nnz)
+        hr = l24.hdr_r
+        tp = l24.buf_r[hr.off_tileptr:hr.off_tileptr + 4 * (hr.n_strips * hr.n_ktiles + 1)]
+        tp = tp.view(torch.int32).cpu().numpy().astype(np.int64)
+        nonempty = (np.diff(tp).reshape(hr.n_strips, hr.n_ktiles) > 0)
+        pairs = nonempty.reshape(-1, 2, hr.n_ktiles).any(axis=1) if hr.n_strips % 2 == 0 else nonempty
+        out[key] = {"density": round(nnz / (N * K), 4), "residual_share": round(nnz_r / max(nnz, 1), 4),
+                    "k_steps_with_residual": round(float(pairs.mean()), 4),
+                    "us": round(us24, 2), "TFLOP/s_useful": round(2.0 * M * nnz / (us24 * 1e-6) / 1e12, 1),
+                    "dense_equivalent_tensor_frac": round(2.0 * M * N * K / (us24 * 1e-6) / 1e12 / tc_peak, 4),
+                    "spw_spmm_us": round(us, 2), "dense_cublas_us": round(dus, 2),
+                    "speedup_vs_spw_spmm": round(us / us24, 3), "speedup_vs_dense": round(dus / us24, 3)}
+        del l24, sl, s24s, brs, wss, bufs, swss, Wds, Wd0, md
+        torch.cuda.empty_cache()
+    out["how"] = ("2:4 part: two tcgen05.mma.sp (K = 32) per 64-column k-step; residual: TCB decode "
+                  "and dense MMA into the same accumulator, skipped for k-steps without residual "
+                  "weights; at most 256 tokens per tile (tensor memory also holds the metadata)")
     return out
 
 
@@ -1113,6 +1182,22 @@ def run_case(args):
             X = _dev(workloads.normal_act(args.m, K, "profile"))
             Y = torch.empty((args.m, N), dtype=torch.float16, device="cuda")
             run = lambda: lin.spmm(X, Y)  # noqa: E731
+        elif args.case == "spmm24":  # 2:4 + residual; --mask24 exact: an exact 2:4 mask
+            mask = (workloads.structured24_mask(N, K, "profile", count=2) if args.mask24 == "exact"
+                    else layer.mask)
+            l24 = spw.SparseLinear24(_dev(layer.W), _dev(mask))
+            X = _dev(workloads.normal_act(args.m, K, "profile"))
+            Y = torch.empty((args.m, N), dtype=torch.float16, device="cuda")
+            ws24 = torch.zeros(max(spw.spw_spmm24_workspace_bytes(l24.hdr_r, args.m), 16),
+                               dtype=torch.uint8, device="cuda")
+            run = lambda: l24.spmm(X, Y, ws24)  # noqa: E731
+        elif args.case == "tokens":  # per-token index sets: 4 domains, SiLU(g) * u values
+            X, _ = workloads.domain_tokens(args.m, K, 4, 0.5, "profile", silu=True)
+            Xd = _dev(X)
+            Y = torch.empty((args.m, N), dtype=torch.float16, device="cuda")
+            wst = torch.zeros(spw.spw_spmm_tokens_workspace_bytes(lin.hdr, args.m), dtype=torch.uint8,
+                              device="cuda")
+            run = lambda: lin.spmm_tokens(Xd, args.t, Y, wst)  # noqa: E731
         else:
             x, t = workloads.decode_act(args.layer, args.batch, K, args.act, "profile")
             xd = _dev(x)
@@ -1148,7 +1233,7 @@ def main():
     ap.add_argument("--sweep", choices=["decode", "prefill", "taxonomy"], default=None)
     ap.add_argument("--quick", action="store_true", help="--sweep: a few points of each sweep")
     ap.add_argument("--out", default=None, help="--sweep: also append the JSON lines to this file")
-    ap.add_argument("--case", choices=["spmv", "spmm", "tc", "ffn"], default=None)
+    ap.add_argument("--case", choices=["spmv", "spmm", "tc", "ffn", "spmm24", "tokens"], default=None)
     ap.add_argument("--layer", default="q", choices=sorted(workloads.LLAMA7B_LAYERS))
     ap.add_argument("--sparsity", type=float, default=0.5)
     ap.add_argument("--batch", type=int, default=1)
@@ -1156,7 +1241,9 @@ def main():
     ap.add_argument("--use-threshold", action="store_true",
                     help="--case spmv/tc: pass the activation threshold instead of 0")
     ap.add_argument("--m", type=int, default=2048, help="--case spmm: tokens")
-    ap.add_argument("--t", type=float, default=0.0, help="--case ffn: threshold on h")
+    ap.add_argument("--t", type=float, default=0.0, help="--case ffn: threshold on h; tokens: on X")
+    ap.add_argument("--mask24", choices=["magnitude", "exact"], default="magnitude",
+                    help="--case spmm24: the 50 %% magnitude mask or an exact 2:4 mask")
     ap.add_argument("--reps", type=int, default=10, help="--case: timed calls")
     args = ap.parse_args()
     if args.sweep:

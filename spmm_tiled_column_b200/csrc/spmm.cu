@@ -706,8 +706,19 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 break;
             }
             const uint32_t rst_s = sbase + p.off_raw + (uint32_t)rs * p.raw_stage_bytes;
-            bool dec = strip_ok;  // warp-uniform
-            if (strip_ok) {
+            // 2:4 mode: a k-tile without residual weights needs no dense W stage (the MMA
+            // warp skips its dense MMAs), so its decode is only the check that the strip's
+            // residual bitmaps are empty too; the W ring (w_full / w_empty, the stage
+            // index) advances only on k-steps with residual weights, on both sides alike.
+            const bool skip = SP24 && residual_empty(kstep(i));
+            bool dec = strip_ok && !skip;  // warp-uniform
+            if (skip && strip_ok) {
+                const uint4 bw = *(const uint4*)(smem + p.off_raw + (size_t)rs * p.raw_stage_bytes +
+                                                 512u * q + 16u * lane);
+                if (__any_sync(0xffffffffu, (bw.x | bw.y | bw.z | bw.w) != 0u) && lane == 0)
+                    raise_status(p.status, SPW_ERR_FORMAT);
+            }
+            if (dec) {
                 // columns 2l and 2l+1 of the strip: counts, starts, and the records of the
                 // warp's 8 columns (lanes 4g .. 4g+3 hold them).  Only those 8 starts are
                 // needed: the kept count of the columns before them (one reduction) plus a
@@ -750,10 +761,6 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 }
             }
             __syncwarp();
-            // 2:4 mode: a k-tile without residual weights needs no dense W stage (the MMA
-            // warp skips its dense MMAs), so the W ring (w_full / w_empty, the stage index)
-            // advances only on k-steps with residual weights, on both sides alike.
-            const bool skip = SP24 && residual_empty(kstep(i));
             if (!skip && wi >= SW &&
                 !__all_sync(0xffffffffu, wait_or_abort(smem_u32(&w_empty[ws]), wph ^ 1u, abort_flag, p.wait_limit))) {
                 abort_both();
