@@ -584,7 +584,7 @@ int orc_split24(const uint8_t* mask, int ld_mask, int N, int K, uint8_t* mask_s,
                 size_t i = (size_t)n * K + k;
                 mask_s[i] = 0;
                 mask_r[i] = 0;
-                if (!mask[(size_t)n * ld_mask + k]) continue;
+                if (mask[(size_t)n * ld_mask + k] == 0) continue; /* not kept */
                 if (taken < 2) {
                     mask_s[i] = 1;
                     taken++;
