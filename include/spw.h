@@ -394,11 +394,12 @@ int spw_spmm_tokens(const spw_format* hdr, const void* d_buf, const uint16_t* d_
  *   values at t * 4096: row r's 32 halves -- for each group of four columns, the values
  *     at its two selected positions, lower position first -- fill bytes 64 r .. 64 r +
  *     63, the 16-byte chunk c (groups 4c .. 4c+3) at position c ^ ((r >> 1) & 3);
- *   metadata at n_tiles * 4096 + t * 512: for each half j of the tile's columns, 64
- *     32-bit words; word L holds row 16 (L/16) + L%8 in bits 0-15 and that row + 8 in
- *     bits 16-31, for columns 32 j + 16 ((L/8) % 2) .. +15 as four 4-bit groups (group g
- *     at bits 4g of the half: the first selected position in bits 0-1, the second in
- *     bits 2-3, first < second).
+ *   metadata at n_tiles * 4096 + t * 1024: 16 bytes per lane L (0..63) = {word for the
+ *     tile's columns 0-31, word for columns 32-63, 0, 0}; a word holds row 16 (L/16) +
+ *     L%8 in bits 0-15 and that row + 8 in bits 16-31, for columns 32 j + 16 ((L/8) % 2)
+ *     .. +15 of its half j as four 4-bit groups (group g at bits 4g of the half: the
+ *     first selected position in bits 0-1, the second in bits 2-3, first < second);
+ *   padding at n_tiles * 5120: 1024 bytes of metadata for a tile with no kept weight.
  * A group with fewer than two kept weights selects the lowest free positions with value
  * 0; rows past N and columns past K keep nothing.  W: N x K fp16 at ldw; mask: N x K u8
  * at ld_mask.  Asynchronous.  Errors: INVALID_ARG, ALIGNMENT (d_s24), BUFFER_TOO_SMALL,

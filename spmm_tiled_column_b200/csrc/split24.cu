@@ -14,12 +14,17 @@
 //             per group of four columns, in column order) fill 64 bytes at 64 r; its four
 //             16-byte chunks (groups 4c .. 4c+3) sit at chunk position c ^ ((r >> 1) & 3)
 //             (the 64-byte swizzle of the MMA's K-major operand layout).
-//   metadata: 512 bytes per tile at n_tiles * 4096 + t * 512: for each half j of the
-//             tile's columns (32 columns = one sparse MMA), 64 words, word L (the tensor
-//             memory lane of the tile's row block) holding rows 16 (L / 16) + L % 8 (bits
-//             0-15) and that row + 8 (bits 16-31), columns 32 j + 16 ((L / 8) % 2) ..
-//             +15 as four 4-bit groups (group g at bits 4 g of its half), each group
-//             {first index, second index} in bits {0-1, 2-3}, first < second.
+//   metadata: 1024 bytes per tile at n_tiles * 4096 + t * 1024: 16 bytes per tensor
+//             memory lane L of the tile's row block (64 lanes), {word for the tile's
+//             columns 0-31, word for columns 32-63, 0, 0} -- one row of the 128 x 16-byte
+//             matrix that tcgen05.cp moves into four tensor-memory columns.  A word holds
+//             rows 16 (L / 16) + L % 8 (bits 0-15) and that row + 8 (bits 16-31), columns
+//             32 j + 16 ((L / 8) % 2) .. +15 of its half j as four 4-bit groups (group g
+//             at bits 4 g of its half), each group {first index, second index} in bits
+//             {0-1, 2-3}, first < second.
+//   padding:  1024 bytes at n_tiles * 5120: the metadata of a tile with no kept weight
+//             (every group {0, 1}), copied for the missing second strip of a weight with
+//             an odd strip count.
 // A group with fewer than two kept weights is padded with the lowest free positions and
 // zero values; rows past N and columns past K hold no kept weight.
 #include "spw_internal.cuh"
@@ -28,7 +33,7 @@ namespace spw {
 namespace {
 
 constexpr int kS24ValBytes = 4096;
-constexpr int kS24MetaBytes = 512;
+constexpr int kS24MetaBytes = 1024;
 
 __global__ void __launch_bounds__(64)
 split24_kernel(const uint16_t* __restrict__ W, int ldw, const uint8_t* __restrict__ mask,
@@ -96,9 +101,12 @@ split24_kernel(const uint16_t* __restrict__ W, int ldw, const uint8_t* __restric
             meta16[j][16 * b + 8 * k1 + i][h] = (uint16_t)((nib[j] >> (16 * k1)) & 0xffffu);
     __syncthreads();
     uint32_t* meta = (uint32_t*)(s24 + (size_t)n_tiles * kS24ValBytes + (size_t)t * kS24MetaBytes);
-#pragma unroll
-    for (int j = 0; j < 2; j++)
-        meta[64 * j + r] = (uint32_t)meta16[j][r][0] | ((uint32_t)meta16[j][r][1] << 16);
+    *(uint4*)(meta + 4 * r) = make_uint4((uint32_t)meta16[0][r][0] | ((uint32_t)meta16[0][r][1] << 16),
+                                         (uint32_t)meta16[1][r][0] | ((uint32_t)meta16[1][r][1] << 16), 0u, 0u);
+    if (t == 0) {  // the padding block after the last tile
+        uint32_t* pad = (uint32_t*)(s24 + (size_t)n_tiles * (kS24ValBytes + kS24MetaBytes));
+        *(uint4*)(pad + 4 * r) = make_uint4(0x44444444u, 0x44444444u, 0u, 0u);
+    }
 }
 
 }  // namespace
@@ -111,7 +119,7 @@ extern "C" {
 uint64_t spw_s24_bytes(int N, int K) {
     if (N < 1 || K < 1) return 0;
     const uint64_t tiles = (uint64_t)((N + 63) / 64) * (uint64_t)((K + 63) / 64);
-    return tiles * (kS24ValBytes + kS24MetaBytes);
+    return tiles * (kS24ValBytes + kS24MetaBytes) + kS24MetaBytes;  // + the padding block
 }
 
 int spw_split24(const uint16_t* d_W, int ldw, const uint8_t* d_mask, int ld_mask, int N, int K,

@@ -72,10 +72,11 @@ constexpr int kThreads = 32 * (3 + kDecoderWarps);      // X producer, MMA, deco
 constexpr uint32_t kWStageBytes = kTileRows * kBK * 2;  // 16 KB
 constexpr int kSmemLimit = 227 * 1024;
 // 2:4 mode (spw_spmm24): per k-step S area = the 2:4 values of both strips (2 x 4 KB, the
-// 64-byte-swizzled K-major layout of split24.cu) and their metadata (2 x 512 bytes), held
-// in the X stage right after the token tile.
+// 64-byte-swizzled K-major layout of split24.cu) and their metadata (2 x 1 KB: 128 lanes
+// x 16 bytes, the source matrix of one tcgen05.cp), held in the X stage right after the
+// token tile.
 constexpr uint32_t kS24ValBytes = 4096;
-constexpr uint32_t kS24MetaBytes = 512;
+constexpr uint32_t kS24MetaBytes = 1024;
 constexpr uint32_t kSStageBytes = kTileStrips * (kS24ValBytes + kS24MetaBytes);  // 9 KB
 constexpr int kMaxTokens24 = 256;  // accumulators <= 256 columns: the metadata slots fit
 
@@ -111,8 +112,8 @@ struct SpmmParams {
     uint32_t off_klist;         // dynamic smem: the visited k-tile count, then the list
     // 2:4 + residual (spw_spmm24): the structured part (split24.cu layout); the TCB
     // sections above then describe the residual.  Each X stage holds the k-step's S area
-    // at byte off_s; the metadata of X stage s sits in tensor-memory columns e_col + 2 s
-    // and e_col + 2 s + 1.
+    // at byte off_s; the MMA thread copies its metadata into tensor-memory columns
+    // e_col + 4 s .. e_col + 4 s + 3 (two used) before the stage's sparse MMAs.
     const uint8_t* s24_vals;
     const uint8_t* s24_meta;
     uint32_t off_s, e_col;
@@ -156,12 +157,18 @@ __device__ inline void umma_f16_sp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_
         : "memory");
 }
 
-// Two 32-bit columns of this warp's 32 tensor-memory lanes (one value per thread each).
-__device__ inline void tmem_st2(uint32_t taddr, uint32_t v0, uint32_t v1) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(v0), "r"(v1)
-                 : "memory");
+// Shared -> tensor memory copy of a 128-row x 16-byte matrix (row r to lane r, four
+// 32-bit columns), issued by the MMA thread: it runs in order with that thread's later
+// tcgen05.mma, so the MMAs that read the columns need no other synchronisation.  The
+// source is one K-major, unswizzled matrix: 8-row core matrices of 128 contiguous bytes.
+__device__ inline void tmem_cp_128x128b(uint32_t taddr, uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)(128 >> 4) << 16;  // between core matrices along K (one here)
+    d |= (uint64_t)(128 >> 4) << 32;  // between 8-row core matrices
+    d |= (uint64_t)1 << 46;           // descriptor version; layout type 0: no swizzle
+    asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
 }
-__device__ inline void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
     return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
@@ -394,9 +401,7 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     uint64_t* acc_full = w_empty + SW;
     uint64_t* drain = acc_full + 1;
     uint64_t* peer_ready = drain + 1;  // PAIR, on rank 0: the other CTA's stages are ready
-    const int SMF = SP24 ? SX : 0;
-    uint64_t* m_full = peer_ready + kPeerSlots;  // 2:4 mode: an X stage's metadata is in tensor memory
-    uint32_t* tmem_slot = (uint32_t*)(m_full + SMF);
+    uint32_t* tmem_slot = (uint32_t*)(peer_ready + kPeerSlots);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     volatile uint32_t* last_flag = (volatile uint32_t*)(tmem_slot + 2);
     uint32_t* tptr = (uint32_t*)(smem + p.off_tptr);
@@ -419,7 +424,6 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         mbar_init(smem_u32(acc_full), 1);
         mbar_init(smem_u32(drain), 1);
         for (int i = 0; i < kPeerSlots; i++) mbar_init(smem_u32(&peer_ready[i]), 1);
-        for (int i = 0; i < SMF; i++) mbar_init(smem_u32(&m_full[i]), 4);  // the four metadata warps
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
@@ -515,18 +519,22 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 if constexpr (SP24) {  // the token tile, then the 2:4 values and metadata
                     xbytes = p.off_s;
                     for (int j = 0; j < kTileStrips; j++)
-                        if (s0 + j < p.n_strips) xbytes += kS24ValBytes + kS24MetaBytes;
+                        xbytes += (s0 + j < p.n_strips ? kS24ValBytes : 0u) + kS24MetaBytes;
                 }
                 mbar_arrive_expect_tx(xbar, xbytes);
                 for (int h = 0; h < p.nh; h++)
                     tma_load_2d(xst + (uint32_t)(h * crows * 128), &tmap_x, kt * kBK,
                                 m0 + h * rows + (int)rank * crows, xbar);
                 if constexpr (SP24) {
+                    // a missing second strip (odd strip count) takes the padding metadata
+                    // block (valid groups, no kept weight); its values are never stored
+                    const size_t pad = (size_t)p.n_strips * nk;
                     for (int j = 0; j < kTileStrips; j++) {
-                        if (s0 + j >= p.n_strips) continue;
-                        const size_t t = (size_t)(s0 + j) * nk + kt;
-                        bulk_g2s(xst + p.off_s + kS24ValBytes * j, p.s24_vals + t * kS24ValBytes,
-                                 kS24ValBytes, xbar);
+                        const bool has = s0 + j < p.n_strips;
+                        const size_t t = has ? (size_t)(s0 + j) * nk + kt : pad;
+                        if (has)
+                            bulk_g2s(xst + p.off_s + kS24ValBytes * j, p.s24_vals + t * kS24ValBytes,
+                                     kS24ValBytes, xbar);
                         bulk_g2s(xst + p.off_s + kTileStrips * kS24ValBytes + kS24MetaBytes * j,
                                  p.s24_meta + t * kS24MetaBytes, kS24MetaBytes, xbar);
                     }
@@ -592,9 +600,6 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                                       wait_or_abort_cluster(smem_u32(&peer_ready[i % kPeerSlots]),
                                                             (uint32_t)((i / kPeerSlots) & 1), abort_flag,
                                                             p.wait_limit));
-            if constexpr (SP24)
-                ok = ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&m_full[xs]), xph, abort_flag,
-                                                                 p.wait_limit));
             if (!ok) {
                 if (lane == 0) abort_both();
                 break;
@@ -604,17 +609,19 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
                 const uint32_t xa = sbase + (uint32_t)xs * p.x_stage_bytes;
                 const uint32_t wa = sbase + p.off_w + (uint32_t)ws * kWStageBytes;
                 if constexpr (SP24) {
-                    // Two sparse MMAs (K = 32 each: 16 stored halves = 32 bytes of the S
-                    // stage's rows, 64 bytes of X's), then the residual's dense MMAs when
-                    // the k-tile holds any residual weight.
+                    // The stage's metadata into its four tensor-memory columns, then two
+                    // sparse MMAs (K = 32 each: 16 stored halves = 32 bytes of the S rows,
+                    // 64 bytes of X's; metadata column e + j of the even column e), then the
+                    // residual's dense MMAs when the k-tile holds any residual weight.
                     const uint32_t sa = xa + p.off_s;
+                    const uint32_t e = tmem + p.e_col + 4u * (uint32_t)xs;
+                    tmem_cp_128x128b(e, sa + kTileStrips * kS24ValBytes);
                     const uint32_t idesc_sp = idesc | (1u << 2);
 #pragma unroll
                     for (int j = 0; j < 2; j++) {
                         const uint64_t adesc = umma_desc_sw64(sa + 32u * j);
                         const uint64_t bdesc = umma_desc_sw128(xa + 64u * j);
-                        umma_f16_sp(tmem, adesc, bdesc, idesc_sp | (uint32_t)j,
-                                    tmem + p.e_col + 2u * (uint32_t)xs, (i > 0 || j > 0) ? 1u : 0u);
+                        umma_f16_sp(tmem, adesc, bdesc, idesc_sp | (uint32_t)j, e, (i > 0 || j > 0) ? 1u : 0u);
                     }
                 }
 #pragma unroll
@@ -801,37 +808,6 @@ spmm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             if (!skip) {
                 wi++;
                 if (++ws == SW) { ws = 0; wph ^= 1u; }
-            }
-            // 2:4 mode: decoder warps 0-3 (one per tensor-memory lane quarter) move the
-            // k-step's metadata from its X stage into that stage's two metadata columns and
-            // arrive on the stage's m_full -- after releasing the raw stage, so that the
-            // TCB ring never waits for the X stage.  The columns are free: the copy waited
-            // for here was issued only after the MMAs of the stage's previous k-step had
-            // completed.
-            if constexpr (SP24) {
-                if (d < 4) {
-                    const int xs_ = i % SX;
-                    if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&x_full[xs_]), (uint32_t)((i / SX) & 1),
-                                                               abort_flag, p.wait_limit))) {
-                        abort_both();
-                        break;
-                    }
-                    const int quarter = warp & 3;
-                    const int gl = 32 * quarter + lane;  // tensor-memory lane = row block lane
-                    const int sq = gl >> 6, L = gl & 63;
-                    uint32_t m0 = 0x44444444u, m1 = 0x44444444u;  // rows past N: {0, 1} groups
-                    if (s0 + sq < p.n_strips) {
-                        const uint32_t* mw = (const uint32_t*)(smem + (size_t)xs_ * p.x_stage_bytes + p.off_s +
-                                                               kTileStrips * kS24ValBytes + kS24MetaBytes * sq);
-                        m0 = mw[L];
-                        m1 = mw[64 + L];
-                    }
-                    tmem_st2(tmem + ((uint32_t)(32 * quarter) << 16) + p.e_col + 2u * (uint32_t)xs_, m0, m1);
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&m_full[xs_]));
-                }
             }
         }
 
@@ -1172,7 +1148,7 @@ int make_spmm_plan(const spw_format* h, int M, bool rule, SpmmPlan* pl, int sm_c
         const uint32_t off_tptr = off_rec + kRecBytesPerWarp * kDecoderWarps;
         const uint32_t off_klist = off_tptr + tptr_bytes;
         const uint32_t off_bar = (uint32_t)round_up_u64(off_klist + klist_bytes, 8);
-        const uint32_t bar_bytes = 8u * (2 * sx + 2 * sr + 2 * sw + 2 + kPeerSlots + (sp24 ? sx : 0)) + 16u;
+        const uint32_t bar_bytes = 8u * (2 * sx + 2 * sr + 2 * sw + 2 + kPeerSlots) + 16u;
         const size_t total = (size_t)off_bar + bar_bytes + 1024;  // + base alignment slack
         if (total <= (size_t)kSmemLimit) {
             pl->sx = sx;
@@ -1502,7 +1478,8 @@ int spw_spmm24(const spw_format* hdr_r, const void* d_buf_r, const void* d_s24, 
     if (!ld_ok(ldx, (int)hdr_r->K, M) || ldy < (int)hdr_r->N) return SPW_ERR_INVALID_ARG;
     if (!aligned16(d_buf_r) || !aligned16(d_s24) || !aligned16(d_X) || !aligned16(d_Y))
         return SPW_ERR_ALIGNMENT;
-    const uint64_t need = (uint64_t)hdr_r->n_strips * hdr_r->n_ktiles * (kS24ValBytes + kS24MetaBytes);
+    const uint64_t need = (uint64_t)hdr_r->n_strips * hdr_r->n_ktiles * (kS24ValBytes + kS24MetaBytes) +
+                          kS24MetaBytes;  // + the padding metadata block
     if (s24_bytes < need) return SPW_ERR_BUFFER_TOO_SMALL;
     return tc_product(hdr_r, d_buf_r, d_X, M, ldx, d_Y, ldy, 0, 0.0f, nullptr, d_ws, ws_bytes,
                       (cudaStream_t)stream, nullptr, nullptr, 0, (const uint8_t*)d_s24);

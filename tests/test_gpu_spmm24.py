@@ -28,7 +28,10 @@ def read_s24(buf: np.ndarray, N: int, K: int) -> np.ndarray:
     T = nk * ns
     S = np.zeros((ns * 64, nk * 64), np.uint16)
     vals = buf[:T * 4096].view(np.uint16).reshape(T, 64, 32)
-    meta = buf[T * 4096:T * 4608].view(np.uint32).reshape(T, 2, 64)
+    meta = buf[T * 4096:T * 5120].view(np.uint32).reshape(T, 64, 4).transpose(0, 2, 1)
+    assert not meta[:, 2:].any()
+    pad = buf[T * 5120:T * 5120 + 1024].view(np.uint32).reshape(64, 4)
+    assert (pad[:, :2] == 0x44444444).all() and not pad[:, 2:].any()
     for t in range(T):
         s, kt = divmod(t, nk)
         for r in range(64):
