@@ -161,3 +161,51 @@ def test_tensor_core_decode_and_ffn_host_validation_without_gpu(spw):
         assert L.spw_spmv_ffn(ctypes.byref(h), good, ctypes.byref(h), good, good, B, 128, 0.0,
                               good, 128, good, good, ws_n, s) == 1
     assert L.spw_spmv_ffn_workspace_bytes(ctypes.byref(h), ctypes.byref(other), 1) == 0
+
+
+def test_grouping_and_2of4_host_validation_without_gpu(spw):
+    L = spw.lib()
+    h = valid_header(spw)
+    P = ctypes.c_void_p
+    good, odd, s = P(0x10000), P(0x10008), P(0)
+    big = ctypes.c_uint64(1 << 30)
+    # token grouping: arguments, limits and alignment are checked before any launch
+    assert L.spw_group_tokens(None, 4, 128, 128, 0.0, 2, good, 128, good, good, good, big, s) == 1
+    assert L.spw_group_tokens(good, 0, 128, 128, 0.0, 2, good, 128, good, good, good, big, s) == 1
+    assert L.spw_group_tokens(good, 4, 128, 128, 0.0, 0, good, 128, good, good, good, big, s) == 1
+    assert L.spw_group_tokens(good, 4, 128, 128, -1.0, 2, good, 128, good, good, good, big, s) == 1
+    assert L.spw_group_tokens(good, 4, 128, 128, 0.0, 2, good, 130, good, good, good, big, s) == 1
+    assert L.spw_group_tokens(good, 4, 128, 100, 0.0, 2, good, 128, good, good, good, big, s) == 1
+    assert L.spw_group_tokens(good, 4, 16385, 16392, 0.0, 2, good, 16392, good, good, good, big, s) == 5
+    assert L.spw_group_tokens(good, 16385, 128, 128, 0.0, 2, good, 128, good, good, good, big, s) == 5
+    assert L.spw_group_tokens(good, 4, 128, 128, 0.0, 2, good, 128, odd, good, good, big, s) == 2
+    assert L.spw_group_tokens(good, 4, 128, 128, 0.0, 2, good, 128, good, good, good,
+                              ctypes.c_uint64(16), s) == 3
+    assert L.spw_group_tokens_workspace_bytes(4, 128) > 0
+    assert L.spw_group_tokens_workspace_bytes(4, 16385) == 0
+    # grouped prefill
+    ws = ctypes.c_uint64(1 << 30)
+    assert L.spw_spmm_tokens(ctypes.byref(h), good, good, 0, 128, 0.0, good, 128, good, ws, s) == 0
+    assert L.spw_spmm_tokens(ctypes.byref(h), None, good, 4, 128, 0.0, good, 128, good, ws, s) == 1
+    assert L.spw_spmm_tokens(ctypes.byref(h), good, good, 4, 128, 0.0, good, 128, None, ws, s) == 1
+    for t in (-1.0, float("nan"), float("inf")):
+        assert L.spw_spmm_tokens(ctypes.byref(h), good, good, 4, 128, t, good, 128, good, ws, s) == 1
+    assert L.spw_spmm_tokens(ctypes.byref(h), good, good, 4, 132, 0.0, good, 128, good, ws, s) == 1
+    assert L.spw_spmm_tokens(ctypes.byref(h), good, odd, 4, 128, 0.0, good, 128, good, ws, s) == 2
+    assert L.spw_spmm_tokens(ctypes.byref(h), good, good, 16385, 128, 0.0, good, 128, good, ws, s) == 5
+    # 2:4 split and prefill
+    assert L.spw_s24_bytes(128, 128) == 4 * 5120 + 1024
+    assert L.spw_split24(None, 128, good, 128, 128, 128, good, big, good, 128, s) == 1
+    assert L.spw_split24(good, 100, good, 128, 128, 128, good, big, good, 128, s) == 1
+    assert L.spw_split24(good, 128, good, 128, 128, 128, odd, big, good, 128, s) == 2
+    assert L.spw_split24(good, 128, good, 128, 128, 128, good, ctypes.c_uint64(100), good, 128, s) == 3
+    n24 = ctypes.c_uint64(4 * 5120 + 1024)
+    assert L.spw_spmm24(ctypes.byref(h), good, good, n24, good, 0, 128, good, 128, None, 0, s) == 0
+    assert L.spw_spmm24(ctypes.byref(h), good, None, n24, good, 4, 128, good, 128, None, 0, s) == 1
+    assert L.spw_spmm24(ctypes.byref(h), good, odd, n24, good, 4, 128, good, 128, None, 0, s) == 2
+    assert L.spw_spmm24(ctypes.byref(h), good, good, ctypes.c_uint64(4 * 5120), good, 4, 128, good, 128,
+                        None, 0, s) == 3
+    assert L.spw_spmm24(ctypes.byref(h), good, good, n24, good, 4, 132, good, 128, None, 0, s) == 1
+    bad = valid_header(spw)
+    bad.magic = 0
+    assert L.spw_spmm24(ctypes.byref(bad), good, good, n24, good, 4, 128, good, 128, None, 0, s) == 4

@@ -129,3 +129,33 @@ def test_plan_errors():
         with pytest.raises(spw.SpwError) as e:
             spw.spw_spmm_plan(h, 64, 0)
         assert e.value.status == spw.SPW_ERR_CUDA
+
+
+@pytest.mark.parametrize("sms", [8, 148])
+@pytest.mark.parametrize("N,K", [(128, 64), (1000, 512), (4096, 4096), (4096, 11008), (300, 100)])
+@pytest.mark.parametrize("M", [1, 16, 100, 512, 2048, 5000])
+def test_2of4_and_token_plans(N, K, M, sms, monkeypatch):
+    monkeypatch.setenv("SPW_SPMM_PAIR", "1")  # neither product uses SM-pair tiles
+    h = header(N, K)
+    p24 = spw.spw_spmm24_plan(h, M, sms)
+    assert p24["cta_pair"] == 0 and p24["weight_tiles"] == -(-N // 128)
+    # tensor memory holds the accumulators and the metadata columns: <= 256 tokens
+    mt = p24["token_tile"]
+    assert mt % 16 == 0 and 16 <= mt <= 256 and mt * p24["token_tiles"] >= M
+    tiles = p24["token_tiles"] * p24["weight_tiles"]
+    assert p24["ctas"] == p24["whole_tiles"] + (tiles - p24["whole_tiles"]) * p24["k_parts"]
+    pt = spw.spw_spmm_tokens_plan(h, M, sms)
+    assert pt["cta_pair"] == 0 and pt["token_tile"] <= 512
+    # the grouped input, permutation, tile signatures and grouping scratch follow the
+    # product's own workspace
+    words = ((K + 63) // 64 + 63) // 64
+    assert pt["workspace_bytes"] >= 2 * M * (-(-K // 8) * 8) + 4 * M + 8 * words * pt["token_tiles"]
+
+
+def test_token_plan_limits():
+    with pytest.raises(spw.SpwError) as e:
+        spw.spw_spmm_tokens_plan(header(256, 16448), 64, 148)
+    assert e.value.status == spw.SPW_ERR_UNSUPPORTED
+    with pytest.raises(spw.SpwError) as e:
+        spw.spw_spmm_tokens_plan(header(256, 256), 16385, 148)
+    assert e.value.status == spw.SPW_ERR_UNSUPPORTED
