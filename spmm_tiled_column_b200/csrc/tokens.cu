@@ -23,6 +23,7 @@ namespace spw {
 namespace {
 
 constexpr int kSigThreads = 256;
+constexpr int kRowChunks = 8;     // 16-byte chunks per thread: 256 x 8 x 8 halves = 16384 columns
 constexpr int kRankTokens = 128;  // tokens per rank block (one per thread)
 constexpr int kRankKeys = 64;     // keys per rank block, staged in shared memory
 
@@ -31,9 +32,10 @@ __device__ inline bool keeps_pair(uint32_t w, float t) {
     return passes_threshold((uint16_t)(w & 0xffffu), t) || passes_threshold((uint16_t)(w >> 16), t);
 }
 
-// One CTA per token: 8 columns per thread and step (a 16-byte load), a warp covers 32
-// such chunks = 4 k-tiles, whose flags come out of one ballot.  Block 0 also clears the
-// tile signatures; every block clears its token's rank counter.
+// One CTA per token: a thread's 16-byte chunks (8 columns each) are all loaded before any
+// is tested, so the row is in flight at once; a warp's 32 consecutive chunks = 4 k-tiles,
+// whose flags come out of one ballot.  Block 0 also clears the tile signatures; every
+// block clears its token's rank counter.
 __global__ void __launch_bounds__(kSigThreads)
 token_sig_kernel(const uint16_t* __restrict__ X, int ldx, int K, float t, int words,
                  uint64_t* __restrict__ sig, uint32_t* __restrict__ rank,
@@ -47,18 +49,23 @@ token_sig_kernel(const uint16_t* __restrict__ X, int ldx, int K, float t, int wo
         for (int i = threadIdx.x; i < tile_words; i += kSigThreads) tile_sig[i] = 0ull;
     __syncthreads();
     const uint16_t* row = X + (size_t)m * ldx;
-    const int chunks = (K + 7) / 8;
-    for (int base = 32 * warp; base < chunks; base += kSigThreads) {
+    const int chunks = (K + 7) / 8;  // <= kSigThreads * kRowChunks
+    uint4 v[kRowChunks];
+#pragma unroll
+    for (int u = 0; u < kRowChunks; u++) {
+        const int c = 32 * warp + kSigThreads * u + lane;
+        v[u] = (8 * c + 8 <= K) ? __ldg((const uint4*)(row + 8 * c)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kRowChunks; u++) {
+        const int base = 32 * warp + kSigThreads * u;  // the warp's first chunk this round
+        if (base >= chunks) break;                       // warp-uniform
         const int c = base + lane;
         bool any = false;
-        if (c < chunks) {
-            const int k0 = 8 * c;
-            if (k0 + 8 <= K) {
-                const uint4 v = __ldg((const uint4*)(row + k0));
-                any = keeps_pair(v.x, t) || keeps_pair(v.y, t) || keeps_pair(v.z, t) || keeps_pair(v.w, t);
-            } else {
-                for (int k = k0; k < K; k++) any = any || passes_threshold(__ldg(row + k), t);
-            }
+        if (8 * c + 8 <= K) {
+            any = keeps_pair(v[u].x, t) || keeps_pair(v[u].y, t) || keeps_pair(v[u].z, t) || keeps_pair(v[u].w, t);
+        } else {
+            for (int k = 8 * c; k < K; k++) any = any || passes_threshold(__ldg(row + k), t);
         }
         const uint32_t b = __ballot_sync(0xffffffffu, any);
         if (lane < 4 && ((b >> (8 * lane)) & 0xffu) != 0u) {
@@ -114,19 +121,26 @@ token_gather_kernel(const uint16_t* __restrict__ X, int ldx, int K, float t, int
                  (unsigned long long)__ldg(sig + (size_t)i * words + threadIdx.x));
     const uint16_t* src = X + (size_t)i * ldx;
     uint16_t* dst = Xg + (size_t)r * ldg;
-    for (int c = threadIdx.x; 8 * c < ldg; c += kSigThreads) {
-        const int k0 = 8 * c;
-        uint32_t v[4] = {0u, 0u, 0u, 0u};
+    // all of this thread's chunks loaded first (the row in flight at once), then stored
+    uint4 q[kRowChunks];
+#pragma unroll
+    for (int u = 0; u < kRowChunks; u++) {
+        const int k0 = 8 * (threadIdx.x + kSigThreads * u);
+        q[u] = make_uint4(0u, 0u, 0u, 0u);
         if (k0 + 8 <= K) {
-            const uint4 q = __ldg((const uint4*)(src + k0));
-            v[0] = q.x;
-            v[1] = q.y;
-            v[2] = q.z;
-            v[3] = q.w;
-        } else {
+            q[u] = __ldg((const uint4*)(src + k0));
+        } else if (k0 < K) {
+            uint32_t w4[4] = {0u, 0u, 0u, 0u};
             for (int e = 0; e < 8 && k0 + e < K; e++)
-                v[e >> 1] |= (uint32_t)__ldg(src + k0 + e) << (16 * (e & 1));
+                w4[e >> 1] |= (uint32_t)__ldg(src + k0 + e) << (16 * (e & 1));
+            q[u] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
+    }
+#pragma unroll
+    for (int u = 0; u < kRowChunks; u++) {
+        const int k0 = 8 * (threadIdx.x + kSigThreads * u);
+        if (k0 >= ldg) break;
+        uint32_t v[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
 #pragma unroll
         for (int e = 0; e < 4; e++) {
             const uint16_t lo = (uint16_t)(v[e] & 0xffffu), hi = (uint16_t)(v[e] >> 16);
