@@ -66,6 +66,16 @@ def test_dense_mask_matches_dense_product():
     assert oracle.rel_err(Y, ref) <= TOL
 
 
+def test_all_ones_mask_matches_cublas():
+    N, K, M = 1024, 2048, 512
+    W = workloads.weight(N, K, "gspmm-cublas")
+    X = workloads.normal_act(M, K, "gspmm-cublas")
+    Y, _ = run(W, np.ones((N, K), np.uint8), X)
+    torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction = False
+    ref = host(torch.matmul(dev(X), dev(W).t())).astype(np.float64)
+    assert oracle.rel_err(Y, ref) <= TOL
+
+
 def test_dropped_weights_never_read():
     N, K, M = 256, 512, 128
     W = workloads.weight(N, K, "gspmm-drop")

@@ -175,12 +175,36 @@ def test_llama13b_full_size_b1(shape, s):
     assert oracle.rel_err(y, ref) <= TOL
 
 
+@pytest.mark.parametrize("shape", [(5120, 5120), (13824, 5120), (5120, 13824)])
+@pytest.mark.parametrize("B", [4, 16])
+def test_llama13b_full_size_batched(shape, B):
+    # the Llama-13B shapes at the batch sizes of the decode sweep, half the entries zeroed
+    N, K = shape
+    layer = workloads.pruned_layer("13b", N, K, 0.5, "cfg4-batched")
+    x, _ = workloads.decode_act("down" if K > N else "q", B, K, 0.5, "cfg4-batched")
+    y, _ = run(layer.W, layer.mask, x)
+    assert oracle.rel_err(y, oracle.spmv(layer.W, layer.mask, x)) <= TOL
+
+
+def test_all_ones_mask_matches_cublas():
+    # every weight kept: the decode equals the dense product cuBLAS computes (fp32
+    # accumulation, no fp16 reduced-precision reductions)
+    N, K, B = 1024, 2048, 16
+    W = workloads.weight(N, K, "ones-cublas")
+    x = workloads.normal_act(B, K, "ones-cublas")
+    y, _ = run(W, np.ones((N, K), np.uint8), x)
+    torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction = False
+    ref = host(torch.matmul(dev(x), dev(W).t())).astype(np.float64)
+    assert oracle.rel_err(y, ref) <= TOL
+    assert oracle.rel_err(y, oracle.spmv(W, np.ones((N, K), np.uint8), x)) <= TOL
+
+
 @pytest.mark.parametrize("N,K,B,a,t,use_bits", [
     (4096, 11008, 1, 0.5, 0.0, False), (4096, 11008, 1, 0.5, 0.3, False),
     (1000, 3000, 4, 0.3, 0.2, False), (300, 200, 16, 0.7, 0.1, False),
     (4096, 4096, 1, 0.0, 0.0, False), (513, 1000, 2, 0.5, 0.0, True),
     (11008, 4096, 8, 0.5, 0.25, True)])
-def test_column_fetch_equals_whole_tiles(N, K, B, a, t, use_bits, monkeypatch):
+def test_column_fetch_equals_whole_tiles(N, K, B, a, t, use_bits):
     # Column fetch (only the active columns' bytes are copied) and whole-tile copies share
     # the work split and the summation order, so they give the same bits; both match the
     # oracle.  spw_set_column_fetch(2) forces column fetch, 0 whole tiles.
