@@ -395,24 +395,25 @@ def run_ours(args, rank, world, local_rank):
 
     # per-linear kernel timing (dominant kernel = spw_spmv) for the roofline, on the
     # launching stream, over graph replays of single linears
-    def time_graphs(make_call, reps=50):
-        gs = []
-        for r in range(N_ROTATE):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
+    def time_graphs(make_call, reps=48):
+        # one graph chains the call over all rotated copies (kernels back to back, as in
+        # the step graph and in the plain-copy and cuBLAS timings); us per call
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for r in range(N_ROTATE):
                 make_call(r)
-            gs.append(g)
+        n_rep = max(1, reps // N_ROTATE)
         with torch.cuda.stream(stream):
-            for i in range(8):
-                gs[i % N_ROTATE].replay()
+            for _ in range(2):
+                g.replay()
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            for i in range(reps):
-                gs[i % N_ROTATE].replay()
+            for _ in range(n_rep):
+                g.replay()
             b.record(stream)
         stream.synchronize()
-        return a.elapsed_time(b) * 1e3 / reps
+        return a.elapsed_time(b) * 1e3 / (n_rep * N_ROTATE)
 
     # each grouped launch on its own, and each linear as a single-layer launch
     per_group = {}
@@ -524,18 +525,10 @@ def run_ours(args, rank, world, local_rank):
         N, K = workloads.LLAMA7B_LAYERS[name]
         Ws = [torch.randn((N, K), device=dev, dtype=torch.float16) * 0.02 for _ in range(6)]
         xd = torch.randn((1, K), device=dev, dtype=torch.float16)
-        reps = 60
-        with torch.cuda.stream(stream):
-            for i in range(6):
-                torch.nn.functional.linear(xd, Ws[i % 6])
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for i in range(reps):
-                torch.nn.functional.linear(xd, Ws[i % 6])
-            b.record(stream)
-        stream.synchronize()
-        us = a.elapsed_time(b) * 1e3 / reps
+        outs = [torch.empty((1, N), device=dev, dtype=torch.float16) for _ in range(6)]
+        # the same chained-graph timing as the sparse launches: six rotated weights (> L2)
+        us = graph_us([(lambda i=i: torch.matmul(xd, Ws[i].t(), out=outs[i])) for i in range(6)],
+                      stream)
         dense[name] = {"us": round(us, 3), "GB/s": round(2 * N * K / (us * 1e-6) / 1e9, 1),
                        "sparse_us": per_linear[name]["us"],
                        "speedup": round(us / per_linear[name]["us"], 3)}
