@@ -1,6 +1,8 @@
 // spmm.cu -- products on tcgen05 tensor cores with the compressed weight as the A operand:
 //   prefill  Y = X . W_masked^T            (spw_spmm, M tokens)
 //   decode   y_b = W_masked . x~_b         (spw_spmv_tc, B <= 16 rows, threshold rule)
+//   prefill with per-token index sets      (spw_spmm_tokens: token-list mode)
+//   prefill on the 2:4 + residual split    (spw_spmm24: 2:4 mode)
 //
 // Method: "Unified Static-Dynamic Pruning for Efficient LLM Inference" (abstract) pairs
 // its bitmap format with a Tensor-Core SpMM for prefill.  Dense tensor cores take only
@@ -45,6 +47,17 @@
 //   * Every mbarrier wait is bounded and also polls a CTA-wide abort flag; on a timeout
 //     the kernel raises SPW_ERR_TIMEOUT, drains outstanding copies and MMAs (bounded),
 //     frees TMEM and returns.
+//   * Token-list mode ("Reduced Matrix Multiplication" §6.1): X holds the grouped rows
+//     (tokens.cu); warp 2 turns the token tile's k-tile signature into an ascending list
+//     in shared memory, every role walks that list instead of 0 .. n_ktiles-1, a tile
+//     with an empty list writes zeros, and the epilogue writes row r to row perm[r].
+//   * 2:4 mode ("Accelerating LLM GPU inference ..." §1, layers (i) and (iii)): each X
+//     stage also carries the k-step's 2:4 values (64-byte swizzle) and metadata
+//     (split24.cu layout); the MMA thread moves the metadata into tensor memory with
+//     tcgen05.cp and issues two tcgen05.mma.sp (K = 32), then the dense MMAs of the
+//     decoded residual tile only when the k-tile holds residual weights (the W ring
+//     advances on those k-steps only); token tiles <= 256 (accumulators + metadata).
+//   * SM-pair mode (opt-in, SPW_SPMM_PAIR=1): see the kernel's comment.
 // A decoded tile holds explicit zeros where the mask drops a weight, so a non-finite
 // activation reaches every row through the MMA (0 * Inf = NaN, as in a dense product);
 // the CUDA-core decode (spmv.cu) skips dropped weights instead.
