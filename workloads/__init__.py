@@ -174,16 +174,22 @@ def domain_tokens(M: int, K: int, n_domains: int, block_density: float, *seed_pa
     return x.astype(np.float16), dom
 
 
-def structured24_mask(N: int, K: int, *seed_parts, extra: float = 0.0) -> np.ndarray:
+def structured24_mask(N: int, K: int, *seed_parts, extra: float = 0.0,
+                      count: int | None = None, dense_channels: float = 0.0) -> np.ndarray:
     """A 2:4-structured mask: in every group of four columns of a row, 0, 1 or 2 kept
-    positions (uniform count, seeded random positions); with extra > 0, each dropped
-    position is then kept with that probability as well (weights outside the 2:4
-    pattern, the residual of a 2:4 + residual split)."""
-    r = rng("mask24", N, K, extra, *seed_parts)
+    positions (uniform count; exactly `count` when given; seeded random positions).
+    Then, outside the 2:4 pattern: each dropped position is kept with probability
+    `extra`, and a seeded `dense_channels` fraction of the input channels (columns) is
+    kept whole -- outlier features left unpruned -- so that the residual of a 2:4 +
+    residual split sits in those columns."""
+    r = rng("mask24", N, K, extra, count, dense_channels, *seed_parts)
     G = -(-K // 4)
-    cnt = r.integers(0, 3, size=(N, G, 1))
+    cnt = (r.integers(0, 3, size=(N, G, 1)) if count is None
+           else np.full((N, G, 1), int(count)))
     rank = np.argsort(np.argsort(r.random((N, G, 4)), axis=2), axis=2)
     keep = (rank < cnt).reshape(N, 4 * G)[:, :K]
     if extra > 0:
         keep |= r.random((N, K)) < extra
+    if dense_channels > 0:
+        keep[:, r.permutation(K)[:max(1, int(round(dense_channels * K)))]] = True
     return keep.astype(np.uint8)
