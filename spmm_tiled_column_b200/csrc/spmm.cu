@@ -269,17 +269,17 @@ __device__ inline void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t 
         : "memory");
 }
 
-// Arrive on the barrier at this offset in both CTAs of the pair once the MMAs issued so
-// far have completed.
-__device__ inline void umma_commit_pair_both(uint32_t bar) {
-    asm volatile(
-        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(bar)
-        : "memory");
-}
+// Arrive on the barrier at this shared-memory address (this CTA's, or the other CTA's
+// through its cluster address) once the MMAs issued so far have completed.
 __device__ inline void umma_commit_pair_local(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
+}
+// The same barrier in both CTAs of the pair (issued by rank 0): two commits, one to each
+// CTA's copy of the barrier, both completing with the same MMAs.
+__device__ inline void umma_commit_pair_both(uint32_t bar) {
+    umma_commit_pair_local(bar);
+    umma_commit_pair_local(map_to_rank(bar, 1u));
 }
 
 __device__ inline void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
