@@ -1201,6 +1201,8 @@ def run_case(args):
                                  dtype=torch.uint8, device="cuda")
                 run = lambda: spw.spw_spmv_tc(lin.hdr, lin.buf, xd, thr, None, y, ws)  # noqa: E731
             else:
+                if args.fetch:  # decode copies only the active columns' 16-byte chunks
+                    spw.spw_set_column_fetch(2)
                 run = lambda: lin.spmv(xd, thr, None, y)  # noqa: E731
     for _ in range(args.warmup):
         run()
@@ -1235,6 +1237,8 @@ def main():
                     help="--case spmv/tc: pass the activation threshold instead of 0")
     ap.add_argument("--m", type=int, default=2048, help="--case spmm: tokens")
     ap.add_argument("--t", type=float, default=0.0, help="--case ffn: threshold on h; tokens: on X")
+    ap.add_argument("--fetch", action="store_true",
+                    help="--case spmv: active-column fetch (spw_set_column_fetch(2))")
     ap.add_argument("--mask24", choices=["magnitude", "exact"], default="magnitude",
                     help="--case spmm24: the 50 %% magnitude mask or an exact 2:4 mask")
     ap.add_argument("--reps", type=int, default=10, help="--case: timed calls")
