@@ -419,8 +419,10 @@ int spw_spmm24_plan(const spw_format* hdr_r, int M, int sm_count, spw_spmm_plan_
  * instruction, metadata in tensor memory) and R (hdr_r / d_buf_r, a TCB v1 buffer of the
  * residual) is decoded in shared memory and runs as dense MMA into the same fp32
  * accumulator; a k-tile whose residual tiles are empty costs no decode and no dense MMA.
- * X, Y, M, ldx, ldy, workspace, determinism and errors as spw_spmm; d_s24 must hold
- * spw_s24_bytes(N, K) bytes (BUFFER_TOO_SMALL otherwise) and be 16-byte aligned. */
+ * X, Y, M, ldx, ldy, workspace, determinism and errors as spw_spmm; d_s24 must be the
+ * buffer spw_split24 wrote for the same weight and mask (same N and K as hdr_r; only its
+ * size, spw_s24_bytes(N, K) bytes, can be checked: BUFFER_TOO_SMALL otherwise) and be
+ * 16-byte aligned. */
 int spw_spmm24(const spw_format* hdr_r, const void* d_buf_r, const void* d_s24, uint64_t s24_bytes,
                const uint16_t* d_X, int M, int ldx, uint16_t* d_Y, int ldy, void* d_ws,
                uint64_t ws_bytes, void* stream);
