@@ -444,6 +444,24 @@ int spw_spmv_tc(const spw_format* hdr, const void* d_buf, const uint16_t* d_x, i
                 float threshold, const uint32_t* d_act_bits, uint16_t* d_y, int ldy, void* d_ws,
                 uint64_t ws_bytes, void* stream);
 
+/* Decode with the path chosen by batch size ([SPDP] abstract: "hybrid" decoding, read as
+ * a runtime choice between the decode paths): spw_spmv_tc for batches of
+ * spw_spmv_auto_path(B) == 1, spw_spmv otherwise, with the same arguments.  The tensor-core
+ * path is taken from the batch where it measured faster on every Llama-7B shape at 50 %
+ * sparsity (14 rows); the choice depends on B alone, is made on the host and costs no
+ * device read.  The result is that of the path taken: what spw_spmv computes,
+ * deterministic, except that on the tensor-core path a non-finite x~ entry reaches every
+ * row (see spw_spmv_tc).
+ *   spw_spmv_auto_path(B): 0 (CUDA cores), 1 (tensor cores), -1 for B outside 1..16.
+ *   spw_spmv_auto_workspace_bytes(hdr, B): the workspace of the path taken, with that
+ *   path's counter rules (zero before the first call, left zero); 0 for B outside 1..16.
+ * Asynchronous.  Errors: those of the path taken; INVALID_ARG for B outside 1..16. */
+int spw_spmv_auto_path(int B);
+uint64_t spw_spmv_auto_workspace_bytes(const spw_format* hdr, int B);
+int spw_spmv_auto(const spw_format* hdr, const void* d_buf, const uint16_t* d_x, int B, int ldx,
+                  float threshold, const uint32_t* d_act_bits, uint16_t* d_y, int ldy, void* d_ws,
+                  uint64_t ws_bytes, void* stream);
+
 /* Synchronise `stream`, then read and clear the library's device status word for the
  * current device: *code = SPW_OK, SPW_ERR_TIMEOUT if a bounded device wait ran out, or
  * SPW_ERR_FORMAT if a product kernel met a tile that disagrees with its header (see

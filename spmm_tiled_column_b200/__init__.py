@@ -76,6 +76,9 @@ SIGNATURES = {
     "spw_spmm": ([_FP, _P, _P, _I, _I, _P, _I, _P, _U64, _P], _I),
     "spw_spmv_tc_workspace_bytes": ([_FP, _I], _U64),
     "spw_spmv_tc": ([_FP, _P, _P, _I, _I, _F, _P, _P, _I, _P, _U64, _P], _I),
+    "spw_spmv_auto_path": ([_I], _I),
+    "spw_spmv_auto_workspace_bytes": ([_FP, _I], _U64),
+    "spw_spmv_auto": ([_FP, _P, _P, _I, _I, _F, _P, _P, _I, _P, _U64, _P], _I),
     "spw_last_device_status": ([_P, _P], _I),
     "spw_spmv_group_workspace_bytes": ([_I, _FP, _I], _U64),
     "spw_spmv_group": ([_I, _FP, _P, _P, _P, _P, _P, _P, _I, _F, _P, _U64, _P], _I),
@@ -519,6 +522,42 @@ def spw_spmv_tc(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.0,
     return y
 
 
+def spw_spmv_auto_path(B: int) -> int:
+    """0 when spw_spmv_auto takes the CUDA-core decode for batch B, 1 for the tensor-core
+    decode, -1 for B outside 1..16."""
+    return int(lib().spw_spmv_auto_path(int(B)))
+
+
+def spw_spmv_auto_workspace_bytes(hdr, B: int) -> int:
+    h = _hdr(hdr)
+    return int(lib().spw_spmv_auto_workspace_bytes(ctypes.byref(h), int(B)))
+
+
+def spw_spmv_auto(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.0,
+                  act_bits: torch.Tensor | None = None, y: torch.Tensor | None = None,
+                  ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decode y (B x N fp16) on the path chosen by batch size; arguments as spw_spmv.  ws:
+    a zero-initialised uint8 workspace of spw_spmv_auto_workspace_bytes(hdr, B) bytes
+    (allocated here when needed and not given)."""
+    h = _hdr(hdr)
+    x2, ldx = _rows(_half(x, "x"), "x")
+    B = x2.shape[0]
+    if y is None:
+        y = torch.empty((B, h.N), dtype=torch.float16, device=x.device)
+    y2, ldy = _rows(_half(y, "y"), "y")
+    _need_buf(buf, h)
+    _need(x2, B, h.K, "x")
+    _need(y2, B, h.N, "y")
+    _need_words(act_bits, h.K)
+    need = spw_spmv_auto_workspace_bytes(h, B)
+    if ws is None and need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=x.device)
+    _check("spw_spmv_auto", lib().spw_spmv_auto(
+        ctypes.byref(h), _ptr(buf), _ptr(x2), B, ldx, float(threshold), _ptr(act_bits),
+        _ptr(y2), ldy, _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return y
+
+
 def spw_spmv_ffn_workspace_bytes(hdr_gate, hdr_up, B: int) -> int:
     return int(lib().spw_spmv_ffn_workspace_bytes(ctypes.byref(_hdr(hdr_gate)),
                                                   ctypes.byref(_hdr(hdr_up)), B))
@@ -702,6 +741,15 @@ class SparseLinear:
         x2 = x if x.dim() == 2 else x.unsqueeze(0)
         return spw_spmv(self.hdr, self.buf, x2, threshold, act_bits, y,
                         self.workspace(x2.shape[0]), stream)
+
+    def spmv_auto(self, x, threshold=0.0, act_bits=None, y=None, stream=None):
+        x2 = x if x.dim() == 2 else x.unsqueeze(0)
+        B = x2.shape[0]
+        if ("auto", B) not in self._ws:
+            self._ws[("auto", B)] = torch.zeros(max(spw_spmv_auto_workspace_bytes(self.hdr, B), 16),
+                                                dtype=torch.uint8, device=self.buf.device)
+        return spw_spmv_auto(self.hdr, self.buf, x2, threshold, act_bits, y,
+                             self._ws[("auto", B)], stream)
 
     def spmm(self, X, Y=None, stream=None):
         return spw_spmm(self.hdr, self.buf, X, Y, stream=stream)

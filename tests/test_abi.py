@@ -209,3 +209,31 @@ def test_grouping_and_2of4_host_validation_without_gpu(spw):
     bad = valid_header(spw)
     bad.magic = 0
     assert L.spw_spmm24(ctypes.byref(bad), good, good, n24, good, 4, 128, good, 128, None, 0, s) == 4
+
+
+def test_auto_decode_path_choice_without_gpu(spw):
+    # The choice depends on the batch alone: the CUDA-core decode below the boundary, the
+    # tensor-core decode from it up to 16 rows; argument errors of the path taken come back
+    # before any device call.
+    L = spw.lib()
+    h = valid_header(spw)
+    P = ctypes.c_void_p
+    good, odd, s = P(0x10000), P(0x10008), P(0)
+    ws_n = ctypes.c_uint64(1 << 20)
+    paths = [L.spw_spmv_auto_path(B) for B in range(1, 17)]
+    assert set(paths) <= {0, 1} and paths[0] == 0 and paths[-1] == 1
+    first_tc = paths.index(1)
+    assert all(p == 1 for p in paths[first_tc:])  # one boundary, monotone in B
+    for B in (0, 17, -3):
+        assert L.spw_spmv_auto_path(B) == -1
+        assert L.spw_spmv_auto_workspace_bytes(ctypes.byref(h), B) == 0
+        assert L.spw_spmv_auto(ctypes.byref(h), good, good, B, 128, 0.0, None, good, 128, good, ws_n, s) == 1
+    for B in (1, first_tc + 1, 16):
+        assert L.spw_spmv_auto(None, good, good, B, 128, 0.0, None, good, 128, good, ws_n, s) == 1
+        assert L.spw_spmv_auto(ctypes.byref(h), good, good, B, 128, float("nan"), None, good, 128,
+                               good, ws_n, s) == 1
+        assert L.spw_spmv_auto(ctypes.byref(h), good, odd, B, 128, 0.0, None, good, 128, good, ws_n, s) == 2
+    bad = valid_header(spw)
+    bad.magic = 0
+    assert L.spw_spmv_auto(ctypes.byref(bad), good, good, 16, 128, 0.0, None, good, 128, good, ws_n, s) == 4
+    assert spw.spw_spmv_auto_path(16) == 1 and spw.spw_spmv_auto_path(0) == -1
