@@ -435,8 +435,9 @@ uint64_t spw_spmv_tc_workspace_bytes(const spw_format* hdr, int B);
  * [RMM] §4.2 reduced product): computes what spw_spmv computes -- same arguments, the
  * threshold rule and column set applied to x in shared memory -- with the decoded weight
  * tiles as the A operand of tcgen05 MMA (M = 128 weight rows, N = B rounded up to 16).
- * Worth it for wide batches (B >= 8), where spw_spmv's per-row multiply-adds grow with
- * B.  As in spw_spmm, a non-finite x~ entry reaches every row, including rows whose weight
+ * Its time hardly changes with B, while spw_spmv's per-row multiply-adds grow with B:
+ * measured faster than spw_spmv from 14 rows on the Llama-7B shapes (from 8 on the
+ * 4096 x 4096 one); spw_spmv_auto makes that choice.  As in spw_spmm, a non-finite x~ entry reaches every row, including rows whose weight
  * in that column is dropped.  Workspace: spw_spmv_tc_workspace_bytes (zero-initialised
  * counters, left zero).  Inactive columns are decoded but contribute zeros.  Deterministic.
  * Asynchronous.  Errors: as spw_spmv. */
