@@ -34,8 +34,10 @@
  *     status code and launches nothing.  No call aborts, traps or prints.
  *   - Alignment: every device pointer must be 16-byte aligned (d_count and d_idx: 4).
  *     Leading dimensions only need to cover a row, except where a call copies rows
- *     with 16-byte bulk or tensor copies: spw_spmv's ldx and spw_spmm's ldx must be
- *     multiples of 8 fp16 elements unless that operand has a single row.  Such copies
+ *     with 16-byte bulk or tensor copies: the ldx of every decode and prefill call
+ *     (spw_spmv and its group, FFN, no-alloc, tensor-core and auto forms; spw_spmm,
+ *     spw_spmm_tokens, spw_spmm24, spw_group_tokens) must be a multiple of 8 fp16
+ *     elements unless that operand has a single row.  Such copies
  *     may read an activation row up to the next 16-byte boundary past its last
  *     element (never across it, so never outside the row's allocation granule).
  *   - Buffer contents: the header is checked on the host.  The product kernels check each
