@@ -113,6 +113,26 @@ MUTANTS = [
     ("split_three_structured", "if (taken < 2) {", "if (taken < 3) {", [SPLIT_PINS]),
     ("split_groups_of_two", "for (int k = g; k < g + 4 && k < K; k++) {",
      "for (int k = g; k < g + 4 && k < K; k++) { if (k == g + 2) taken = 0;", [SPLIT_PINS]),
+    ("topk_keeps_one_more", "for (int i = 0; i < k; i++) act_bits",
+     "for (int i = 0; i < k + (k < K); i++) act_bits", [SELECT_PINS]),
+    ("topk_nonfinite_lowest", "cols[c].score = finite ? s : INFINITY;",
+     "cols[c].score = finite ? s : -1.0;", [SELECT_PINS]),
+    ("tileptr_shifted", "put_u32(buf + g.off_tileptr + 4 * t, (uint32_t)unit);",
+     "put_u32(buf + g.off_tileptr + 4 * t, (uint32_t)(unit + (t > 0)));", [FORMAT_PINS]),
+    ("spmm_rows_ignored",
+     "int m = rows ? rows[i] : i;\n        if (m < 0 || m >= M) return ORC_ERR_ARG;\n"
+     "        for (int n = 0; n < N; n++) {\n            double acc = 0.0;\n"
+     "            for (int k = 0; k < K; k++)\n",
+     "int m = i;\n        if (m < 0 || m >= M) return ORC_ERR_ARG;\n"
+     "        for (int n = 0; n < N; n++) {\n            double acc = 0.0;\n"
+     "            for (int k = 0; k < K; k++)\n", [PRODUCT_PINS]),
+    ("tokens_rows_ignored",
+     "int m = rows ? rows[i] : i;\n        if (m < 0 || m >= M) return ORC_ERR_ARG;\n"
+     "        for (int n = 0; n < N; n++) {\n            double acc = 0.0;\n"
+     "            for (int k = 0; k < K; k++) {\n",
+     "int m = i;\n        if (m < 0 || m >= M) return ORC_ERR_ARG;\n"
+     "        for (int n = 0; n < N; n++) {\n            double acc = 0.0;\n"
+     "            for (int k = 0; k < K; k++) {\n", [TOKEN_PINS]),
     ("split_last_two_structured", "if (taken < 2) {",
      "if (taken < 2 && !(k == g && mask[(size_t)n * ld_mask + k + (k + 1 < K)])) {", [SPLIT_PINS]),
 ]
