@@ -177,9 +177,36 @@ def _need_buf(buf: torch.Tensor, h, name: str = "buf"):
                          f"header says {h.bytes_total}")
 
 
+def _nbytes(t: torch.Tensor | None, name: str = "ws") -> int:
+    """Bytes of a raw buffer handed to the library with its size (0 for None); the
+    library writes through its pointer on the device, so it must be a CUDA tensor."""
+    if t is None:
+        return 0
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    return t.numel() * t.element_size()
+
+
 def _need_words(a: torch.Tensor | None, n: int, name: str = "act_bits"):
-    if a is not None and a.numel() * a.element_size() < 4 * ((n + 31) // 32):
+    """A column-set or output bit array of ceil(n / 32) 32-bit words, on the GPU."""
+    if a is not None and _nbytes(a, name) < 4 * ((n + 31) // 32):
         raise ValueError(f"{name} needs at least {(n + 31) // 32} 32-bit words")
+
+
+def _need_u32(a: torch.Tensor, n: int, name: str):
+    """An output array of n 32-bit entries, on the GPU."""
+    if _nbytes(a, name) < 4 * n:
+        raise ValueError(f"{name} needs at least {n} 32-bit entries")
+
+
+def _mask_like(mask: torch.Tensor, N: int, K: int) -> tuple[torch.Tensor, int]:
+    """An N x K uint8 CUDA mask with unit column stride, and its leading dimension."""
+    m, ld = _rows(mask, "mask")
+    if m.dtype != torch.uint8 or not m.is_cuda:
+        raise TypeError("mask must be a CUDA uint8 tensor")
+    if tuple(m.shape) != (N, K):
+        raise ValueError(f"mask is {tuple(m.shape)}; the weight is {N} x {K}")
+    return m, ld
 
 
 def _hdr(h) -> spw_format:
@@ -231,23 +258,21 @@ def spw_compress(W: torch.Tensor, mask: torch.Tensor, buf: torch.Tensor | None =
                  stream=None) -> tuple[torch.Tensor, spw_format]:
     """Compress W * mask into a TCB v1 buffer; returns (uint8 device buffer, header)."""
     W, ldw = _rows(_half(W, "W"), "W")
-    mask, ldm = _rows(mask, "mask")
     N, K = W.shape
-    if tuple(mask.shape) != (N, K) or mask.dtype != torch.uint8:
-        raise ValueError("mask must be uint8 with W's shape")
+    mask, ldm = _mask_like(mask, N, K)
     if buf is None:
         nbytes, _ = spw_format_query(mask, stream)
         buf = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
     hdr = spw_format()
     _check("spw_compress", lib().spw_compress(
-        _ptr(W), ldw, _ptr(mask), ldm, N, K, _ptr(buf), buf.numel(), ctypes.byref(hdr),
+        _ptr(W), ldw, _ptr(mask), ldm, N, K, _ptr(buf), _nbytes(buf, "buf"), ctypes.byref(hdr),
         _stream(stream)))
     return buf, hdr
 
 
 def spw_format_read(buf: torch.Tensor, stream=None) -> spw_format:
     hdr = spw_format()
-    _check("spw_format_read", lib().spw_format_read(_ptr(buf), buf.numel(), ctypes.byref(hdr),
+    _check("spw_format_read", lib().spw_format_read(_ptr(buf), _nbytes(buf, "buf"), ctypes.byref(hdr),
                                                     _stream(stream)))
     return hdr
 
@@ -281,6 +306,8 @@ def spw_select_threshold(x: torch.Tensor, t: float, act_bits: torch.Tensor | Non
         act_bits = torch.empty(_act_words(K) + 3, dtype=torch.int32, device=x.device)
     if count is None:
         count = torch.empty(1, dtype=torch.int32, device=x.device)
+    _need_words(act_bits, K)
+    _need_u32(count, 1, "count")
     _check("spw_select_threshold", lib().spw_select_threshold(
         _ptr(x), B, K, ldx, float(t), _ptr(act_bits), _ptr(count), _stream(stream)))
     return act_bits, count
@@ -295,6 +322,8 @@ def spw_select_topk(x: torch.Tensor, k: int, act_bits: torch.Tensor | None = Non
         act_bits = torch.empty(_act_words(K) + 3, dtype=torch.int32, device=x.device)
     if idx is None:
         idx = torch.empty(max(int(k), 1), dtype=torch.int32, device=x.device)
+    _need_words(act_bits, K)
+    _need_u32(idx, int(k), "idx")
     _check("spw_select_topk", lib().spw_select_topk(
         _ptr(x), B, K, ldx, int(k), _ptr(act_bits), _ptr(idx), _stream(stream)))
     return act_bits, idx[:k]
@@ -329,7 +358,7 @@ def spw_spmv(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.0,
                          device=x.device)
     _check("spw_spmv", lib().spw_spmv(
         ctypes.byref(h), _ptr(buf), _ptr(x2), B, ldx, float(threshold), _ptr(act_bits),
-        _ptr(y2), ldy, _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(y2), ldy, _ptr(ws), _nbytes(ws), _stream(stream)))
     return y
 
 
@@ -370,7 +399,7 @@ def spw_spmv_group(hdrs, bufs, xs, threshold: float = 0.0, act_bits=None, ys=Non
     _check("spw_spmv_group", lib().spw_spmv_group(
         n, harr, P(*[b.data_ptr() for b in bufs]), P(*[t.data_ptr() for t, _ in x2]),
         I(*[ld for _, ld in x2]), ab, P(*[t.data_ptr() for t, _ in y2]), I(*[ld for _, ld in y2]),
-        B, float(threshold), _ptr(ws), ws.numel(), _stream(stream)))
+        B, float(threshold), _ptr(ws), _nbytes(ws), _stream(stream)))
     return ys
 
 
@@ -419,7 +448,7 @@ def spw_spmm(hdr, buf: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = N
         ws = torch.zeros(need, dtype=torch.uint8, device=X.device)
     _check("spw_spmm", lib().spw_spmm(
         ctypes.byref(h), _ptr(buf), _ptr(X2), M, ldx, _ptr(Y2), ldy, _ptr(ws),
-        0 if ws is None else ws.numel(), _stream(stream)))
+        _nbytes(ws), _stream(stream)))
     return Y
 
 
@@ -451,7 +480,7 @@ def spw_group_tokens(X: torch.Tensor, t: float, token_tile: int, ws: torch.Tenso
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=X.device)
     _check("spw_group_tokens", lib().spw_group_tokens(
         _ptr(X2), M, K, ldx, ctypes.c_float(t), int(token_tile), _ptr(Xg), ldg, _ptr(perm),
-        _ptr(tsig), _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(tsig), _ptr(ws), _nbytes(ws), _stream(stream)))
     return Xg, perm, tsig
 
 
@@ -488,7 +517,7 @@ def spw_spmm_tokens(hdr, buf: torch.Tensor, X: torch.Tensor, threshold: float,
                          device=X.device)
     _check("spw_spmm_tokens", lib().spw_spmm_tokens(
         ctypes.byref(h), _ptr(buf), _ptr(X2), M, ldx, ctypes.c_float(threshold), _ptr(Y2), ldy,
-        _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(ws), _nbytes(ws), _stream(stream)))
     return Y
 
 
@@ -518,7 +547,7 @@ def spw_spmv_tc(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.0,
         ws = torch.zeros(need, dtype=torch.uint8, device=x.device)
     _check("spw_spmv_tc", lib().spw_spmv_tc(
         ctypes.byref(h), _ptr(buf), _ptr(x2), B, ldx, float(threshold), _ptr(act_bits),
-        _ptr(y2), ldy, _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+        _ptr(y2), ldy, _ptr(ws), _nbytes(ws), _stream(stream)))
     return y
 
 
@@ -554,7 +583,7 @@ def spw_spmv_auto(hdr, buf: torch.Tensor, x: torch.Tensor, threshold: float = 0.
         ws = torch.zeros(need, dtype=torch.uint8, device=x.device)
     _check("spw_spmv_auto", lib().spw_spmv_auto(
         ctypes.byref(h), _ptr(buf), _ptr(x2), B, ldx, float(threshold), _ptr(act_bits),
-        _ptr(y2), ldy, _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+        _ptr(y2), ldy, _ptr(ws), _nbytes(ws), _stream(stream)))
     return y
 
 
@@ -589,7 +618,7 @@ def spw_spmv_ffn(hdr_gate, buf_gate: torch.Tensor, hdr_up, buf_up: torch.Tensor,
         ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=x.device)
     _check("spw_spmv_ffn", lib().spw_spmv_ffn(
         ctypes.byref(hg), _ptr(buf_gate), ctypes.byref(hu), _ptr(buf_up), _ptr(x2), B, ldx,
-        float(threshold), _ptr(h2), ldh, _ptr(act_bits), _ptr(ws), ws.numel(), _stream(stream)))
+        float(threshold), _ptr(h2), ldh, _ptr(act_bits), _ptr(ws), _nbytes(ws), _stream(stream)))
     return h, act_bits
 
 
@@ -654,7 +683,7 @@ class DecodeGroup:
             ab = self._pab
         _check("spw_spmv_group", lib().spw_spmv_group(
             self.n, self._harr, self._pbufs, self._px, self._ldx, ab, self._py, self._ldy,
-            self.B, float(threshold), _ptr(self.ws), self.ws.numel(), _stream(stream)))
+            self.B, float(threshold), _ptr(self.ws), _nbytes(self.ws), _stream(stream)))
         return ys
 
 
@@ -666,13 +695,11 @@ def spw_split24(W: torch.Tensor, mask: torch.Tensor, stream=None) -> tuple[torch
     """2:4 + residual split: (s24 uint8 buffer of the 2:4 part, residual mask uint8 N x K);
     see spw_split24 in include/spw.h."""
     W2, ldw = _rows(_half(W, "W"), "W")
-    m2, ldm = _rows(mask, "mask")
-    if m2.dtype != torch.uint8:
-        raise ValueError("mask must be uint8")
     N, K = W2.shape
+    m2, ldm = _mask_like(mask, N, K)
     s24 = torch.empty(spw_s24_bytes(N, K), dtype=torch.uint8, device=W.device)
     mask_r = torch.empty((N, K), dtype=torch.uint8, device=W.device)
-    _check("spw_split24", lib().spw_split24(_ptr(W2), ldw, _ptr(m2), ldm, N, K, _ptr(s24), s24.numel(),
+    _check("spw_split24", lib().spw_split24(_ptr(W2), ldw, _ptr(m2), ldm, N, K, _ptr(s24), _nbytes(s24, "s24"),
                                             _ptr(mask_r), K, _stream(stream)))
     return s24, mask_r
 
@@ -704,8 +731,8 @@ def spw_spmm24(hdr_r, buf_r: torch.Tensor, s24: torch.Tensor, X: torch.Tensor,
     if ws is None and need:
         ws = torch.zeros(need, dtype=torch.uint8, device=X.device)
     _check("spw_spmm24", lib().spw_spmm24(
-        ctypes.byref(h), _ptr(buf_r), _ptr(s24), s24.numel(), _ptr(X2), M, ldx, _ptr(Y2), ldy,
-        _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+        ctypes.byref(h), _ptr(buf_r), _ptr(s24), _nbytes(s24, "s24"), _ptr(X2), M, ldx, _ptr(Y2), ldy,
+        _ptr(ws), _nbytes(ws), _stream(stream)))
     return Y
 
 

@@ -237,3 +237,46 @@ def test_auto_decode_path_choice_without_gpu(spw):
     bad.magic = 0
     assert L.spw_spmv_auto(ctypes.byref(bad), good, good, 16, 128, 0.0, None, good, 128, good, ws_n, s) == 4
     assert spw.spw_spmv_auto_path(16) == 1 and spw.spw_spmv_auto_path(0) == -1
+
+
+class _FakeDeviceTensor:
+    """Stands in for a CUDA tensor in the size checks (they read only these three)."""
+    is_cuda = True
+
+    def __init__(self, n, element_size=4):
+        self.n, self.es = n, element_size
+
+    def numel(self):
+        return self.n
+
+    def element_size(self):
+        return self.es
+
+
+def test_binding_refuses_host_tensors_and_short_buffers_without_gpu(spw):
+    # The library writes through raw pointers and cannot see tensor sizes or devices, so
+    # the binding refuses host tensors and short output / workspace buffers before any
+    # library call.
+    import torch
+    host_x = torch.zeros((2, 64), dtype=torch.float16)
+    with pytest.raises(ValueError):
+        spw.spw_select_threshold(host_x, 0.0)
+    with pytest.raises(ValueError):
+        spw.spw_compress(host_x, torch.ones((2, 64), dtype=torch.uint8))
+    with pytest.raises(ValueError):
+        spw._nbytes(torch.zeros(16, dtype=torch.uint8), "ws")
+    with pytest.raises(ValueError):
+        spw._need_words(torch.zeros(4, dtype=torch.int32), 64)
+    with pytest.raises(TypeError):
+        spw._mask_like(torch.zeros((2, 64), dtype=torch.uint8), 2, 64)
+    F = _FakeDeviceTensor
+    assert spw._nbytes(None) == 0 and spw._nbytes(F(10, 2)) == 20
+    spw._need_words(F(2), 64)
+    with pytest.raises(ValueError):
+        spw._need_words(F(1), 64)
+    spw._need_words(F(3), 65)
+    with pytest.raises(ValueError):
+        spw._need_words(F(5, 1), 33)  # 5 bytes hold one word, two are needed
+    spw._need_u32(F(4), 4, "idx")
+    with pytest.raises(ValueError):
+        spw._need_u32(F(3), 4, "idx")
