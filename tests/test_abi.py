@@ -280,3 +280,15 @@ def test_binding_refuses_host_tensors_and_short_buffers_without_gpu(spw):
     spw._need_u32(F(4), 4, "idx")
     with pytest.raises(ValueError):
         spw._need_u32(F(3), 4, "idx")
+
+
+def test_header_compiles_as_plain_c_and_cpp(tmp_path):
+    # the boundary is a C ABI: the header must stand alone in C11 and C++17, warning-free
+    src = tmp_path / "use_spw.c"
+    src.write_text('#include "spw.h"\nint main(void) { return spw_version() > 0 ? 0 : 1; }\n')
+    import subprocess
+    inc = os.path.join(ROOT, "include")
+    for cmd in (["gcc", "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror"],
+                ["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-x", "c++"]):
+        proc = subprocess.run(cmd + ["-fsyntax-only", "-I", inc, str(src)], capture_output=True, text=True)
+        assert proc.returncode == 0, proc.stderr
