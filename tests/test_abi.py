@@ -292,3 +292,30 @@ def test_header_compiles_as_plain_c_and_cpp(tmp_path):
                 ["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-x", "c++"]):
         proc = subprocess.run(cmd + ["-fsyntax-only", "-I", inc, str(src)], capture_output=True, text=True)
         assert proc.returncode == 0, proc.stderr
+
+
+def test_plain_c_program_links_and_calls_the_library(spw, tmp_path):
+    # a C caller (no Python, no torch) links libspw.so and calls host-side entry points
+    import subprocess
+    src = tmp_path / "caller.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "spw.h"
+int main(void) {
+    if (spw_version() != 100) return 1;
+    if (strcmp(spw_status_string(SPW_OK), "SPW_OK") != 0) return 2;
+    if (spw_spmv_auto_path(16) != 1 || spw_spmv_auto_path(1) != 0 || spw_spmv_auto_path(0) != -1) return 3;
+    if (spw_s24_bytes(128, 128) != 4 * 5120 + 1024) return 4;
+    if (spw_spmv(NULL, NULL, NULL, 1, 128, 0.0f, NULL, NULL, 128, NULL, 0, NULL) != SPW_ERR_INVALID_ARG)
+        return 5;
+    puts("ok");
+    return 0;
+}
+''')
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(spw_build.LIB)
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-L", libdir,
+                    "-l:libspw.so", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    proc = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert proc.returncode == 0 and proc.stdout.strip() == "ok", (proc.returncode, proc.stderr)
