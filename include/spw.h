@@ -80,7 +80,7 @@ typedef enum {
     SPW_ERR_ALIGNMENT = 2,        /* pointer or leading dimension breaks the 16-B rule   */
     SPW_ERR_BUFFER_TOO_SMALL = 3, /* format buffer or workspace smaller than required    */
     SPW_ERR_FORMAT = 4,           /* header magic/version/geometry does not match TCB v1 */
-    SPW_ERR_UNSUPPORTED = 5,      /* valid request this build does not handle            */
+    SPW_ERR_UNSUPPORTED = 5,      /* valid request the library does not handle           */
     SPW_ERR_CUDA = 6,             /* a CUDA runtime call failed (launch, copy, device)   */
     SPW_ERR_TIMEOUT = 7           /* a bounded device-side wait ran out (see below)      */
 } spw_status;
